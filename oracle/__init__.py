@@ -1,0 +1,15 @@
+"""Float64 CPU oracle (test infrastructure only; see la_oracle.py)."""
+
+from .la_oracle import (  # noqa: F401
+    FEATURE_MAPS,
+    brute_force,
+    brute_force_head,
+    brute_force_rows,
+    feature_map,
+    forward,
+    linear_causal_head,
+    linear_noncausal_head,
+    phi_elu1,
+    phi_relu,
+    rows,
+)

@@ -1,0 +1,212 @@
+"""Float64 CPU oracle for linear-time kernelised ("phi") attention.
+
+TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT. Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this module. The CUDA library never calls it and shares no code with it.
+
+What it computes (page "NNT Define Linear Attention", sections "The inputs" and
+"How it works"): a non-negative feature map phi is applied to queries and keys;
+the similarity of query i and key j is phi(q_i).phi(k_j); every output row is
+the similarity-weighted sum of value rows, divided by the sum of the weights
+plus ``eps``.  The page's "How it works" section states the fast form that
+groups the product as phi(Q) (phi(K)^T V) and normalises by
+1 / (phi(Q) . sum_j phi(k_j) + eps); the definition below is the ungrouped
+weighted sum, and the grouped form is implemented separately so that each can
+be checked against the other.
+
+Readings of the pages taken here (each one is listed in the design doc):
+  * elu is the standard ELU with alpha = 1, so elu(x)+1 is x+1 for x > 0 and
+    exp(x) for x <= 0 (page "NNT Define Linear Attention", "The inputs").
+  * eps is added once per query row to the summed weights (same page, "How it
+    works": normalise by 1 / (Q . sum(K) + eps)).
+  * causal means each query sees keys j <= i, itself included (same page,
+    "The inputs": tokens attend only to earlier tokens; the diagonal is kept so
+    that row 0 is defined).
+  * no 1/sqrt(D) temperature is applied (the page names none).
+  * the optional projection (page "Flux2TTRTrainer", "Inputs worth setting":
+    feature_dim is a multiple of 256) is one D x F matrix per head, shared by
+    queries and keys, applied before the feature map: phi(x) = fmap(x W_h).
+
+Everything is float64 with numpy; ``@`` (a library matmul) is the only
+primitive used beyond elementwise numpy.  Arrays are [B, H, N, D] with the
+feature axis last; W is [H, D, F] (one matrix per head) or [D, F] (shared).
+"""
+
+import numpy as np
+
+FEATURE_MAPS = ("elu", "relu")
+
+
+# --------------------------------------------------------------------------
+# Feature maps (page "NNT Define Linear Attention", "The inputs": feature_map
+# is elu, mapped as elu(x)+1, or relu; both are non-negative).
+# --------------------------------------------------------------------------
+
+def phi_elu1(x):
+    """elu(x) + 1 with alpha = 1: x + 1 where x > 0, exp(x) where x <= 0."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x > 0.0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def phi_relu(x):
+    """relu(x) = max(x, 0)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.maximum(x, 0.0)
+
+
+def feature_map(x, fmap, W=None):
+    """phi(x) for rows x[..., D].
+
+    With ``W`` (D x F) the map is fmap(x W) (the projected-feature form, page
+    "Flux2TTRTrainer", "Inputs worth setting"); without it, fmap acts on x
+    directly and F = D.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if W is not None:
+        x = x @ np.asarray(W, dtype=np.float64)
+    if fmap == "elu":
+        return phi_elu1(x)
+    if fmap == "relu":
+        return phi_relu(x)
+    raise ValueError(f"unknown feature map {fmap!r}")
+
+
+def _head_W(W, h):
+    if W is None:
+        return None
+    W = np.asarray(W, dtype=np.float64)
+    return W if W.ndim == 2 else W[h]
+
+
+# --------------------------------------------------------------------------
+# The definition: explicit weights, O(N^2) per head.
+# --------------------------------------------------------------------------
+
+def brute_force_head(q, k, v, fmap, eps, causal, W=None):
+    """One head by the definition.
+
+    out_i = sum_j w_ij v_j / (sum_j w_ij + eps),  w_ij = phi(q_i) . phi(k_j),
+    with j over all keys (non-causal) or over j <= i (causal).
+    q, k: [N, D]; v: [N, Dv]. Returns [N, Dv] float64.
+    """
+    pq = feature_map(q, fmap, W)
+    pk = feature_map(k, fmap, W)
+    v = np.asarray(v, dtype=np.float64)
+    w = pq @ pk.T                      # w[i, j] = phi(q_i) . phi(k_j)
+    if causal:
+        w = np.tril(w)                 # keep j <= i
+    num = w @ v
+    den = w.sum(axis=1) + eps
+    return num / den[:, None]
+
+
+def brute_force_rows(q, k, v, rows, fmap, eps, causal, W=None):
+    """Selected query rows of one head by the definition, one row at a time.
+
+    Costs O(len(rows) * N * (F + D)); used to check single outputs of large
+    problems.  Returns [len(rows), Dv] float64.
+    """
+    pk = feature_map(k, fmap, W)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty((len(rows), v.shape[1]), dtype=np.float64)
+    for r, i in enumerate(rows):
+        pqi = feature_map(q[i:i + 1], fmap, W)[0]
+        jend = i + 1 if causal else pk.shape[0]
+        w = pk[:jend] @ pqi            # w_j = phi(q_i) . phi(k_j)
+        out[r] = (w @ v[:jend]) / (w.sum() + eps)
+    return out
+
+
+# --------------------------------------------------------------------------
+# The grouped (linear-time) forms the method uses.
+# --------------------------------------------------------------------------
+
+def linear_noncausal_head(q, k, v, fmap, eps, W=None):
+    """Grouped form of page "NNT Define Linear Attention", "How it works".
+
+    kv = phi(K)^T V (F x Dv), ksum = sum_j phi(k_j) (F),
+    out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).
+    """
+    pq = feature_map(q, fmap, W)
+    pk = feature_map(k, fmap, W)
+    v = np.asarray(v, dtype=np.float64)
+    kv = pk.T @ v
+    ksum = pk.sum(axis=0)
+    num = pq @ kv
+    den = pq @ ksum + eps
+    return num / den[:, None]
+
+
+def linear_causal_head(q, k, v, fmap, eps, W=None):
+    """Causal grouped form as a token-by-token recurrence.
+
+    The state S = sum_{j<=i} phi(k_j) v_j^T and z = sum_{j<=i} phi(k_j) are
+    updated with token i first, then row i is read out from them, so query i
+    sees keys 0..i (the inclusive reading of "earlier tokens").
+    """
+    pq = feature_map(q, fmap, W)
+    pk = feature_map(k, fmap, W)
+    v = np.asarray(v, dtype=np.float64)
+    n, f = pk.shape
+    S = np.zeros((f, v.shape[1]), dtype=np.float64)
+    z = np.zeros(f, dtype=np.float64)
+    out = np.empty((n, v.shape[1]), dtype=np.float64)
+    for i in range(n):
+        S += np.outer(pk[i], v[i])
+        z += pk[i]
+        out[i] = (pq[i] @ S) / (pq[i] @ z + eps)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Whole [B, H, N, D] problems.
+# --------------------------------------------------------------------------
+
+def _check(q, k, v, fmap, eps):
+    if fmap not in FEATURE_MAPS:
+        raise ValueError(f"unknown feature map {fmap!r}")
+    if eps < 0:
+        raise ValueError("eps must be >= 0")
+    if q.ndim != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k, v must be [B, H, N, D] with matching B, H, N")
+
+
+def forward(q, k, v, fmap="elu", eps=1e-6, causal=False, W=None):
+    """Grouped form over all heads; returns float64 [B, H, N, Dv]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    _check(q, k, v, fmap, eps)
+    B, H, N, _ = q.shape
+    out = np.empty(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            Wh = _head_W(W, h)
+            if causal:
+                out[b, h] = linear_causal_head(q[b, h], k[b, h], v[b, h], fmap, eps, Wh)
+            else:
+                out[b, h] = linear_noncausal_head(q[b, h], k[b, h], v[b, h], fmap, eps, Wh)
+    return out
+
+
+def brute_force(q, k, v, fmap="elu", eps=1e-6, causal=False, W=None):
+    """The definition over all heads; returns float64 [B, H, N, Dv]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    _check(q, k, v, fmap, eps)
+    B, H, N, _ = q.shape
+    out = np.empty(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            out[b, h] = brute_force_head(q[b, h], k[b, h], v[b, h], fmap, eps, causal,
+                                         _head_W(W, h))
+    return out
+
+
+def rows(q, k, v, b, h, idx, fmap="elu", eps=1e-6, causal=False, W=None):
+    """Rows ``idx`` of head (b, h) by the definition; float64 [len(idx), Dv]."""
+    return brute_force_rows(np.asarray(q[b, h], dtype=np.float64),
+                            np.asarray(k[b, h], dtype=np.float64),
+                            np.asarray(v[b, h], dtype=np.float64),
+                            list(idx), fmap, eps, causal, _head_W(W, h))

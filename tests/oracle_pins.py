@@ -1,0 +1,333 @@
+"""Pins that tie the float64 oracle to facts fixed outside the oracle itself.
+
+Each pin takes an oracle namespace ``ora`` (the real ``oracle.la_oracle`` or a
+copy with a planted mistake) and raises AssertionError when ``ora`` disagrees
+with a hand-derived worked example, a closed form, an invariant of the method
+or a library routine.  The definition they check is the one on page "NNT Define
+Linear Attention" ("The inputs", "How it works"):
+
+    out_i = sum_j w_ij v_j / (sum_j w_ij + eps),   w_ij = phi(q_i) . phi(k_j)
+
+with j <= i for the causal variant, phi = elu(x)+1 or relu, optionally after a
+per-head D x F projection (page "Flux2TTRTrainer", "Inputs worth setting").
+"""
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- fixtures --
+
+def load_golden(name):
+    """Parse a tests/golden text fixture into float64 arrays."""
+    sections = {}
+    cur = None
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for raw in fh:
+            line = raw.split("#", 1)[0].strip()
+            if not line:
+                continue
+            parts = line.split()
+            if parts[0] in ("fmap", "eps"):
+                sections[parts[0]] = parts[1]
+                cur = None
+            elif len(parts) == 1 and not _is_number(parts[0]):
+                cur = parts[0]
+                sections[cur] = []
+            else:
+                sections[cur].append([float(Fraction(p)) for p in parts])
+    out = {"fmap": sections["fmap"], "eps": float(Fraction(sections["eps"]))}
+    for key in ("q", "k", "v", "W", "out_noncausal", "out_causal"):
+        if key in sections:
+            out[key] = np.array(sections[key], dtype=np.float64)
+    return out
+
+
+def _is_number(tok):
+    try:
+        Fraction(tok)
+        return True
+    except ValueError:
+        return False
+
+
+def _as4(x):
+    return np.asarray(x, dtype=np.float64)[None, None]
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, rtol=1e-12, atol=1e-13):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    assert np.all(np.isfinite(a)), "non-finite values"
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    scale = max(np.max(np.abs(b)) if b.size else 0.0, 1.0)
+    assert err <= atol + rtol * scale, f"max |diff| = {err:.3e}"
+
+
+# -------------------------------------------------------------------- pins --
+
+def pin_feature_maps(ora):
+    """phi values fixed by the definitions of elu(x)+1 and relu."""
+    x = np.array([-3.0, -1.0, -0.25, 0.0, 0.5, 2.0], dtype=np.float64)
+    expect_elu = np.array([math.exp(-3.0), math.exp(-1.0), math.exp(-0.25), 1.0, 1.5, 3.0])
+    _close(ora.phi_elu1(x), expect_elu, rtol=1e-15, atol=0)
+    _close(ora.feature_map(x[None], "elu")[0], expect_elu, rtol=1e-15, atol=0)
+    _close(ora.phi_relu(x), np.array([0, 0, 0, 0, 0.5, 2.0]), rtol=0, atol=0)
+    _close(ora.feature_map(x[None], "relu")[0], np.array([0, 0, 0, 0, 0.5, 2.0]), rtol=0, atol=0)
+
+
+def pin_feature_map_vs_torch(ora):
+    """elu(x)+1 against the library ELU (alpha = 1) on a wide range."""
+    import torch
+    x = np.linspace(-30.0, 30.0, 2001)
+    ref = torch.nn.functional.elu(torch.from_numpy(x), alpha=1.0).numpy() + 1.0
+    _close(ora.phi_elu1(x), ref, rtol=1e-14, atol=1e-300)
+    ref_relu = torch.relu(torch.from_numpy(x)).numpy()
+    _close(ora.phi_relu(x), ref_relu, rtol=0, atol=0)
+
+
+def pin_golden(ora):
+    """Hand-derived worked examples (tests/golden/*.txt), every oracle entry."""
+    for name in ("tiny_elu_rational.txt", "tiny_relu_rational.txt",
+                 "tiny_projected_rational.txt"):
+        g = load_golden(name)
+        q, k, v, W = _as4(g["q"]), _as4(g["k"]), _as4(g["v"]), g.get("W")
+        Wf = None if W is None else W[None]  # [H=1, D, F]
+        for causal, key in ((False, "out_noncausal"), (True, "out_causal")):
+            exp = g[key]
+            _close(ora.forward(q, k, v, g["fmap"], g["eps"], causal, Wf)[0, 0], exp,
+                   rtol=1e-14, atol=1e-15)
+            _close(ora.brute_force(q, k, v, g["fmap"], g["eps"], causal, Wf)[0, 0], exp,
+                   rtol=1e-14, atol=1e-15)
+            _close(ora.rows(q, k, v, 0, 0, range(exp.shape[0]), g["fmap"], g["eps"],
+                            causal, Wf), exp, rtol=1e-14, atol=1e-15)
+
+
+def pin_negative_elu_closed_form(ora):
+    """One query, keys on both elu branches, worked out with math.exp.
+
+    q = [-1], k = [1, -2], v = [3, 5]:  phi(q) = e^-1, phi(k) = [2, e^-2],
+    out = (3*2 + 5 e^-2) e^-1 / ((2 + e^-2) e^-1 + eps).
+    """
+    eps = 1e-3
+    q = _as4([[-1.0], [-1.0]])
+    k = _as4([[1.0], [-2.0]])
+    v = _as4([[3.0], [5.0]])
+    e1, e2 = math.exp(-1.0), math.exp(-2.0)
+    full = (6.0 + 5.0 * e2) * e1 / ((2.0 + e2) * e1 + eps)
+    first = 6.0 * e1 / (2.0 * e1 + eps)
+    for f in (ora.forward, ora.brute_force):
+        _close(f(q, k, v, "elu", eps, False)[0, 0, :, 0], [full, full], rtol=1e-14)
+        _close(f(q, k, v, "elu", eps, True)[0, 0, :, 0], [first, full], rtol=1e-14)
+
+
+def pin_constant_values(ora):
+    """v_j = c for all j gives out_i = c * s_i / (s_i + eps) (s_i: row weight sum)."""
+    rng = _rng(11)
+    B, H, N, D = 1, 2, 37, 8
+    q = rng.standard_normal((B, H, N, D))
+    k = rng.standard_normal((B, H, N, D))
+    c = rng.standard_normal(D)
+    v = np.broadcast_to(c, (B, H, N, D)).copy()
+    for fmap in ("elu", "relu"):
+        for causal in (False, True):
+            for f in (ora.forward, ora.brute_force):
+                o0 = f(q, k, v, fmap, 0.0, causal)
+                _close(o0, v, rtol=1e-12, atol=1e-12)     # eps = 0: exactly c
+            # eps > 0: every row is c scaled by the same factor in (0, 1]
+            o = ora.forward(q, k, v, fmap, 0.5, causal)
+            ratio = o / c
+            assert np.all(ratio <= 1.0 + 1e-12) and np.all(ratio > 0.0)
+            _close(ratio, np.repeat(ratio[..., :1], D, axis=-1), rtol=1e-12)
+
+
+def pin_zero_qk_closed_form(ora):
+    """Q = K = 0 under elu+1: phi = 1, every weight is D.
+
+    Non-causal out_i = mean_j v_j * N D / (N D + eps);
+    causal    out_i = mean_{j<=i} v_j * (i+1) D / ((i+1) D + eps).
+    """
+    rng = _rng(12)
+    B, H, N, D = 1, 1, 23, 5
+    z = np.zeros((B, H, N, D))
+    v = rng.standard_normal((B, H, N, 3))
+    eps = 0.75
+    mean = v[0, 0].mean(axis=0)
+    exp_nc = np.tile(mean * (N * D) / (N * D + eps), (N, 1))
+    cnt = np.arange(1, N + 1)[:, None]
+    exp_c = np.cumsum(v[0, 0], axis=0) / cnt * (cnt * D) / (cnt * D + eps)
+    for f in (ora.forward, ora.brute_force):
+        _close(f(z, z, v, "elu", eps, False)[0, 0], exp_nc, rtol=1e-13)
+        _close(f(z, z, v, "elu", eps, True)[0, 0], exp_c, rtol=1e-13)
+
+
+def pin_identity_values_give_weights(ora):
+    """With N <= Dv and V = I, row i of the output is the normalised weight row.
+
+    Weights are non-negative; each row sums to s_i / (s_i + eps) <= 1; entries
+    are proportional to phi(q_i).phi(k_j) computed here by explicit loops.
+    """
+    rng = _rng(13)
+    N, D = 9, 6
+    q = rng.standard_normal((1, 1, N, D))
+    k = rng.standard_normal((1, 1, N, D))
+    v = np.eye(N)[None, None]
+    for fmap in ("elu", "relu"):
+        for causal in (False, True):
+            for f in (ora.forward, ora.brute_force):
+                w = f(q, k, v, fmap, 1e-6, causal)[0, 0]
+                assert np.all(w >= -1e-15)
+                assert np.all(w.sum(axis=1) <= 1.0 + 1e-12)
+                if fmap == "elu":     # elu+1 > 0: rows sum to 1 up to eps
+                    _close(w.sum(axis=1), np.ones(N), rtol=0, atol=1e-5)
+                if causal:
+                    assert np.all(np.triu(w, 1) == 0.0)
+                # proportionality to explicit dot products of the feature map
+                for i in range(N):
+                    pq = [(x + 1.0 if x > 0 else math.exp(x)) if fmap == "elu" else max(x, 0.0)
+                          for x in q[0, 0, i]]
+                    raw = []
+                    for j in range(N):
+                        pk = [(x + 1.0 if x > 0 else math.exp(x)) if fmap == "elu" else max(x, 0.0)
+                              for x in k[0, 0, j]]
+                        raw.append(sum(a * b for a, b in zip(pq, pk)) if (not causal or j <= i) else 0.0)
+                    s = sum(raw)
+                    exp = [r / (s + 1e-6) for r in raw]
+                    _close(w[i], exp, rtol=1e-12, atol=1e-14)
+
+
+def pin_linear_equals_definition(ora):
+    """The grouped form phi(Q)(phi(K)^T V) equals the weighted-sum definition."""
+    rng = _rng(14)
+    B, H, N, D = 2, 3, 41, 7
+    q = rng.standard_normal((B, H, N, D))
+    k = rng.standard_normal((B, H, N, D))
+    v = rng.standard_normal((B, H, N, D))
+    W = rng.standard_normal((H, D, 16)) / math.sqrt(D)
+    for fmap in ("elu", "relu"):
+        for causal in (False, True):
+            for Wx in (None, W, W[1]):
+                a = ora.forward(q, k, v, fmap, 1e-6, causal, Wx)
+                b = ora.brute_force(q, k, v, fmap, 1e-6, causal, Wx)
+                _close(a, b, rtol=1e-12, atol=1e-13)
+                r = ora.rows(q, k, v, 1, 2, [0, 5, N - 1], fmap, 1e-6, causal, Wx)
+                _close(r, b[1, 2, [0, 5, N - 1]], rtol=1e-12, atol=1e-13)
+
+
+def pin_causal_structure(ora):
+    """Row 0 sees only key 0; the last causal row equals the last non-causal row;
+    row i of a causal problem equals the non-causal answer on the first i+1 tokens."""
+    rng = _rng(15)
+    N, D = 17, 4
+    q = rng.standard_normal((1, 1, N, D))
+    k = rng.standard_normal((1, 1, N, D))
+    v = rng.standard_normal((1, 1, N, D))
+    for fmap in ("elu", "relu"):
+        c = ora.forward(q, k, v, fmap, 1e-6, True)
+        nc = ora.forward(q, k, v, fmap, 1e-6, False)
+        _close(c[0, 0, -1], nc[0, 0, -1], rtol=1e-12)
+        for i in (0, 3, 9):
+            pre = ora.forward(q[:, :, :i + 1], k[:, :, :i + 1], v[:, :, :i + 1], fmap, 1e-6, False)
+            _close(c[0, 0, i], pre[0, 0, i], rtol=1e-12)
+        # row 0: s = phi(q_0).phi(k_0), out = v_0 s/(s+eps)
+        pq = ora.feature_map(q[0, 0, :1], fmap)[0]
+        pk = ora.feature_map(k[0, 0, :1], fmap)[0]
+        s = float(sum(a * b for a, b in zip(pq, pk)))
+        _close(c[0, 0, 0], v[0, 0, 0] * s / (s + 1e-6), rtol=1e-12)
+
+
+def pin_invariances(ora):
+    """Linear in V; non-causal output invariant to a joint permutation of the
+    key/value rows; relu with eps = 0 invariant to scaling a query by c > 0."""
+    rng = _rng(16)
+    B, H, N, D = 1, 2, 29, 6
+    q = rng.standard_normal((B, H, N, D))
+    k = rng.standard_normal((B, H, N, D))
+    v1 = rng.standard_normal((B, H, N, D))
+    v2 = rng.standard_normal((B, H, N, D))
+    for causal in (False, True):
+        lhs = ora.forward(q, k, 2.0 * v1 - 3.0 * v2, "elu", 1e-6, causal)
+        rhs = 2.0 * ora.forward(q, k, v1, "elu", 1e-6, causal) - 3.0 * ora.forward(q, k, v2, "elu", 1e-6, causal)
+        _close(lhs, rhs, rtol=1e-11)
+    perm = rng.permutation(N)
+    _close(ora.forward(q, k[:, :, perm], v1[:, :, perm], "elu", 1e-6, False),
+           ora.forward(q, k, v1, "elu", 1e-6, False), rtol=1e-12)
+    # permuting the queries permutes the rows
+    _close(ora.forward(q[:, :, perm], k, v1, "relu", 1e-6, False),
+           ora.forward(q, k, v1, "relu", 1e-6, False)[:, :, perm], rtol=1e-12)
+    qpos = np.abs(q) + 0.1
+    _close(ora.forward(3.5 * qpos, k, v1, "relu", 0.0, False),
+           ora.forward(qpos, k, v1, "relu", 0.0, False), rtol=1e-12)
+
+
+def pin_relu_zero_denominator(ora):
+    """relu with a query row <= 0: every weight is 0 and the row is 0/eps = 0."""
+    rng = _rng(17)
+    N, D = 8, 4
+    q = rng.standard_normal((1, 1, N, D))
+    q[0, 0, 3] = -np.abs(q[0, 0, 3])
+    k = rng.standard_normal((1, 1, N, D))
+    v = rng.standard_normal((1, 1, N, D))
+    for causal in (False, True):
+        for f in (ora.forward, ora.brute_force):
+            o = f(q, k, v, "relu", 1e-6, causal)
+            assert np.all(o[0, 0, 3] == 0.0)
+            assert np.all(np.isfinite(o))
+
+
+def pin_projection_reduction(ora):
+    """W = [I_D | 0] (D x F): phi(xW) = [elu(x)+1, 1, ..., 1], so
+    w_ij = (elu(q_i)+1).(elu(k_j)+1) + (F - D); checked against weights built
+    here from the unprojected feature map.  A per-head W is indexed by head."""
+    rng = _rng(18)
+    B, H, N, D, F = 1, 2, 13, 4, 12
+    q = rng.standard_normal((B, H, N, D))
+    k = rng.standard_normal((B, H, N, D))
+    v = rng.standard_normal((B, H, N, D))
+    W = np.zeros((D, F))
+    W[:, :D] = np.eye(D)
+    for causal in (False, True):
+        got = ora.forward(q, k, v, "elu", 1e-6, causal, W)
+        for h in range(H):
+            pq = ora.phi_elu1(q[0, h])
+            pk = ora.phi_elu1(k[0, h])
+            w = pq @ pk.T + (F - D)
+            if causal:
+                w = np.tril(w)
+            exp = (w @ v[0, h]) / (w.sum(axis=1) + 1e-6)[:, None]
+            _close(got[0, h], exp, rtol=1e-12)
+    # per-head matrices: head 1 gets a permuted identity, which must not change
+    # the result, while head 0 gets a scaled one, which must
+    Wh = np.stack([2.0 * W, W[:, rng.permutation(F)]])
+    got = ora.forward(q, k, v, "elu", 1e-6, False, Wh)
+    _close(got[0, 1], ora.forward(q, k, v, "elu", 1e-6, False, W)[0, 1], rtol=1e-12)
+    pq = ora.phi_elu1(2.0 * q[0, 0])
+    pk = ora.phi_elu1(2.0 * k[0, 0])
+    w = pq @ pk.T + (F - D)
+    _close(got[0, 0], (w @ v[0, 0]) / (w.sum(axis=1) + 1e-6)[:, None], rtol=1e-12)
+
+
+ALL_PINS = [
+    pin_feature_maps,
+    pin_feature_map_vs_torch,
+    pin_golden,
+    pin_negative_elu_closed_form,
+    pin_constant_values,
+    pin_zero_qk_closed_form,
+    pin_identity_values_give_weights,
+    pin_linear_equals_definition,
+    pin_causal_structure,
+    pin_invariances,
+    pin_relu_zero_denominator,
+    pin_projection_reduction,
+]

@@ -1,0 +1,91 @@
+"""The float64 oracle against facts fixed outside it (CPU only).
+
+Every pin in ``oracle_pins`` must pass on the oracle, and each mistake planted
+below in a copy of the oracle's source must make at least one pin fail, so that
+the pins are known to see a dropped term, a wrong sign or index, a transposed
+operand or a shifted causal mask.
+"""
+
+import importlib.util
+import os
+import types
+
+import pytest
+
+import oracle_pins
+from oracle import la_oracle
+
+ORACLE_SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "oracle", "la_oracle.py")
+
+
+@pytest.mark.parametrize("pin", oracle_pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(pin):
+    pin(la_oracle)
+
+
+# (name, text in the oracle, planted replacement)
+MUTANTS = [
+    ("elu_drops_plus_one", "x > 0.0, x + 1.0, np.exp", "x > 0.0, x, np.exp"),
+    ("elu_wrong_sign", "np.exp(np.minimum(x, 0.0))", "np.exp(-np.minimum(x, 0.0))"),
+    ("elu_branch_at_wrong_point", "np.where(x > 0.0,", "np.where(x > 1.0,"),
+    ("relu_is_abs", "np.maximum(x, 0.0)", "np.abs(x)"),
+    ("definition_transposed", "w = pq @ pk.T ", "w = pk @ pq.T "),
+    ("definition_drops_eps", "den = w.sum(axis=1) + eps", "den = w.sum(axis=1)"),
+    ("definition_eps_inside", "den = w.sum(axis=1) + eps", "den = (w + eps).sum(axis=1)"),
+    ("definition_exclusive_causal", "w = np.tril(w) ", "w = np.tril(w, -1) "),
+    ("definition_key_normaliser", "den = w.sum(axis=1) + eps", "den = w.sum(axis=0) + eps"),
+    ("grouped_drops_eps", "den = pq @ ksum + eps", "den = pq @ ksum"),
+    ("grouped_ksum_wrong_axis", "ksum = pk.sum(axis=0)", "ksum = pq.sum(axis=0)"),
+    ("grouped_kv_uses_queries", "kv = pk.T @ v", "kv = pq.T @ v"),
+    ("recurrence_reads_before_update",
+     "        S += np.outer(pk[i], v[i])\n        z += pk[i]\n        out[i] = (pq[i] @ S) / (pq[i] @ z + eps)",
+     "        out[i] = (pq[i] @ S) / (pq[i] @ z + eps)\n        S += np.outer(pk[i], v[i])\n        z += pk[i]"),
+    ("recurrence_transposed_state", "S += np.outer(pk[i], v[i])", "S += np.outer(pk[i], v[i]) if pk.shape[1] != v.shape[1] else np.outer(v[i], pk[i])"),
+    ("rows_exclusive_causal", "jend = i + 1 if causal", "jend = i if causal"),
+    ("projection_after_map", "        x = x @ np.asarray(W, dtype=np.float64)\n    if fmap == \"elu\":\n        return phi_elu1(x)",
+     "        pass\n    if fmap == \"elu\":\n        return phi_elu1(x) if W is None else phi_elu1(x) @ np.asarray(W, dtype=np.float64)"),
+    ("projection_head_zero", "return W if W.ndim == 2 else W[h]", "return W if W.ndim == 2 else W[0]"),
+]
+
+
+def _load_mutant(old, new):
+    with open(ORACLE_SRC) as fh:
+        src = fh.read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    src = src.replace(old, new)
+    mod = types.ModuleType("la_oracle_mutant")
+    exec(compile(src, "la_oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new):
+    mod = _load_mutant(old, new)
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mod)
+        except Exception as exc:  # AssertionError or a shape error
+            failed.append((pin.__name__, type(exc).__name__))
+    assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_oracle_rejects_bad_arguments():
+    import numpy as np
+    x = np.zeros((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        la_oracle.forward(x, x, x, "softmax")
+    with pytest.raises(ValueError):
+        la_oracle.forward(x, x, x, "elu", eps=-1.0)
+    with pytest.raises(ValueError):
+        la_oracle.forward(x[0], x[0], x[0])
+
+
+def test_oracle_module_spec_is_standalone():
+    """The oracle imports nothing from the CUDA package."""
+    spec = importlib.util.spec_from_file_location("o", ORACLE_SRC)
+    with open(ORACLE_SRC) as fh:
+        src = fh.read()
+    assert "linear_attention_diffusion_phi_b200" not in src
+    assert spec is not None
