@@ -1,0 +1,128 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) linear-time kernelised attention library.
+ *
+ * The operation (page "NNT Define Linear Attention", sections "The inputs" and
+ * "How it works"): per head, a non-negative feature map phi is applied to the
+ * query and key rows, the sequence is collapsed into the state
+ *     kv = sum_j phi(k_j) v_j^T   (F x D)      ksum = sum_j phi(k_j)   (F)
+ * and every output row is
+ *     out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).
+ * This equals the weighted sum  sum_j w_ij v_j / (sum_j w_ij + eps)  with
+ * w_ij = phi(q_i) . phi(k_j); the N x N weight matrix is never formed.
+ *   feature maps  LA_PHI_ELU1: elu(x)+1 (alpha = 1);  LA_PHI_RELU: max(x, 0)
+ *   causal        query i sees keys j <= i (itself included)
+ *   projection    F > 0: phi(x) = fmap(x W_h) with a D x F matrix per head
+ *                 (page "Flux2TTRTrainer", "Inputs worth setting": feature_dim
+ *                 is a multiple of 256); F = 0: phi acts on x itself (F = D).
+ *
+ * Memory.  Every pointer passed to the library is owned by the caller.  The
+ * library allocates no device memory and keeps only non-owning pointers in a
+ * handle; scratch space ("workspace") is a caller-owned device buffer of
+ * la_workspace_bytes() bytes.  Device pointers must address memory of the
+ * device that is current when la_forward is called.
+ *
+ * Layout.  q, k, v and out are dense row-major [B, H, N, D] tensors (D
+ * innermost), all of the handle's dtype; out never aliases q, k or v.
+ * W is [H, D, F] row-major (F innermost) with head stride head_stride
+ * elements (0: one matrix shared by all heads).
+ *
+ * Asynchrony.  la_forward only enqueues kernels on the given stream (a
+ * cudaStream_t passed as void*, NULL = legacy default stream) and returns.
+ *
+ * Errors.  Argument errors are detected on the host before anything is
+ * enqueued; out is then untouched.  Launch failures return LA_ERR_CUDA.
+ * Errors detected on the device (a bounded wait that ran out) are recorded in a
+ * status word inside the workspace and reported by la_sync_status().
+ *
+ * Threading.  A handle may be used by one host thread at a time.  Calls that
+ * share a workspace must be ordered on the device (same stream, or events).
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct la_handle_s* la_handle_t;
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, eps < 0, bad enum */
+  LA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape/dtype this build runs   */
+  LA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
+  LA_ERR_WORKSPACE = 4,     /* no workspace bound, or it is too small         */
+  LA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed    */
+  LA_ERR_TIMEOUT = 6,       /* a kernel gave up on a bounded device-side wait */
+  LA_ERR_NO_DEVICE = 7      /* no usable sm_100 device is current             */
+} la_status_t;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype_t;
+typedef enum { LA_PHI_ELU1 = 0, LA_PHI_RELU = 1 } la_feature_map_t;
+
+/* Create a handle for one storage dtype (LA_F32 or LA_BF16).  Allocates host
+ * memory only.  LA_F32 runs fp32 CUDA-core kernels with fp32 accumulation;
+ * LA_BF16 runs tcgen05 tensor-core kernels with fp32 accumulation. */
+la_status_t la_create(la_handle_t* handle, int dtype);
+
+/* Destroy a handle.  Frees host memory only; pending work is not waited on. */
+la_status_t la_destroy(la_handle_t handle);
+
+/* Bind the projection used when la_forward is called with F > 0.
+ * W: device pointer, [H, D, F] of the handle's dtype, 16-byte aligned, not
+ * copied (it must stay valid while calls that use it are pending).
+ * head_stride: elements between consecutive heads' matrices, D*F for one
+ * matrix per head, 0 for one matrix shared by all heads.  F must be a positive
+ * multiple of 256 (page "Flux2TTRTrainer", "Inputs worth setting").
+ * W = NULL unbinds. */
+la_status_t la_set_projection(la_handle_t handle, const void* W, int H, int D, int F,
+                              long long head_stride);
+
+/* Workspace bytes la_forward needs for this problem (0 if the arguments are
+ * invalid for the handle).  The size depends only on the arguments and the
+ * device's SM count; it is at most a few MB for the shapes above. */
+size_t la_workspace_bytes(la_handle_t handle, int B, int H, int N, int D, int F, int causal);
+
+/* Bind a caller-owned device workspace (256-byte aligned).  The library writes
+ * partial states and its status word there.  Bytes = 0 or ptr = NULL unbinds. */
+la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
+
+/* Enqueue out = phi-attention(q, k, v) on `stream` (see the top of this file).
+ * B, H, N >= 0 (any of them 0: nothing is enqueued, LA_OK); D > 0; F = 0 or a
+ * positive multiple of 256 with a projection bound; feature_map is a
+ * la_feature_map_t; eps >= 0; causal is 0 or 1.
+ * Supported: LA_F32: D <= 128, D % 4 == 0, F in {0, 256}.
+ *            LA_BF16: D in {64, 128}; F in {0, 256} with D = 128 when F > 0;
+ *            causal with F = 0.
+ * The result is deterministic: the same arguments give bitwise the same out. */
+la_status_t la_forward(la_handle_t handle, const void* q, const void* k, const void* v,
+                       void* out, int B, int H, int N, int D, int F, int feature_map,
+                       float eps, int causal, void* stream);
+
+/* End-to-end variant over HOST buffers: copies q, k, v (host, pinned for
+ * asynchrony) into the caller's device buffers dq, dk, dv, runs la_forward into
+ * dout and copies dout back to out_host, all enqueued on `stream`.  The host
+ * buffers must stay valid until the stream reaches the end of the copies. */
+la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* k_host,
+                            const void* v_host, void* out_host, void* dq, void* dk, void* dv,
+                            void* dout, int B, int H, int N, int D, int F, int feature_map,
+                            float eps, int causal, void* stream);
+
+/* Wait for `stream`, then read and clear the device status word of the bound
+ * workspace.  Returns LA_OK, LA_ERR_TIMEOUT (a kernel abandoned a bounded
+ * wait; its output is undefined) or LA_ERR_CUDA. */
+la_status_t la_sync_status(la_handle_t handle, void* stream);
+
+/* Static description of a status code. */
+const char* la_status_string(la_status_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

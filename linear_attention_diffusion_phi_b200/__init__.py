@@ -1,0 +1,195 @@
+"""Python binding of the B200 linear-time phi-attention library (libla_phi.so).
+
+The functions named ``la_*`` are one-to-one ctypes wrappers of the C ABI in
+``include/la.h`` (argument marshalling only: pointers are plain integers and
+every step of the computation runs in the library's CUDA kernels).
+``LinearAttention`` is a convenience layer over them for torch tensors: torch
+supplies device memory (the workspace) and the current stream, nothing else.
+There is no fallback: without the built library every call raises.
+"""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libla_phi.so")
+
+LA_F32, LA_BF16 = 0, 1
+LA_PHI_ELU1, LA_PHI_RELU = 0, 1
+FEATURE_MAPS = {"elu": LA_PHI_ELU1, "relu": LA_PHI_RELU}
+
+LA_OK = 0
+STATUS_NAMES = {
+    0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_MISALIGNED",
+    4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT", 7: "LA_ERR_NO_DEVICE",
+}
+
+EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
+            "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version")
+
+
+class LAError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({la_status_string(status)})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libla_phi.so (built by ``build.build()``); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                           "(run linear_attention_diffusion_phi_b200.build.build())")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+    L.la_create.argtypes = [ctypes.POINTER(vp), i32]
+    L.la_destroy.argtypes = [vp]
+    L.la_set_projection.argtypes = [vp, vp, i32, i32, i32, i64]
+    L.la_workspace_bytes.argtypes = [vp, i32, i32, i32, i32, i32, i32]
+    L.la_workspace_bytes.restype = sz
+    L.la_set_workspace.argtypes = [vp, vp, sz]
+    L.la_forward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
+    L.la_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
+    L.la_sync_status.argtypes = [vp, vp]
+    L.la_status_string.argtypes = [i32]
+    L.la_status_string.restype = ctypes.c_char_p
+    L.la_version.argtypes = []
+    for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
+                 "la_forward_host", "la_sync_status"):
+        getattr(L, name).restype = i32
+    _lib = L
+    return L
+
+
+# ------------------------------------------------------------ C-ABI wrappers
+
+def la_create(dtype):
+    h = ctypes.c_void_p()
+    st = lib().la_create(ctypes.byref(h), dtype)
+    if st != LA_OK:
+        raise LAError(st, "la_create")
+    return h.value
+
+
+def la_destroy(handle):
+    return lib().la_destroy(handle)
+
+
+def la_set_projection(handle, W_ptr, H, D, F, head_stride):
+    return lib().la_set_projection(handle, W_ptr, H, D, F, head_stride)
+
+
+def la_workspace_bytes(handle, B, H, N, D, F, causal):
+    return lib().la_workspace_bytes(handle, B, H, N, D, F, int(causal))
+
+
+def la_set_workspace(handle, ptr, nbytes):
+    return lib().la_set_workspace(handle, ptr, nbytes)
+
+
+def la_forward(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, causal, stream):
+    return lib().la_forward(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, int(causal), stream)
+
+
+def la_forward_host(handle, q_host, k_host, v_host, out_host, dq, dk, dv, dout, B, H, N, D, F,
+                    feature_map, eps, causal, stream):
+    return lib().la_forward_host(handle, q_host, k_host, v_host, out_host, dq, dk, dv, dout, B, H, N, D, F,
+                                 feature_map, eps, int(causal), stream)
+
+
+def la_sync_status(handle, stream):
+    return lib().la_sync_status(handle, stream)
+
+
+def la_status_string(status):
+    try:
+        return lib().la_status_string(status).decode()
+    except RuntimeError:
+        return "library not loaded"
+
+
+def la_version():
+    return lib().la_version()
+
+
+def check(status, what="la call"):
+    if status != LA_OK:
+        raise LAError(status, what)
+
+
+# ------------------------------------------------------- torch convenience
+
+class LinearAttention:
+    """out = phi-attention(q, k, v) for torch CUDA tensors [B, H, N, D].
+
+    dtype: torch.bfloat16 (tensor-core path) or torch.float32 (CUDA-core path).
+    W: optional projection [H, D, F] (or [D, F], shared by all heads).
+    """
+
+    def __init__(self, dtype, feature_map="elu", eps=1e-6, causal=False, W=None):
+        import torch
+        self.torch = torch
+        self.dtype = dtype
+        self.code = LA_BF16 if dtype == torch.bfloat16 else LA_F32
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+        self.fmap = FEATURE_MAPS[feature_map]
+        self.eps = float(eps)
+        self.causal = bool(causal)
+        self.handle = la_create(self.code)
+        self.W = None
+        self.F = 0
+        self._ws = None
+        if W is not None:
+            self.set_projection(W)
+
+    def set_projection(self, W):
+        if W.dim() == 2:
+            H, (D, F), stride = 1, W.shape, 0
+        else:
+            H, D, F = W.shape
+            stride = D * F
+        W = W.contiguous()
+        check(la_set_projection(self.handle, W.data_ptr(), H, D, F, stride), "la_set_projection")
+        self.W, self.F = W, F
+
+    def workspace_bytes(self, B, H, N, D):
+        return la_workspace_bytes(self.handle, B, H, N, D, self.F, self.causal)
+
+    def _bind_workspace(self, B, H, N, D, device):
+        need = self.workspace_bytes(B, H, N, D)
+        if need == 0:
+            raise LAError(1, "la_workspace_bytes")
+        if self._ws is None or self._ws.numel() < need or self._ws.device != device:
+            self._ws = self.torch.empty(need, dtype=self.torch.uint8, device=device)
+            check(la_set_workspace(self.handle, self._ws.data_ptr(), self._ws.numel()), "la_set_workspace")
+
+    def __call__(self, q, k, v, out=None, stream=None):
+        B, H, N, D = q.shape
+        if out is None:
+            out = self.torch.empty_like(q)
+        self._bind_workspace(B, H, N, D, q.device)
+        s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
+        check(la_forward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         B, H, N, D, self.F, self.fmap, self.eps, self.causal, s), "la_forward")
+        return out
+
+    def sync_status(self, stream=None):
+        s = stream if stream is not None else self.torch.cuda.current_stream().cuda_stream
+        return la_sync_status(self.handle, s)
+
+    def close(self):
+        if self.handle:
+            la_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

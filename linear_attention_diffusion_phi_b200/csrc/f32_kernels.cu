@@ -1,0 +1,287 @@
+// f32_kernels.cu -- fp32 CUDA-core path for every mode (non-causal, causal,
+// projected).  fp32 inputs are held to a 1e-5 relative bar, which the bf16 /
+// tf32 tensor-core operand formats cannot meet, so this path uses FFMA with
+// fp32 accumulation and the accurate expf.
+//
+// Method (page "NNT Define Linear Attention", "How it works"): the state
+// kv = phi(K)^T V and ksum = sum_j phi(k_j) is reduced over the sequence, then
+// out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).  The causal variant carries
+// the state over the sequence: each segment's state is reduced, an exclusive
+// scan over segments gives every segment its starting state, and each segment
+// then walks its tokens in order (update with token i, then read row i).
+#include <cuda_runtime.h>
+
+#include "la_internal.h"
+#include "sm100.cuh"
+
+namespace la {
+namespace {
+
+constexpr int kT = 16;      // tokens per chunk
+constexpr int kFB = 32;     // features per state block
+constexpr int kMaxD = 128;
+constexpr int kMaxFe = 256;
+
+// phi of token row `t` (already in shared memory) for feature f.
+__device__ __forceinline__ float feature(const float* xs, int D, const float* W, int F, int f, int fmap) {
+  float x;
+  if (F) {
+    x = 0.f;
+    for (int d = 0; d < D; ++d) x = fmaf(xs[d], __ldg(W + static_cast<size_t>(d) * F + f), x);
+  } else {
+    x = xs[f];
+  }
+  return phi_accurate(x, fmap);
+}
+
+__device__ __forceinline__ void load_rows(float* dst, const float* src, int rows_valid, int D) {
+  // dst[kT][kMaxD]; rows >= rows_valid are zero-filled.  D % 4 == 0.
+  const int d4 = D / 4;
+  for (int e = threadIdx.x; e < kT * d4; e += blockDim.x) {
+    const int t = e / d4, c = e % d4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < rows_valid) x = *reinterpret_cast<const float4*>(src + static_cast<size_t>(t) * D + 4 * c);
+    *reinterpret_cast<float4*>(dst + t * kMaxD + 4 * c) = x;
+  }
+}
+
+// Partial state of tokens [s*seg, min(N, (s+1)*seg)) of head bh, features
+// [32*blockIdx.z, +32): part[bh][s][f][d] and part_ksum[bh][s][f].
+__global__ void __launch_bounds__(256) f32_state_partial(const float* __restrict__ k, const float* __restrict__ v,
+                                                         const float* __restrict__ W, long long wstride,
+                                                         float* __restrict__ part, float* __restrict__ part_ksum,
+                                                         int H, int N, int D, int F, int Fe, int fmap, int seg,
+                                                         int S) {
+  __shared__ __align__(16) float Ks[kT * kMaxD];
+  __shared__ __align__(16) float Vs[kT * kMaxD];
+  __shared__ float Ps[kT * kFB];
+  const int s = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const int fb = blockIdx.z * kFB;
+  const float* Wh = F ? W + static_cast<size_t>(bh % H) * wstride : nullptr;
+  const float* kh = k + static_cast<size_t>(bh) * N * D;
+  const float* vh = v + static_cast<size_t>(bh) * N * D;
+  const int t0 = s * seg, t1 = min(N, t0 + seg);
+  const int fl = threadIdx.x / 8, dl = threadIdx.x % 8;
+  float acc[kMaxD / 8];
+#pragma unroll
+  for (int j = 0; j < kMaxD / 8; ++j) acc[j] = 0.f;
+  float ks = 0.f;
+  for (int tc = t0; tc < t1; tc += kT) {
+    const int rows = min(kT, t1 - tc);
+    load_rows(Ks, kh + static_cast<size_t>(tc) * D, rows, D);
+    load_rows(Vs, vh + static_cast<size_t>(tc) * D, rows, D);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * kFB; e += blockDim.x) {
+      const int t = e / kFB, f = fb + e % kFB;
+      Ps[e] = (t < rows && f < Fe) ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+    }
+    __syncthreads();
+    for (int t = 0; t < kT; ++t) {
+      const float p = Ps[t * kFB + fl];
+#pragma unroll
+      for (int j = 0; j < kMaxD / 8; ++j) {
+        const int d = dl + 8 * j;
+        if (d < D) acc[j] = fmaf(p, Vs[t * kMaxD + d], acc[j]);
+      }
+      ks += p;
+    }
+    __syncthreads();
+  }
+  const int f = fb + fl;
+  if (f < Fe) {
+    float* dst = part + ((static_cast<size_t>(bh) * S + s) * Fe + f) * D;
+#pragma unroll
+    for (int j = 0; j < kMaxD / 8; ++j) {
+      const int d = dl + 8 * j;
+      if (d < D) dst[d] = acc[j];
+    }
+    if (dl == 0) part_ksum[(static_cast<size_t>(bh) * S + s) * Fe + f] = ks;
+  }
+}
+
+// final[bh] = sum_{s=0..S-1} part[bh][s], summed in ascending s.
+__global__ void f32_state_combine(const float* __restrict__ part, const float* __restrict__ part_ksum,
+                                  float* __restrict__ fin, float* __restrict__ fin_ksum, int Fe, int D, int S) {
+  const long long bh = blockIdx.x;
+  const int n_kv = Fe * D;
+  const int e = blockIdx.y * blockDim.x + threadIdx.x;
+  if (e < n_kv) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(static_cast<size_t>(bh) * S + s) * n_kv + e];
+    fin[static_cast<size_t>(bh) * n_kv + e] = acc;
+  } else if (e < n_kv + Fe) {
+    const int f = e - n_kv;
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part_ksum[(static_cast<size_t>(bh) * S + s) * Fe + f];
+    fin_ksum[static_cast<size_t>(bh) * Fe + f] = acc;
+  }
+}
+
+// In-place exclusive scan over segments (ascending s): part[s] <- sum_{s'<s}.
+__global__ void f32_state_scan(float* __restrict__ part, float* __restrict__ part_ksum, int Fe, int D, int S) {
+  const long long bh = blockIdx.x;
+  const int n_kv = Fe * D;
+  const int e = blockIdx.y * blockDim.x + threadIdx.x;
+  float* base;
+  int stride;
+  if (e < n_kv) {
+    base = part + static_cast<size_t>(bh) * S * n_kv + e;
+    stride = n_kv;
+  } else if (e < n_kv + Fe) {
+    base = part_ksum + static_cast<size_t>(bh) * S * Fe + (e - n_kv);
+    stride = Fe;
+  } else {
+    return;
+  }
+  float run = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float x = base[static_cast<size_t>(s) * stride];
+    base[static_cast<size_t>(s) * stride] = run;
+    run += x;
+  }
+}
+
+// out rows [blockIdx.x*16, +16) of head bh from the final state.
+__global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, const float* __restrict__ W,
+                                                 long long wstride, const float* __restrict__ fin,
+                                                 const float* __restrict__ fin_ksum, float* __restrict__ out,
+                                                 int H, int N, int D, int F, int Fe, int fmap, float eps) {
+  __shared__ __align__(16) float Qs[kT * kMaxD];
+  __shared__ float Ps[kT * kMaxFe];
+  __shared__ float den[kT];
+  const long long bh = blockIdx.y;
+  const int t0 = blockIdx.x * kT;
+  const int rows = min(kT, N - t0);
+  const float* Wh = F ? W + static_cast<size_t>(bh % H) * wstride : nullptr;
+  const float* kv = fin + static_cast<size_t>(bh) * Fe * D;
+  const float* ksum = fin_ksum + static_cast<size_t>(bh) * Fe;
+  load_rows(Qs, q + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
+  __syncthreads();
+  for (int e = threadIdx.x; e < kT * Fe; e += blockDim.x) {
+    const int t = e / Fe, f = e % Fe;
+    Ps[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+  }
+  __syncthreads();
+  // den[t] = phi(q_t) . ksum + eps : one warp per two rows, lanes split f.
+  {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int t = warp; t < kT; t += blockDim.x / 32) {
+      float acc = 0.f;
+      for (int f = lane; f < Fe; f += 32) acc = fmaf(Ps[t * kMaxFe + f], ksum[f], acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) den[t] = acc + eps;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
+    const int t = e / D, d = e % D;
+    float num = 0.f;
+    for (int f = 0; f < Fe; ++f) num = fmaf(Ps[t * kMaxFe + f], kv[static_cast<size_t>(f) * D + d], num);
+    out[(static_cast<size_t>(bh) * N + t0 + t) * D + d] = num / den[t];
+  }
+}
+
+// Causal: segment s of head bh starts from the exclusive prefix state
+// pre[bh][s] and walks its tokens in order.  Dynamic shared memory holds the
+// state St[Fe][D] and z[Fe].
+__global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict__ q, const float* __restrict__ k,
+                                                        const float* __restrict__ v, const float* __restrict__ W,
+                                                        long long wstride, const float* __restrict__ pre,
+                                                        const float* __restrict__ pre_ksum,
+                                                        float* __restrict__ out, int H, int N, int D, int F,
+                                                        int Fe, int fmap, float eps, int seg, int S) {
+  extern __shared__ __align__(16) float dyn[];
+  float* Qs = dyn;                 // kT * kMaxD
+  float* Ks = Qs + kT * kMaxD;
+  float* Vs = Ks + kT * kMaxD;
+  float* Pq = Vs + kT * kMaxD;     // kT * kMaxFe
+  float* Pk = Pq + kT * kMaxFe;
+  float* St = Pk + kT * kMaxFe;    // Fe * D
+  float* z = St + Fe * D;          // Fe
+  const int s = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const float* Wh = F ? W + static_cast<size_t>(bh % H) * wstride : nullptr;
+  const size_t head = static_cast<size_t>(bh) * N * D;
+  const int t0 = s * seg, t1 = min(N, t0 + seg);
+  const float* p0 = pre + (static_cast<size_t>(bh) * S + s) * Fe * D;
+  for (int e = threadIdx.x; e < Fe * D; e += blockDim.x) St[e] = p0[e];
+  for (int f = threadIdx.x; f < Fe; f += blockDim.x) z[f] = pre_ksum[(static_cast<size_t>(bh) * S + s) * Fe + f];
+  for (int tc = t0; tc < t1; tc += kT) {
+    const int rows = min(kT, t1 - tc);
+    __syncthreads();
+    load_rows(Qs, q + head + static_cast<size_t>(tc) * D, rows, D);
+    load_rows(Ks, k + head + static_cast<size_t>(tc) * D, rows, D);
+    load_rows(Vs, v + head + static_cast<size_t>(tc) * D, rows, D);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * Fe; e += blockDim.x) {
+      const int t = e / Fe, f = e % Fe;
+      Pq[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+      Pk[t * kMaxFe + f] = t < rows ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+    }
+    __syncthreads();
+    for (int t = 0; t < rows; ++t) {
+      for (int e = threadIdx.x; e < Fe * D; e += blockDim.x) {
+        const int f = e / D, d = e % D;
+        St[e] = fmaf(Pk[t * kMaxFe + f], Vs[t * kMaxD + d], St[e]);
+      }
+      for (int f = threadIdx.x; f < Fe; f += blockDim.x) z[f] += Pk[t * kMaxFe + f];
+      __syncthreads();
+      for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float num = 0.f, den = 0.f;
+        for (int f = 0; f < Fe; ++f) {
+          const float p = Pq[t * kMaxFe + f];
+          num = fmaf(p, St[f * D + d], num);
+          den = fmaf(p, z[f], den);
+        }
+        out[head + static_cast<size_t>(tc + t) * D + d] = num / (den + eps);
+      }
+      __syncthreads();
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_f32(const LaunchArgs& a) {
+  const Plan& p = *a.p;
+  const float* q = static_cast<const float*>(a.q);
+  const float* k = static_cast<const float*>(a.k);
+  const float* v = static_cast<const float*>(a.v);
+  const float* W = static_cast<const float*>(a.W);
+  float* out = static_cast<float*>(a.out);
+  float* part = reinterpret_cast<float*>(a.ws + p.off_partial);
+  float* part_ksum = reinterpret_cast<float*>(a.ws + p.off_ksum_partial);
+  const int S = p.splits;
+  const int n_state = p.Fe * p.D + p.Fe;
+
+  dim3 g1(S, static_cast<unsigned>(p.BH), (p.Fe + kFB - 1) / kFB);
+  f32_state_partial<<<g1, 256, 0, a.stream>>>(k, v, W, a.w_head_stride, part, part_ksum, p.H, p.N, p.D, p.F, p.Fe,
+                                              p.fmap, p.seg_len, S);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dim3 g2(static_cast<unsigned>(p.BH), (n_state + 255) / 256);
+  if (!p.causal) {
+    float* fin = reinterpret_cast<float*>(a.ws + p.off_final);
+    float* fin_ksum = reinterpret_cast<float*>(a.ws + p.off_final_ksum);
+    f32_state_combine<<<g2, 256, 0, a.stream>>>(part, part_ksum, fin, fin_ksum, p.Fe, p.D, S);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    dim3 g3((p.N + kT - 1) / kT, static_cast<unsigned>(p.BH));
+    f32_apply<<<g3, 256, 0, a.stream>>>(q, W, a.w_head_stride, fin, fin_ksum, out, p.H, p.N, p.D, p.F, p.Fe, p.fmap,
+                                        p.eps);
+    return cudaGetLastError();
+  }
+  f32_state_scan<<<g2, 256, 0, a.stream>>>(part, part_ksum, p.Fe, p.D, S);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const size_t dyn = (3 * kT * kMaxD + 2 * kT * kMaxFe) * sizeof(float) +
+                     (static_cast<size_t>(p.Fe) * p.D + p.Fe) * sizeof(float);
+  err = cudaFuncSetAttribute(f32_causal_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
+  if (err != cudaSuccess) return err;
+  dim3 g3(S, static_cast<unsigned>(p.BH));
+  f32_causal_apply<<<g3, 256, dyn, a.stream>>>(q, k, v, W, a.w_head_stride, part, part_ksum, out, p.H, p.N, p.D, p.F,
+                                               p.Fe, p.fmap, p.eps, p.seg_len, S);
+  return cudaGetLastError();
+}
+
+}  // namespace la

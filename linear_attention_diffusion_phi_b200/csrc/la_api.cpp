@@ -1,0 +1,351 @@
+// la_api.cpp -- the C ABI of include/la.h: argument validation, the launch
+// plan (splits and workspace layout), TMA descriptor encoding and dispatch to
+// the fp32 CUDA-core or bf16 tensor-core kernels.  No device memory is ever
+// allocated here; the caller owns every buffer.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "la.h"
+#include "la_internal.h"
+
+struct la_handle_s {
+  int dtype;
+  const void* W;
+  int wH, wD, wF;
+  long long w_head_stride;
+  void* ws;
+  size_t ws_bytes;
+};
+
+namespace {
+
+using la::Plan;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+struct DeviceInfo {
+  int sms = 0, major = 0, minor = 0;
+};
+
+// SM count and compute capability of the current device (cached per device).
+bool device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  return true;
+}
+
+// Shape/dtype validation shared by la_workspace_bytes and la_forward.
+la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap, float eps,
+                        int causal) {
+  if (B < 0 || H < 0 || N < 0 || D <= 0 || F < 0) return LA_ERR_INVALID_ARG;
+  if (fmap != LA_PHI_ELU1 && fmap != LA_PHI_RELU) return LA_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || eps != eps) return LA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LA_ERR_INVALID_ARG;
+  if (F % 256 != 0) return LA_ERR_INVALID_ARG;   // feature_dim: a multiple of 256
+  if (static_cast<long long>(B) * H > 65535) return LA_ERR_UNSUPPORTED;
+  if (h->dtype == LA_F32) {
+    if (D > 128 || D % 4 != 0) return LA_ERR_UNSUPPORTED;
+    if (F != 0 && F != 256) return LA_ERR_UNSUPPORTED;
+  } else {
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    if (F != 0 && (F != 256 || D != 128)) return LA_ERR_UNSUPPORTED;
+    if (causal && F != 0) return LA_ERR_UNSUPPORTED;
+  }
+  return LA_OK;
+}
+
+void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap, float eps, int causal,
+               int num_sms, Plan* p) {
+  memset(p, 0, sizeof(*p));
+  p->dtype = h->dtype;
+  p->B = B; p->H = H; p->N = N; p->D = D; p->F = F;
+  p->Fe = F ? F : D;
+  p->fmap = fmap; p->causal = causal; p->eps = eps;
+  p->BH = static_cast<long long>(B) * H;
+  p->tiles = static_cast<int>(cdiv(N, la::kTileTokens));
+  p->num_sms = num_sms > 0 ? num_sms : 148;
+  const long long BH = std::max<long long>(p->BH, 1);
+  size_t partial_floats = 0, ksum_floats = 0, final_bytes = 0, final_ksum_bytes = 0, blob_total = 0;
+  if (h->dtype == LA_F32) {
+    // Enough (head, split, feature-block) blocks for ~2 waves; splits of whole
+    // 16-token chunks (non-causal) or >= 64 tokens (causal).
+    const long long fblocks = cdiv(p->Fe, 32);
+    long long want = std::max<long long>(1, cdiv(2LL * p->num_sms, BH * (causal ? 1 : fblocks)));
+    const int quantum = causal ? 64 : 16;
+    long long seg = std::max<long long>(quantum, cdiv(cdiv(std::max(N, 1), want), quantum) * quantum);
+    p->seg_len = static_cast<int>(seg);
+    p->splits = static_cast<int>(std::max<long long>(1, cdiv(std::max(N, 1), seg)));
+    partial_floats = static_cast<size_t>(BH) * p->splits * p->Fe * D;
+    ksum_floats = static_cast<size_t>(BH) * p->splits * p->Fe;
+    if (!causal) {
+      final_bytes = static_cast<size_t>(BH) * p->Fe * D * 4;
+      final_ksum_bytes = static_cast<size_t>(BH) * p->Fe * 4;
+    }
+  } else {
+    const int tiles = std::max(p->tiles, 1);
+    const long long want = std::max<long long>(1, p->num_sms / BH);
+    p->tiles_per_split = static_cast<int>(cdiv(tiles, std::min<long long>(want, tiles)));
+    p->splits = static_cast<int>(cdiv(tiles, p->tiles_per_split));
+    p->seg_len = p->tiles_per_split * la::kTileTokens;
+    partial_floats = static_cast<size_t>(BH) * p->splits * p->Fe * D;
+    ksum_floats = static_cast<size_t>(BH) * p->splits * p->Fe;
+    p->blob_bytes = la::blob_bytes_for(D, p->Fe);
+    blob_total = static_cast<size_t>(BH) * p->blob_bytes;
+  }
+  size_t off = 0;
+  p->off_status = off;        off += 256;
+  p->off_partial = off;       off = align256(off + partial_floats * 4);
+  p->off_ksum_partial = off;  off = align256(off + ksum_floats * 4);
+  p->off_final = off;         off = align256(off + final_bytes);
+  p->off_final_ksum = off;    off = align256(off + final_ksum_bytes);
+  p->off_blob = off;          off = align256(off + blob_total);
+  p->bytes = off;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// [outer, rows, cols] bf16 tensor, box [1, 128, 64] with the 128-byte swizzle.
+bool encode_bf16_3d(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,
+                    long long outer_stride_elems, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(outer_stride_elems) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+la_status_t la_create(la_handle_t* handle, int dtype) {
+  if (!handle) return LA_ERR_INVALID_ARG;
+  *handle = nullptr;
+  if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+  la_handle_s* h = new (std::nothrow) la_handle_s();
+  if (!h) return LA_ERR_INVALID_ARG;
+  h->dtype = dtype;
+  *handle = h;
+  return LA_OK;
+}
+
+la_status_t la_destroy(la_handle_t handle) {
+  if (!handle) return LA_ERR_INVALID_ARG;
+  delete handle;
+  return LA_OK;
+}
+
+la_status_t la_set_projection(la_handle_t h, const void* W, int H, int D, int F, long long head_stride) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  if (!W) {
+    h->W = nullptr;
+    h->wH = h->wD = h->wF = 0;
+    h->w_head_stride = 0;
+    return LA_OK;
+  }
+  if (H <= 0 || D <= 0 || F <= 0 || F % 256 != 0 || head_stride < 0) return LA_ERR_INVALID_ARG;
+  if (head_stride != 0 && head_stride < static_cast<long long>(D) * F) return LA_ERR_INVALID_ARG;
+  if (!aligned16(W) || head_stride % 8 != 0) return LA_ERR_MISALIGNED;
+  h->W = W;
+  h->wH = H;
+  h->wD = D;
+  h->wF = F;
+  h->w_head_stride = head_stride;
+  return LA_OK;
+}
+
+size_t la_workspace_bytes(la_handle_t h, int B, int H, int N, int D, int F, int causal) {
+  if (!h) return 0;
+  if (check_shape(h, B, H, N, D, F, LA_PHI_ELU1, 0.f, causal) != LA_OK) return 0;
+  DeviceInfo di;
+  const int sms = device_info(&di) ? di.sms : 148;
+  Plan p;
+  make_plan(h, B, H, N, D, F, LA_PHI_ELU1, 0.f, causal, sms, &p);
+  return p.bytes;
+}
+
+la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  if (!ptr || bytes == 0) {
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    return LA_OK;
+  }
+  if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return LA_ERR_MISALIGNED;
+  if (bytes < 256) return LA_ERR_WORKSPACE;
+  // Clear the device status word once, so that later reads see only errors
+  // of calls made with this workspace.
+  if (cudaMemset(ptr, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  h->ws = ptr;
+  h->ws_bytes = bytes;
+  return LA_OK;
+}
+
+la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                       int D, int F, int fmap, float eps, int causal, void* stream) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  la_status_t st = check_shape(h, B, H, N, D, F, fmap, eps, causal);
+  if (st != LA_OK) return st;
+  if (static_cast<long long>(B) * H * N == 0) return LA_OK;
+  if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_MISALIGNED;
+  if (F > 0) {
+    if (!h->W) return LA_ERR_INVALID_ARG;
+    if (h->wD != D || h->wF != F || (h->w_head_stride != 0 && h->wH < H)) return LA_ERR_INVALID_ARG;
+  }
+  DeviceInfo di;
+  if (!device_info(&di)) return LA_ERR_NO_DEVICE;
+  if (di.major != 10 || di.minor != 0) return LA_ERR_NO_DEVICE;   // kernels are built for sm_100a
+  Plan p;
+  make_plan(h, B, H, N, D, F, fmap, eps, causal, di.sms, &p);
+  if (!h->ws || h->ws_bytes < p.bytes) return LA_ERR_WORKSPACE;
+
+  la::LaunchArgs a = {};
+  a.p = &p;
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.W = F ? h->W : nullptr;
+  a.w_head_stride = h->w_head_stride;
+  a.ws = static_cast<char*>(h->ws);
+  a.stream = static_cast<cudaStream_t>(stream);
+
+  cudaError_t err;
+  if (h->dtype == LA_F32) {
+    err = la::launch_f32(a);
+  } else {
+    CUtensorMap tq, tk, tv, to, tw;
+    const long long BH = p.BH;
+    const long long hs = static_cast<long long>(N) * D;
+    if (!encode_bf16_3d(&tq, q, BH, N, D, hs, 128) || !encode_bf16_3d(&tk, k, BH, N, D, hs, 128) ||
+        !encode_bf16_3d(&tv, v, BH, N, D, hs, 128) || !encode_bf16_3d(&to, out, BH, N, D, hs, 128))
+      return LA_ERR_CUDA;
+    a.tm_q = &tq; a.tm_k = &tk; a.tm_v = &tv; a.tm_out = &to;
+    if (F > 0) {
+      const long long nW = h->w_head_stride ? H : 1;
+      const long long ws = h->w_head_stride ? h->w_head_stride : static_cast<long long>(D) * F;
+      if (!encode_bf16_3d(&tw, h->W, nW, D, F, ws, 128)) return LA_ERR_CUDA;
+      a.tm_w = &tw;
+    }
+    err = causal ? la::launch_bf16_causal(a) : la::launch_bf16_noncausal(a);
+  }
+  if (err == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
+  if (err != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
+la_status_t la_forward_host(la_handle_t h, const void* q_host, const void* k_host, const void* v_host,
+                            void* out_host, void* dq, void* dk, void* dv, void* dout, int B, int H, int N, int D,
+                            int F, int fmap, float eps, int causal, void* stream) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  la_status_t st = check_shape(h, B, H, N, D, F, fmap, eps, causal);
+  if (st != LA_OK) return st;
+  const size_t n = static_cast<size_t>(B) * H * N * D * (h->dtype == LA_F32 ? 4 : 2);
+  if (n == 0) return LA_OK;
+  if (!q_host || !k_host || !v_host || !out_host) return LA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  st = la_forward(h, dq, dk, dv, dout, B, H, N, D, F, fmap, eps, causal, stream);
+  if (st != LA_OK) return st;
+  if (cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
+la_status_t la_sync_status(la_handle_t h, void* stream) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  if (!h->ws) return LA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemcpy(&word, h->ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  if (word == 0) return LA_OK;
+  if (cudaMemset(h->ws, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return word == la::kDeviceTimeout ? LA_ERR_TIMEOUT : LA_ERR_CUDA;
+}
+
+const char* la_status_string(la_status_t s) {
+  switch (s) {
+    case LA_OK: return "ok";
+    case LA_ERR_INVALID_ARG: return "invalid argument";
+    case LA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case LA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case LA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LA_ERR_CUDA: return "CUDA error";
+    case LA_ERR_TIMEOUT: return "device-side wait timed out";
+    case LA_ERR_NO_DEVICE: return "no sm_100 device current";
+  }
+  return "unknown status";
+}
+
+int la_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// la_internal.h -- plan and launcher declarations shared by the host code and
+// the kernel translation units of the linear-attention library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace la {
+
+// Device-side wait limit: a kernel that waits this long on one barrier gives up.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kDeviceTimeout = 6;                            // == LA_ERR_TIMEOUT
+
+constexpr int kTileTokens = 128;   // tokens per tensor-core tile (MMA M or K)
+
+// Everything la_forward decides on the host, shared with la_workspace_bytes.
+struct Plan {
+  int dtype;       // 0 f32, 1 bf16
+  int B, H, N, D, F, Fe;   // Fe = F ? F : D (features per head)
+  int fmap, causal;
+  float eps;
+  long long BH;
+  int tiles;       // ceil(N / 128)
+  int splits;      // non-causal: N-splits per head; causal: segments per head
+  int tiles_per_split;   // in 128-token tiles (bf16) or tokens per split (f32, see seg_len)
+  int seg_len;     // tokens per split/segment
+  int num_sms;
+  // workspace layout (byte offsets from the workspace base, 256-aligned)
+  size_t off_status, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
+  size_t blob_bytes;   // bf16 B-operand image per head
+};
+
+// Per-head layout of the bf16 [kv | ksum | 0] B-operand image used by the
+// apply kernels: MN-major, 128-byte swizzle, N atoms of 64 columns.
+__host__ __device__ constexpr int blob_atoms(int D) { return (D + 16 + 63) / 64; }
+__host__ __device__ constexpr size_t blob_bytes_for(int D, int Fe) {
+  return static_cast<size_t>(blob_atoms(D)) * Fe * 128;
+}
+
+struct LaunchArgs {
+  const Plan* p;
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  const void* W;
+  long long w_head_stride;   // elements
+  char* ws;                  // workspace base
+  cudaStream_t stream;
+  // tensor maps (bf16 path); built on the host per call
+  const CUtensorMap* tm_q;
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+  const CUtensorMap* tm_out;
+  const CUtensorMap* tm_w;
+};
+
+// f32 CUDA-core path (all modes).
+cudaError_t launch_f32(const LaunchArgs& a);
+// bf16 tensor-core paths.
+cudaError_t launch_bf16_noncausal(const LaunchArgs& a);
+cudaError_t launch_bf16_causal(const LaunchArgs& a);
+
+}  // namespace la

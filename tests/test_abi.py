@@ -1,0 +1,147 @@
+"""The C-ABI library: it loads, exports every symbol include/la.h declares, and
+rejects bad arguments on the host before touching a device (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_diffusion_phi_b200 as la
+from linear_attention_diffusion_phi_b200 import build as la_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    la_build.build()
+    yield
+
+
+def declared_functions():
+    names = []
+    for path in HEADERS:
+        with open(path) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(la_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in la.EXPORTED:
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol():
+    L = la.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+
+
+def test_version_and_status_strings():
+    assert la.la_version() >= 100
+    for code in range(8):
+        s = la.la_status_string(code)
+        assert s and s != "unknown status"
+    assert la.la_status_string(99) == "unknown status"
+
+
+def test_create_destroy_and_bad_dtype():
+    h = la.la_create(la.LA_BF16)
+    assert h
+    assert la.la_destroy(h) == la.LA_OK
+    with pytest.raises(la.LAError):
+        la.la_create(7)
+    L = la.lib()
+    assert L.la_create(None, 0) == 1
+    assert L.la_destroy(None) == 1
+
+
+@pytest.fixture
+def handles():
+    hs = {"f32": la.la_create(la.LA_F32), "bf16": la.la_create(la.LA_BF16)}
+    yield hs
+    for h in hs.values():
+        la.la_destroy(h)
+
+
+def fwd(h, B=1, H=2, N=256, D=64, F=0, fmap=0, eps=1e-6, causal=0, ptr=0x1000, out=0x2000):
+    return la.la_forward(h, ptr, ptr, ptr, out, B, H, N, D, F, fmap, eps, causal, None)
+
+
+def test_forward_argument_validation(handles):
+    f32, b16 = handles["f32"], handles["bf16"]
+    # bad values
+    assert fwd(f32, B=-1) == 1
+    assert fwd(f32, D=0) == 1
+    assert fwd(f32, fmap=2) == 1
+    assert fwd(f32, eps=-1.0) == 1
+    assert fwd(f32, eps=float("nan")) == 1
+    assert fwd(f32, causal=2) == 1
+    assert fwd(f32, F=100) == 1            # feature_dim must be a multiple of 256
+    assert fwd(b16, F=128, D=128) == 1
+    # valid but not run by this build
+    assert fwd(f32, D=130) == 2
+    assert fwd(f32, D=6) == 2
+    assert fwd(b16, D=96) == 2
+    assert fwd(b16, D=64, F=256) == 2
+    assert fwd(b16, D=128, F=512) == 2
+    assert fwd(b16, D=128, F=256, causal=1) == 2
+    assert fwd(f32, B=300, H=300) == 2      # B*H beyond the grid limit
+    # empty problems are a no-op
+    assert fwd(f32, N=0, ptr=0, out=0) == 0
+    assert fwd(b16, B=0, D=128, ptr=0, out=0) == 0
+    # null and misaligned pointers
+    assert fwd(f32, ptr=0) == 1
+    assert fwd(f32, ptr=0x1004) == 3
+    assert fwd(b16, D=128, out=0x2008) == 3
+    # projection requested but none bound
+    assert fwd(b16, D=128, F=256) == 1
+
+
+def test_projection_validation(handles):
+    h = handles["bf16"]
+    assert la.la_set_projection(h, 0x1000, 24, 128, 255, 0) == 1
+    assert la.la_set_projection(h, 0x1000, 24, 128, 256, -1) == 1
+    assert la.la_set_projection(h, 0x1000, 24, 128, 256, 100) == 1   # stride < D*F
+    assert la.la_set_projection(h, 0x1008, 24, 128, 256, 0) == 3
+    assert la.la_set_projection(h, 0x1000, 24, 128, 256, 128 * 256) == 0
+    assert fwd(h, D=64, F=256) == 2
+    assert la.la_set_projection(h, None, 0, 0, 0, 0) == 0
+    assert fwd(h, D=128, F=256) == 1
+
+
+def test_workspace_bytes_and_binding(handles):
+    for name, h in handles.items():
+        n = la.la_workspace_bytes(h, 1, 24, 4608, 128 if name == "bf16" else 64, 0, 0)
+        assert n > 256 and n % 256 == 0
+        assert n < 64 << 20
+        assert la.la_workspace_bytes(h, 1, 24, 4608, 130, 0, 0) == 0
+    h = handles["bf16"]
+    # bf16 workspace for the Flux-1024 shape holds per-split fp32 states and
+    # the per-head bf16 operand images
+    n = la.la_workspace_bytes(h, 1, 24, 4608, 128, 0, 0)
+    assert n >= 24 * (128 * 128 * 4) + 24 * 3 * 128 * 128
+    assert la.la_workspace_bytes(h, 1, 24, 4608, 128, 256, 0) > n
+    assert la.la_set_workspace(h, 0x1010, 4096) == 3          # not 256-aligned
+    assert la.la_set_workspace(h, None, 0) == 0
+    assert la.la_sync_status(h, None) == 4                    # no workspace bound
+
+
+def test_no_device_is_reported_not_faked(handles):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert fwd(handles["f32"]) == 7
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(la, "_lib", None)
+    monkeypatch.setattr(la, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        la.la_version()

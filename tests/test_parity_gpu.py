@@ -1,0 +1,208 @@
+"""CUDA path against the float64 oracle on the same seeded inputs (B200 only).
+
+Tolerances: fp32 storage, ||g - o||_inf / ||o||_inf <= 1e-5; bf16 storage with
+fp32 accumulation, max |g - o| <= 2e-2 and mean |g - o| <= 2e-3, plus
+||g - o||_2 / ||o||_2 <= 1e-2 so that a near-zero output cannot pass.
+"""
+
+import numpy as np
+import pytest
+
+import linear_attention_diffusion_phi_b200 as la
+from linear_attention_diffusion_phi_b200 import build as la_build
+from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, Workload, as_float64, make_inputs
+from oracle import la_oracle as ora
+
+pytestmark = pytest.mark.gpu
+
+F32_REL = 1e-5
+BF16_MAX, BF16_MEAN, BF16_RL2 = 2e-2, 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    la_build.build()
+    yield
+
+
+def torch_dtype(w):
+    import torch
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def run_gpu(w, q, k, v, W=None, runs=1):
+    import torch
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch_dtype(w), w.fmap, w.eps, w.causal,
+                            None if W is None else W.to(dev))
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    outs = []
+    for _ in range(runs):
+        outs.append(op(qd, kd, vd).cpu())
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    return outs if runs > 1 else outs[0]
+
+
+def errors(got, ref):
+    g = as_float64(got) if not isinstance(got, np.ndarray) else got
+    d = np.abs(g - ref)
+    return {
+        "max_abs": float(d.max()) if d.size else 0.0,
+        "mean_abs": float(d.mean()) if d.size else 0.0,
+        "rel_inf": float(d.max() / max(np.abs(ref).max(), 1e-30)) if d.size else 0.0,
+        "rel_l2": float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30)) if d.size else 0.0,
+    }
+
+
+def assert_parity(got, ref, dtype):
+    e = errors(got, ref)
+    assert np.all(np.isfinite(as_float64(got) if not isinstance(got, np.ndarray) else got))
+    if dtype == "f32":
+        assert e["rel_inf"] <= F32_REL, e
+    else:
+        assert e["max_abs"] <= BF16_MAX and e["mean_abs"] <= BF16_MEAN and e["rel_l2"] <= BF16_RL2, e
+    return e
+
+
+def oracle_full(w, q, k, v, W):
+    return ora.forward(as_float64(q), as_float64(k), as_float64(v), w.fmap, w.eps, w.causal, as_float64(W))
+
+
+def check_workload(w, seed=None):
+    q, k, v, W = make_inputs(w, seed)
+    got = run_gpu(w, q, k, v, W)
+    return assert_parity(got, oracle_full(w, q, k, v, W), w.dtype)
+
+
+# ------------------------------------------------------------------ fp32 path
+
+def test_tiny_f32_against_definition():
+    """Tiny fp32 workload (B=1, H=2, N=256, D=64, elu+1) against the O(N^2)
+    definition itself."""
+    w = WORKLOADS["tiny_f32"]
+    q, k, v, _ = make_inputs(w)
+    got = run_gpu(w, q, k, v)
+    ref = ora.brute_force(as_float64(q), as_float64(k), as_float64(v), w.fmap, w.eps, False)
+    assert_parity(got, ref, "f32")
+
+
+F32_CASES = [
+    dict(N=1, D=64), dict(N=37, D=4), dict(N=300, D=36, fmap="relu"), dict(N=1000, D=128),
+    dict(N=129, D=64, causal=True), dict(N=700, D=128, causal=True, fmap="relu"),
+    dict(N=200, D=128, F=256), dict(N=333, D=64, F=256, causal=True),
+]
+
+
+@pytest.mark.parametrize("case", F32_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_f32_modes(case):
+    w = Workload("f32case", B=1, H=3, dtype="f32", seed=77, **case)
+    check_workload(w)
+
+
+def test_f32_shared_projection_and_empty_rows():
+    import torch
+    w = Workload("f32shared", B=2, H=2, N=150, D=32, F=256, dtype="f32", seed=5)
+    q, k, v, W = make_inputs(w)
+    W0 = W[0]
+    got = run_gpu(w, q, k, v, W0)
+    ref = ora.forward(as_float64(q), as_float64(k), as_float64(v), "elu", w.eps, False, as_float64(W0))
+    assert_parity(got, ref, "f32")
+    # relu with a query row <= 0 gives an all-zero row (0 / eps)
+    w2 = Workload("f32zero", B=1, H=1, N=40, D=16, fmap="relu", dtype="f32", seed=6)
+    q, k, v, _ = make_inputs(w2)
+    q[0, 0, 5] = -q[0, 0, 5].abs()
+    got = run_gpu(w2, q, k, v)
+    assert torch.all(got[0, 0, 5] == 0)
+
+
+# ------------------------------------------------------------------ bf16 path
+
+BF16_CASES = [
+    dict(N=1, D=128), dict(N=127, D=128), dict(N=129, D=128, fmap="relu"), dict(N=300, D=64),
+    dict(N=1000, D=64, fmap="relu"), dict(N=4607, D=128), dict(N=2048, D=128, B=3, H=5),
+]
+
+
+@pytest.mark.parametrize("case", BF16_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_noncausal_shapes(case):
+    case = dict(case)
+    B, H = case.pop("B", 1), case.pop("H", 2)
+    w = Workload("bf16case", B=B, H=H, seed=88, **case)
+    check_workload(w)
+
+
+def test_flux1024_full():
+    """Flux-1024 shape (B=1, H=24, N=4608, D=128, elu+1, unit-norm x sqrt(D)
+    queries and keys), every output element against the oracle."""
+    check_workload(WORKLOADS["flux1024"])
+
+
+def test_flux2048_cfg_full():
+    """Flux-2048 CFG pair (B=2, H=24, N=16896, D=128, relu), every element."""
+    check_workload(WORKLOADS["flux2048_cfg"])
+
+
+def test_bf16_deterministic_and_guard_bands():
+    import torch
+    w = WORKLOADS["flux1024"]
+    q, k, v, _ = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    n = q.numel()
+    pad = 4096
+    sentinel = torch.full((n + 2 * pad,), -12345.0, dtype=torch.bfloat16, device=dev)
+    out = sentinel[pad:pad + n].view_as(qd)
+    op(qd, kd, vd, out=out)
+    first = out.clone()
+    for _ in range(3):
+        op(qd, kd, vd, out=out)
+        assert torch.equal(out, first)
+    torch.cuda.synchronize()
+    assert torch.all(sentinel[:pad] == -12345.0) and torch.all(sentinel[pad + n:] == -12345.0)
+
+
+def test_bf16_weights_property():
+    """N <= D and V = I: output row i is the normalised weight row: entries
+    >= 0, rows sum to ~1 under elu+1, and agree with the oracle."""
+    import torch
+    w = Workload("weights", B=1, H=2, N=96, D=128, seed=9)
+    q, k, _, _ = make_inputs(w)
+    v = torch.zeros(1, 2, 96, 128)
+    v[0, :, :, :96] = torch.eye(96)
+    v = v.to(torch.bfloat16)
+    got = as_float64(run_gpu(w, q, k, v))
+    assert got.min() >= 0.0
+    np.testing.assert_allclose(got.sum(axis=-1), 1.0, atol=2e-2)
+    assert_parity(got, oracle_full(w, q, k, v, None), "bf16")
+
+
+def test_bf16_constant_values():
+    import torch
+    w = Workload("const", B=1, H=3, N=1500, D=64, seed=10)
+    q, k, _, _ = make_inputs(w)
+    c = torch.linspace(-2, 2, 64)
+    v = c.expand(1, 3, 1500, 64).contiguous().to(torch.bfloat16)
+    got = as_float64(run_gpu(w, q, k, v))
+    np.testing.assert_allclose(got, np.broadcast_to(as_float64(v[0, 0, 0]), got.shape), atol=2e-2)
+
+
+def test_host_buffer_entry_point_matches_device_path():
+    import torch
+    w = Workload("e2e", B=1, H=4, N=1000, D=128, seed=12)
+    q, k, v, _ = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, "elu", w.eps)
+    ref = op(q.to(dev), k.to(dev), v.to(dev)).cpu()
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    dq, dk, dv, do = (torch.empty_like(q, device=dev) for _ in range(4))
+    s = torch.cuda.current_stream().cuda_stream
+    st = la.la_forward_host(op.handle, qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), do.data_ptr(),
+                            1, 4, 1000, 128, 0, la.LA_PHI_ELU1, w.eps, 0, s)
+    assert st == la.LA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref)
