@@ -115,6 +115,29 @@ la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* 
  * wait; its output is undefined) or LA_ERR_CUDA. */
 la_status_t la_sync_status(la_handle_t handle, void* stream);
 
+/* Size of the static scratch array behind la_forward_noalloc (16 MiB).  A
+ * device holds it from the moment the library's code is loaded on it (at the
+ * latest, the first la_forward_noalloc call there) until the process exits. */
+#define LA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* For callers that cannot allocate device memory (no cudaMalloc, no pool of
+ * their own, nothing to bind with la_set_workspace): the bf16, non-causal,
+ * F = 0 forward of la_forward, with its scratch in a static device array of
+ * LA_NOALLOC_SCRATCH_BYTES inside this library instead of a workspace.  The
+ * pages have no counterpart; this entry point exists only for such callers.
+ * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward; D is 64
+ * or 128.  No handle is used and nothing is allocated, on host or device.
+ * Problems whose scratch would exceed the array return LA_ERR_WORKSPACE
+ * before anything is enqueued (the Flux-1024 shape B=1, H=24, N=4608, D=128
+ * needs about 11 MB).  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call on a device shares the one
+ * array and it keeps the last call's contents: calls that overlap on the GPU
+ * (different streams without ordering between them) race and give undefined
+ * results.  Device-side timeouts of this entry point are not reported. */
+la_status_t la_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                               int D, int feature_map, float eps, void* stream);
+
 /* Static description of a status code. */
 const char* la_status_string(la_status_t status);
 

@@ -25,7 +25,8 @@ STATUS_NAMES = {
 }
 
 EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
-            "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version")
+            "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version",
+            "la_forward_noalloc")
 
 
 class LAError(RuntimeError):
@@ -56,11 +57,12 @@ def lib():
     L.la_forward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
     L.la_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
     L.la_sync_status.argtypes = [vp, vp]
+    L.la_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_version.argtypes = []
     for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
-                 "la_forward_host", "la_sync_status"):
+                 "la_forward_host", "la_sync_status", "la_forward_noalloc"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -100,6 +102,12 @@ def la_forward_host(handle, q_host, k_host, v_host, out_host, dq, dk, dv, dout, 
                     feature_map, eps, causal, stream):
     return lib().la_forward_host(handle, q_host, k_host, v_host, out_host, dq, dk, dv, dout, B, H, N, D, F,
                                  feature_map, eps, int(causal), stream)
+
+
+def la_forward_noalloc(q, k, v, out, B, H, N, D, feature_map, eps, stream):
+    """bf16 non-causal forward whose scratch is a static device array inside the
+    library, for callers that cannot allocate device memory."""
+    return lib().la_forward_noalloc(q, k, v, out, B, H, N, D, feature_map, eps, stream)
 
 
 def la_sync_status(handle, stream):

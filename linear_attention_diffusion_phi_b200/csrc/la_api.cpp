@@ -167,6 +167,28 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+namespace la {
+
+void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p) {
+  la_handle_s h = {};
+  h.dtype = LA_BF16;
+  make_plan(&h, B, H, N, D, 0, fmap, eps, 0, num_sms, p);
+}
+
+bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,
+                          long long outer_stride_elems) {
+  return encode_bf16_3d(m, base, outer, rows, cols, outer_stride_elems, 128);
+}
+
+bool current_sm100(int* num_sms) {
+  DeviceInfo di;
+  if (!device_info(&di) || di.major != 10 || di.minor != 0) return false;
+  *num_sms = di.sms;
+  return true;
+}
+
+}  // namespace la
+
 extern "C" {
 
 la_status_t la_create(la_handle_t* handle, int dtype) {

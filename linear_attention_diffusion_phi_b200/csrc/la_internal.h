@@ -57,6 +57,15 @@ struct LaunchArgs {
   const CUtensorMap* tm_w;
 };
 
+// Host helpers defined in la_api.cpp for other host translation units.
+// Plan of a bf16 non-causal F = 0 problem (the caller validated the shape).
+void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p);
+// [outer, rows, cols] bf16 tensor map, 128-row x 64-column boxes, 128-byte swizzle.
+bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,
+                          long long outer_stride_elems);
+// SM count of the current device; false unless it is an sm_100 device.
+bool current_sm100(int* num_sms);
+
 // f32 CUDA-core path (all modes).
 cudaError_t launch_f32(const LaunchArgs& a);
 // bf16 tensor-core paths.

@@ -1,0 +1,51 @@
+"""la_forward_noalloc, the entry point for callers that cannot allocate device
+memory: its scratch is a static array inside the library.  It must give the
+same result as la_forward with a caller-owned workspace, call after call, even
+though every call reuses the same array.  (This file is collected last.)"""
+
+import numpy as np
+import pytest
+
+import linear_attention_diffusion_phi_b200 as la
+from linear_attention_diffusion_phi_b200 import build as la_build
+from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, Workload, as_float64, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX, BF16_MEAN = 2e-2, 2e-3
+
+
+def _close(a, b):
+    d = np.abs(as_float64(a) - as_float64(b))
+    assert d.max() <= BF16_MAX and d.mean() <= BF16_MEAN, (d.max(), d.mean())
+
+
+def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
+    import torch
+    la_build.build()
+    dev = torch.device("cuda:0")
+    s = torch.cuda.current_stream().cuda_stream
+    cases = [WORKLOADS["flux1024"], Workload("noalloc_relu64", B=2, H=3, N=1001, D=64, fmap="relu", seed=21)]
+    for w in cases:
+        q, k, v, _ = make_inputs(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps)
+        ref = op(qd, kd, vd).clone()
+        for _ in range(2):
+            out = torch.full_like(qd, float("nan"))
+            st = la.la_forward_noalloc(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(),
+                                       w.B, w.H, w.N, w.D, la.FEATURE_MAPS[w.fmap], w.eps, s)
+            assert st == la.LA_OK, la.la_status_string(st)
+            torch.cuda.synchronize()
+            _close(out.cpu(), ref.cpu())
+        op.close()
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    import torch
+    la_build.build()
+    dev = torch.device("cuda:0")
+    x = torch.empty(16, dtype=torch.bfloat16, device=dev)   # never read: rejected on the host
+    st = la.la_forward_noalloc(x.data_ptr(), x.data_ptr(), x.data_ptr(), x.data_ptr(),
+                               64, 24, 4608, 128, la.LA_PHI_ELU1, 1e-6, torch.cuda.current_stream().cuda_stream)
+    assert st == 4   # LA_ERR_WORKSPACE
