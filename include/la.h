@@ -115,10 +115,10 @@ la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* 
  * wait; its output is undefined) or LA_ERR_CUDA. */
 la_status_t la_sync_status(la_handle_t handle, void* stream);
 
-/* Size of the static scratch array behind la_forward_noalloc (16 MiB).  A
+/* Size of the static scratch array behind la_forward_noalloc (2 MiB).  A
  * device holds it from the moment the library's code is loaded on it (at the
  * latest, the first la_forward_noalloc call there) until the process exits. */
-#define LA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+#define LA_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
 
 /* For callers that cannot allocate device memory (no cudaMalloc, no pool of
  * their own, nothing to bind with la_set_workspace): the bf16, non-causal,
@@ -127,9 +127,10 @@ la_status_t la_sync_status(la_handle_t handle, void* stream);
  * pages have no counterpart; this entry point exists only for such callers.
  * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward; D is 64
  * or 128.  No handle is used and nothing is allocated, on host or device.
- * Problems whose scratch would exceed the array return LA_ERR_WORKSPACE
- * before anything is enqueued (the Flux-1024 shape B=1, H=24, N=4608, D=128
- * needs about 11 MB).  The first call on a device looks up the array's device
+ * The scratch this path needs (a status word and per-head barrier words,
+ * about 1 MiB) does not grow with N, so every supported shape fits; a plan
+ * that needed more than the array would return LA_ERR_WORKSPACE before
+ * anything is enqueued.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
  * call before any stream capture.  Every call on a device shares the one
  * array and it keeps the last call's contents: calls that overlap on the GPU

@@ -5,20 +5,31 @@
 // sequence into kv = phi(K)^T V and ksum = sum_j phi(k_j), then
 // out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).
 //
-// Three kernels, chained with programmatic dependent launch:
-//   kv_partial  grid (S, B*H): TMA streams 128-token K/V tiles of one N-split
-//               into shared memory, four warps apply phi to K in place and sum
-//               ksum, one thread issues tcgen05.mma  kv += phi(K_tile)^T V_tile
-//               into tensor memory; the fp32 partial is written to workspace.
-//   kv_combine  grid (B*H, F/8): sums the S partials in ascending order (no
-//               atomics, bitwise reproducible) and writes, per head, the bf16
-//               image of [kv | ksum | 0] laid out as the MMA's B operand.
-//   apply       persistent grid: per 128-query tile, TMA load, phi in place,
-//               one MMA [num | den] = phi(Q) [kv | ksum], epilogue
-//               out = num / (den + eps) rounded to bf16, TMA store.
+// One kernel.  Each head is served by a thread-block cluster of S CTAs (one
+// per SM); CTA r owns the r-th run of 128-token tiles of the head.
+//   phase 1  TMA streams the CTA's K and V tiles into a ring of shared-memory
+//            slots; eight warps apply phi to K in place; one thread issues
+//            tcgen05.mma  kv^T += V^T phi(K)  and  ksum^T += 1^T phi(K)  into
+//            tensor memory (fp32).
+//   combine  four warps copy the CTA's partial (kv | ksum)^T from tensor
+//            memory into its own shared memory, rounded to bf16 and already in
+//            the layout of the apply MMA's B operand; after a cluster
+//            handshake eight warps of every CTA sum their share of that image
+//            over the cluster's CTAs in ascending order (no atomics, so bitwise
+//            reproducible), reading the peers' shared memory, and store the
+//            sums into the shared memory of every CTA of the cluster
+//            (distributed shared memory, no global round trip).
+//   phase 2  the CTA's Q tiles (prefetched during the combine) get phi in
+//            place, one MMA per tile computes [num | den] = phi(Q) [kv | ksum],
+//            and four warps write out = num / (den + eps) as bf16 into the Q
+//            tile's own slot, which TMA stores to global memory.
+// S is the largest cluster size (<= 8) whose clusters for all heads can be
+// resident at once on this device.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "la_internal.h"
 #include "sm100.cuh"
@@ -29,306 +40,147 @@ namespace {
 constexpr uint32_t kBoxBytes = 128 * 128;   // one TMA box: 128 rows x 64 bf16 (128 B)
 
 template <int D>
-struct TileCfg {
+struct Cfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr uint32_t kTileBytes = 128u * D * 2u;    // 128 tokens x D bf16
-  static constexpr int kChunksPerRow = D / 8;               // 16-byte chunks per token row
-  static constexpr int kThreadsPerChunk = 128 / kChunksPerRow;
+  static constexpr uint32_t kSlotBytes = 128u * D * 2u;          // one 128-token tile
+  static constexpr int kNB = D + 16;                               // apply MMA N: values + den
+  // [kv | ksum | 0]^T as the apply MMA's B operand, K-major with the 128-byte
+  // swizzle: row n < D holds kv[.][n], row D holds ksum, rows above are zero;
+  // each row's D features are split in 64-feature k-atoms of kNB rows.
+  static constexpr uint32_t kBlobAtomBytes = kNB * 128;
+  static constexpr uint32_t kBlobBytes = (D / 64) * kBlobAtomBytes;
+  // This CTA's partial (kv | ksum)^T in bf16, same layout as the image (rows
+  // 0..D), read by the cluster's CTAs.
+  static constexpr uint32_t kStageBytes = kBlobBytes;
+  static constexpr uint32_t kOnesBytes = 2048;                     // A of the ksum MMA (64 x 16)
+  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr uint32_t kSmemBytes = kBlobBytes + kStageBytes + kOnesBytes + kSlots * kSlotBytes + 1024;
+  static constexpr uint32_t kAccStride = D == 128 ? 256 : 128;    // TMEM columns per accumulator
+  static constexpr uint32_t kTmemCols = 2 * kAccStride;
+  static constexpr int kPhiWarps = 8;
+  static constexpr int kPhiThreads = 32 * kPhiWarps;
+  static constexpr int kChunksPerRow = D / 8;                      // 16-byte chunks per token row
+  static constexpr int kThreadsPerChunk = kPhiThreads / kChunksPerRow;
   static constexpr int kRowsPerThread = 128 / kThreadsPerChunk;
+  static constexpr int kCombWarp0 = 2 + kPhiWarps;                 // 4 warps: partial, combine
+  static constexpr int kEpiWarp0 = kCombWarp0 + 4;                 // 4 warps: outputs
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 };
 
-// Byte offset of (row r, logical 16-byte chunk cc) inside a [128 x D] bf16 tile
-// stored as D/64 TMA boxes with the 128-byte swizzle.
+// Byte offset of (row r, logical 16-byte chunk cc) in a [128 x D] bf16 tile
+// held as D/64 TMA boxes with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t swz_off(int r, int cc) {
   return static_cast<uint32_t>((cc >> 3) * kBoxBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
 }
 
-// Apply phi to 8 bf16 values in place (one 16-byte chunk); returns the rounded
-// values as floats in y[] so that sums use exactly what the MMA will read.
+// phi on 8 bf16 values (one 16-byte chunk), branch-free and rounded once to
+// bf16.  elu(x)+1 = max(x, 0) + exp(min(x, 0)): for x > 0 the exponential is
+// exactly 1 and the bf16 add rounds x + 1 once; for x <= 0 the max is 0 and
+// the sum is the bf16-rounded exponential.  exp(y) = 2^(y log2 e) uses the
+// hardware ex2 on fp32.  relu = max(x, 0) is exact in bf16.
 template <int FMAP>
-__device__ __forceinline__ uint4 phi_chunk(uint4 x, float (&y)[8]) {
-  uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
-    float2 f = __bfloat1622float2(b);
-    __nv_bfloat162 r = __floats2bfloat162_rn(phi_fast<FMAP>(f.x), phi_fast<FMAP>(f.y));
-    float2 g = __bfloat1622float2(r);
-    y[2 * i] = g.x;
-    y[2 * i + 1] = g.y;
-    w[i] = *reinterpret_cast<uint32_t*>(&r);
+__device__ __forceinline__ uint32_t phi_pair(uint32_t w) {
+  const __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&w);
+  const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+  __nv_bfloat162 r = __hmax2(x, zero);
+  if (FMAP == 0) {
+    const float2 n = __bfloat1622float2(__hmin2(x, zero));
+    const __nv_bfloat162 e = __floats2bfloat162_rn(ex2_approx(n.x * kLog2e), ex2_approx(n.y * kLog2e));
+    r = __hadd2(r, e);
   }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// Lane 0 waits on the barrier, the result is broadcast so the warp stays
-// converged.  Returns false on timeout.
+template <int FMAP>
+__device__ __forceinline__ uint4 phi_chunk(uint4 x) {
+  return make_uint4(phi_pair<FMAP>(x.x), phi_pair<FMAP>(x.y), phi_pair<FMAP>(x.z), phi_pair<FMAP>(x.w));
+}
+
+// Lane 0 waits, the verdict is broadcast so the warp stays converged.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
   return ok != 0;
 }
 
-// =============================================================== kv_partial
-
-template <int D>
-struct PartialCfg : TileCfg<D> {
-  static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr uint32_t kStageBytes = 2 * TileCfg<D>::kTileBytes;   // K then V
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024;  // +1024 for alignment
-  static constexpr uint32_t kTmemCols = D;                             // fp32 accumulator D x D
-};
+// 16-byte load from a cluster CTA's shared memory.
+__device__ __forceinline__ void ld_cluster_v4(uint32_t cluster_addr, uint32_t (&v)[4]) {
+  asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(cluster_addr)
+               : "memory");
+}
 
 template <int D, int FMAP>
-__global__ void __launch_bounds__(192, 1)
-    kv_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      float* __restrict__ part, float* __restrict__ part_ksum, int* status, int N, int tiles,
-                      int tiles_per_split, int S) {
-  using C = PartialCfg<D>;
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
+    fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                 int* status, int N, int tiles, float eps) {
+  using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[C::kStages], phi_bar[C::kStages], empty_bar[C::kStages];
-  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t full[C::kSlots], ready[C::kSlots], empty[C::kSlots];
+  // Tensor-memory accumulators a = 0, 1: phase 1 uses accumulator 0 once
+  // (p1full / p1empty, consumed by the combine warps); phase-2 tile u uses
+  // accumulator u & 1 (accfull / accempty, consumed by the output warps).
+  // Separate barriers keep each barrier's phases consumed in order by one
+  // consumer, so parity waits cannot alias.
+  __shared__ __align__(8) uint64_t p1full, p1empty, accfull[2], accempty[2];
+  __shared__ __align__(8) uint64_t stage_ready, blob_ready;   // arrivals from every CTA of the cluster
   __shared__ uint32_t tmem_slot;
+  __shared__ int comb_flag, ep_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = blockIdx.x;
+  const int S = static_cast<int>(gridDim.x);   // CTAs per head == cluster size
+  const int rank = static_cast<int>(cluster_ctarank());
   const int bh = blockIdx.y;
-  const int tile0 = s * tiles_per_split;
-  const int ntile = min(tiles, tile0 + tiles_per_split) - tile0;
+  const int tile0 = rank * tiles / S;
+  const int T = (rank + 1) * tiles / S - tile0;   // >= 1 because S <= tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  // Let the combine kernel's blocks get scheduled; they wait for this grid.
-  pdl_launch_dependents();
+  uint8_t* blob = smem;
+  uint8_t* stage = blob + C::kBlobBytes;
+  uint8_t* ones = stage + C::kStageBytes;
+  uint8_t* slots = ones + C::kOnesBytes;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&phi_bar[i], 4);
-      mbar_init(&empty_bar[i], 1);
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&ready[i], C::kPhiWarps);
+      mbar_init(&empty[i], 1);
     }
-    mbar_init(&acc_bar, 1);
-    fence_mbarrier_init();
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-  }
-  if (warp == 1) {
-    tmem_alloc(&tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      for (int i = 0; i < ntile; ++i) {
-        const int st = i % C::kStages, round = i / C::kStages;
-        if (i >= C::kStages && !mbar_wait(&empty_bar[st], (round - 1) & 1, status)) break;
-        uint8_t* ks = smem + st * C::kStageBytes;
-        uint8_t* vs = ks + C::kTileBytes;
-        mbar_arrive_expect_tx(&full_bar[st], C::kStageBytes);
-        const int tok = (tile0 + i) * kTileTokens;
-#pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b) tma_load_3d(ks + b * kBoxBytes, &tm_k, &full_bar[st], 64 * b, tok, bh);
-#pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b) tma_load_3d(vs + b * kBoxBytes, &tm_v, &full_bar[st], 64 * b, tok, bh);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      // kv[f][n] += sum_t phi(K)[t][f] V[t][n]: A = phi(K)^T (M = D features,
-      // MN-major), B = V (N = D, MN-major), K = 16 tokens per instruction.
-      constexpr uint32_t idesc = idesc_bf16_f32(D, D, 1, 1);
-      for (int i = 0; i < ntile; ++i) {
-        const int st = i % C::kStages, round = i / C::kStages;
-        if (!mbar_wait(&phi_bar[st], round & 1, status)) break;
-        tc_fence_after();
-        const uint32_t ka = smem_u32(smem + st * C::kStageBytes);
-        const uint32_t va = ka + C::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < kTileTokens / 16; ++k) {
-          const uint64_t adesc = smem_desc_sw128(ka + k * 2048, kBoxBytes, 1024);
-          const uint64_t bdesc = smem_desc_sw128(va + k * 2048, kBoxBytes, 1024);
-          umma_bf16(tmem, adesc, bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
-        }
-        umma_commit(&empty_bar[st]);
-      }
-      umma_commit(&acc_bar);
-    }
-  } else {
-    // --------------------------------------------- phi on K, ksum, epilogue
-    const int pt = threadIdx.x - 64;    // 0..127
-    const int cc = pt / C::kThreadsPerChunk;
-    const int r0 = pt % C::kThreadsPerChunk;
-    float ks[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ks[e] = 0.f;
-    bool ok = true;
-    for (int i = 0; i < ntile && ok; ++i) {
-      const int st = i % C::kStages, round = i / C::kStages;
-      if (!warp_wait(&full_bar[st], round & 1, status)) {
-        ok = false;
-        break;
-      }
-      uint8_t* kt = smem + st * C::kStageBytes;
-      const int tok0 = (tile0 + i) * kTileTokens;
-#pragma unroll 4
-      for (int j = 0; j < C::kRowsPerThread; ++j) {
-        const int r = r0 + j * C::kThreadsPerChunk;
-        uint4* p = reinterpret_cast<uint4*>(kt + swz_off(r, cc));
-        float y[8];
-        uint4 x = phi_chunk<FMAP>(*p, y);
-        if (tok0 + r >= N) {   // rows past the sequence end contribute nothing
-          x = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = 0.f;
-        }
-        *p = x;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ks[e] += y[e];
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&phi_bar[st]);
-    }
-    // ksum: reduce the threads that share chunk column cc (consecutive lanes).
-#pragma unroll
-    for (int o = 1; o < C::kThreadsPerChunk; o <<= 1)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], o);
-    float* ksd = part_ksum + (static_cast<size_t>(bh) * S + s) * D;
-    if (r0 == 0) {
-      reinterpret_cast<float4*>(ksd + cc * 8)[0] = make_float4(ks[0], ks[1], ks[2], ks[3]);
-      reinterpret_cast<float4*>(ksd + cc * 8)[1] = make_float4(ks[4], ks[5], ks[6], ks[7]);
-    }
-    // Epilogue: TMEM lane = feature row (M = 128: row = lane; M = 64: rows
-    // 16q..16q+15 sit in lanes 32q..32q+15).
-    if (ok && warp_wait(&acc_bar, 0, status)) {
-      tc_fence_after();
-      const int q = warp & 3;
-      const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      const bool valid = (D == 128) || lane < 16;
-      const int f = (D == 128) ? 32 * q + lane : 16 * q + lane;
-      float* dst = part + ((static_cast<size_t>(bh) * S + s) * D + f) * D;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float v[32];
-        tmem_ld32(trow + c0, v);
-        tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
-}
-
-// =============================================================== kv_combine
-
-// Writes, for head bh and k-group g (features 8g..8g+7), the 128-byte-swizzled
-// MN-major image of rows [kv[f][0..D) | ksum[f] | 0 ...] of the apply MMA's B
-// operand.  One thread per 16-byte chunk.
-__global__ void __launch_bounds__(256) kv_combine_kernel(const float* __restrict__ part,
-                                                         const float* __restrict__ part_ksum,
-                                                         uint8_t* __restrict__ blobs, int D, int Fe, int S,
-                                                         size_t blob_bytes) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int bh = blockIdx.x, g = blockIdx.y;
-  const int atoms = blob_atoms(D);
-  const int chunks_per_row = atoms * 8;
-  const int t = threadIdx.x;
-  if (t >= 8 * chunks_per_row) return;
-  const int r = t / chunks_per_row, ch = t % chunks_per_row;
-  const int a = ch >> 3, c = ch & 7;
-  const int f = 8 * g + r;
-  const int n0 = 64 * a + 8 * c;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  if (n0 + 8 <= D) {
-    for (int s = 0; s < S; ++s) {
-      const float4* src =
-          reinterpret_cast<const float4*>(part + ((static_cast<size_t>(bh) * S + s) * Fe + f) * D + n0);
-      const float4 x0 = src[0], x1 = src[1];
-      acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
-      acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
-    }
-  } else if (n0 <= D && D < n0 + 8) {
-    for (int s = 0; s < S; ++s) acc[D - n0] += part_ksum[(static_cast<size_t>(bh) * S + s) * Fe + f];
-  }
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&b);
-  }
-  uint8_t* dst = blobs + static_cast<size_t>(bh) * blob_bytes + static_cast<size_t>(a) * Fe * 128 + g * 1024 +
-                 r * 128 + ((c ^ r) << 4);
-  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// ==================================================================== apply
-
-template <int D>
-struct ApplyCfg : TileCfg<D> {
-  static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kNB = D + 16;                       // MMA N: D value columns + den
-  static constexpr uint32_t kAccCols = D == 128 ? 256 : 128;
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;
-  static constexpr uint32_t kBlobBytes = blob_atoms(D) * D * 128;
-  static constexpr uint32_t kSmemBytes = kStages * TileCfg<D>::kTileBytes + kBlobBytes +
-                                         2 * TileCfg<D>::kTileBytes + 1024;
-};
-
-template <int D, int FMAP>
-__global__ void __launch_bounds__(320, 1)
-    apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                 const uint8_t* __restrict__ blobs, int* status, float eps, int tiles, long long total) {
-  using C = ApplyCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t qfull[C::kStages], qphi[C::kStages], qempty[C::kStages];
-  __shared__ __align__(8) uint64_t accfull[2], accempty[2], blobfull, blobempty;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int ep_abort;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qs = smem;
-  uint8_t* blob = qs + C::kStages * C::kTileBytes;
-  uint8_t* os = blob + C::kBlobBytes;
-
-  const long long per = total / gridDim.x, rem = total % gridDim.x;
-  const long long begin = blockIdx.x * per + min(static_cast<long long>(blockIdx.x), rem);
-  const int count = static_cast<int>(per + (blockIdx.x < rem ? 1 : 0));
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&qfull[i], 1);
-      mbar_init(&qphi[i], 4);
-      mbar_init(&qempty[i], 1);
-    }
+    mbar_init(&p1full, 1);
+    mbar_init(&p1empty, 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accfull[i], 1);
       mbar_init(&accempty[i], 4);
     }
-    mbar_init(&blobfull, 1);
-    mbar_init(&blobempty, 1);
+    mbar_init(&stage_ready, S);
+    mbar_init(&blob_ready, S);
     fence_mbarrier_init();
     prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_out);
-    ep_abort = 0;
+    comb_flag = 0;
+    ep_flag = 0;
   }
+  // A operand of the ksum MMA: 64 (m) x 16 (k) bf16, K-major without swizzle
+  // (core matrices of 8 rows x 16 bytes; m-groups 128 B apart, k-groups
+  // 1024 B apart); row m = 0 is all ones, the rest zero, so row 0 of the
+  // product is 1^T phi(K) = ksum^T.
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    const int off = 16 * i;
+    const bool one = ((off % 1024) / 128 == 0) && ((off % 128) / 16 == 0);
+    const uint32_t w = one ? 0x3F803F80u : 0u;
+    *reinterpret_cast<uint4*>(ones + off) = make_uint4(w, w, w, w);
+  }
+  // Rows D+1..kNB-1 of the operand image are the MMA's zero padding.
+  for (int i = threadIdx.x; i < (D / 64) * (C::kNB - D - 1) * 8; i += blockDim.x) {
+    const int a = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
+    const int n = D + 1 + rem / 8, c = rem % 8;
+    *reinterpret_cast<uint4*>(blob + a * C::kBlobAtomBytes + n * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(&tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -338,191 +190,364 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
+  // ------------------------------------------------------------ producer
+  // Slot sequence: K, V of each phase-1 tile, then the Q tiles.  The first
+  // round of slots is issued before the cluster handshake.
+  int seq = 0;
+  auto issue = [&](int upto) {
+    while (seq < upto) {
+      const int s = seq % C::kSlots, round = seq / C::kSlots;
+      if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, status)) return;
+      const CUtensorMap* m = seq >= 2 * T ? &tm_q : ((seq & 1) ? &tm_v : &tm_k);
+      const int tile = seq >= 2 * T ? seq - 2 * T : seq / 2;
+      uint8_t* dst = slots + s * C::kSlotBytes;
+      mbar_arrive_expect_tx(&full[s], C::kSlotBytes);
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b)
+        tma_load_3d(dst + b * kBoxBytes, m, &full[s], 64 * b, (tile0 + tile) * kTileTokens, bh);
+      ++seq;
+    }
+  };
+  // Every CTA's barriers exist (fence.mbarrier_init above) before any remote
+  // arrival: relaxed arrive, first loads, then the acquiring wait.
+  cluster_arrive_relaxed();
+  if (warp == 0 && lane == 0) issue(min(C::kSlots, 3 * T));
+  cluster_wait();
+
   if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      pdl_wait();   // the state images come from the previous kernel
-      long long cur = -1;
-      int nblob = 0;
-      for (int li = 0; li < count; ++li) {
-        const long long item = begin + li;
-        const int bh = static_cast<int>(item / tiles), tile = static_cast<int>(item % tiles);
-        if (bh != cur) {
-          if (nblob > 0 && !mbar_wait(&blobempty, (nblob - 1) & 1, status)) break;
-          mbar_arrive_expect_tx(&blobfull, C::kBlobBytes);
-          bulk_load(blob, blobs + static_cast<size_t>(bh) * C::kBlobBytes, C::kBlobBytes, &blobfull);
-          cur = bh;
-          ++nblob;
-        }
-        const int st = li % C::kStages, round = li / C::kStages;
-        if (li >= C::kStages && !mbar_wait(&qempty[st], (round - 1) & 1, status)) break;
-        mbar_arrive_expect_tx(&qfull[st], C::kTileBytes);
-        uint8_t* dst = qs + st * C::kTileBytes;
-#pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_3d(dst + b * kBoxBytes, &tm_q, &qfull[st], 64 * b, tile * kTileTokens, bh);
-      }
-    }
+    if (lane == 0) issue(3 * T);
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      // [num | den] (128 x (D+16)) = phi(Q) (128 x D, K-major) x [kv | ksum]
-      // (D x (D+16), MN-major image from kv_combine).
-      constexpr uint32_t idesc = idesc_bf16_f32(128, C::kNB, 0, 1);
-      const uint32_t ba = smem_u32(blob);
-      long long cur = -1;
-      int nblob = 0;
-      for (int li = 0; li < count; ++li) {
-        const long long item = begin + li;
-        const int bh = static_cast<int>(item / tiles);
-        if (bh != cur) {
-          if (nblob > 0) umma_commit(&blobempty);
-          if (!mbar_wait(&blobfull, nblob & 1, status)) break;
-          cur = bh;
-          ++nblob;
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(D, D, 1, 1);     // kv^T: M = D values, N = D features
+      constexpr uint32_t idesc_ks = idesc_bf16_f32(64, D, 0, 1);    // ksum^T: M = 64 (row 0 used)
+      constexpr uint32_t idesc_ap = idesc_bf16_f32(128, C::kNB, 0, 0);
+      const uint64_t ones_desc = smem_desc_noswz(smem_u32(ones), 1024, 128);
+      bool ok = true;
+      for (int t = 0; t < T; ++t) {
+        const int qk = 2 * t, qv = 2 * t + 1;
+        const int sk = qk % C::kSlots, sv = qv % C::kSlots;
+        if (!mbar_wait(&ready[sk], (qk / C::kSlots) & 1, status) ||
+            !mbar_wait(&ready[sv], (qv / C::kSlots) & 1, status)) {
+          ok = false;
+          break;
         }
-        const int st = li % C::kStages, round = li / C::kStages;
-        const int a = li & 1, ar = li >> 1;
-        if (!mbar_wait(&qphi[st], round & 1, status)) break;
-        if (li >= 2 && !mbar_wait(&accempty[a], (ar - 1) & 1, status)) break;
         tc_fence_after();
-        const uint32_t qa = smem_u32(qs + st * C::kTileBytes);
+        const uint32_t ka = smem_u32(slots + sk * C::kSlotBytes);
+        const uint32_t va = smem_u32(slots + sv * C::kSlotBytes);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t adesc = smem_desc_sw128(qa + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(ba + k * 2048, D * 128, 1024);
-          umma_bf16(tmem + a * C::kAccCols, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+        for (int k = 0; k < kTileTokens / 16; ++k) {
+          // kv^T: A = V^T (MN-major: values contiguous), B = phi(K) (MN-major:
+          // features contiguous); ksum^T: A = ones block, same B.
+          const uint64_t vdesc = smem_desc_sw128(va + k * 2048, kBoxBytes, 1024);
+          const uint64_t kdesc = smem_desc_sw128(ka + k * 2048, kBoxBytes, 1024);
+          const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
+          umma_bf16(tmem, vdesc, kdesc, idesc_kv, acc);
+          umma_bf16(tmem + D, ones_desc, kdesc, idesc_ks, acc);
         }
-        umma_commit(&qempty[st]);
-        umma_commit(&accfull[a]);
+        umma_commit(&empty[sk]);
+        umma_commit(&empty[sv]);
+      }
+      umma_commit(&p1full);
+      if (ok && mbar_wait_cluster(&blob_ready, 0, status)) {
+        fence_proxy_async_smem();   // the cluster's stores into `blob` feed the tensor core
+        const uint32_t ba = smem_u32(blob);
+        for (int u = 0; u < T; ++u) {
+          const int qq = 2 * T + u, s = qq % C::kSlots;
+          const int a = u & 1, ar = u >> 1;
+          bool got = mbar_wait(&ready[s], (qq / C::kSlots) & 1, status);
+          if (got && ar == 0 && a == 0) got = mbar_wait(&p1empty, 0, status);   // freed by the combine warps
+          if (got && ar > 0) got = mbar_wait(&accempty[a], (ar - 1) & 1, status);
+          if (!got) break;
+          tc_fence_after();
+          const uint32_t qa = smem_u32(slots + s * C::kSlotBytes);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            // A = phi(Q) and B = [kv | ksum]^T, both K-major (features contiguous).
+            const uint64_t adesc = smem_desc_sw128(qa + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(ba + (k >> 2) * C::kBlobAtomBytes + (k & 3) * 32, 16, 1024);
+            umma_bf16(tmem + a * C::kAccStride, adesc, bdesc, idesc_ap, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&accfull[a]);
+        }
       }
     }
-  } else if (warp < 6) {
-    // ----------------------------------------------------------- phi on Q
+  } else if (warp < C::kCombWarp0) {
+    // ------------------------------------- phi on K and Q; V passes through
+    // Every slot use, whatever it holds, completes one phase of full[] and one
+    // of ready[], so the phase parity of both follows the slot's round.
     const int pt = threadIdx.x - 64;
     const int cc = pt / C::kThreadsPerChunk;
     const int r0 = pt % C::kThreadsPerChunk;
-    for (int li = 0; li < count; ++li) {
-      const int st = li % C::kStages, round = li / C::kStages;
-      if (!warp_wait(&qfull[st], round & 1, status)) break;
-      uint8_t* qt = qs + st * C::kTileBytes;
+    for (int seq = 0; seq < 3 * T; ++seq) {
+      const bool in_kv = seq < 2 * T;
+      const bool is_v = in_kv && (seq & 1);
+      const int s = seq % C::kSlots, round = seq / C::kSlots;
+      if (!warp_wait(&full[s], round & 1, status)) break;
+      if (!is_v) {
+        uint8_t* tile = slots + s * C::kSlotBytes;
+        // key rows past the sequence end must not reach ksum
+        const int valid = in_kv ? min(kTileTokens, N - (tile0 + seq / 2) * kTileTokens) : kTileTokens;
 #pragma unroll 4
-      for (int j = 0; j < C::kRowsPerThread; ++j) {
-        const int r = r0 + j * C::kThreadsPerChunk;
-        uint4* p = reinterpret_cast<uint4*>(qt + swz_off(r, cc));
-        float y[8];
-        *p = phi_chunk<FMAP>(*p, y);
+        for (int j = 0; j < C::kRowsPerThread; ++j) {
+          const int r = r0 + j * C::kThreadsPerChunk;
+          uint4* p = reinterpret_cast<uint4*>(tile + swz_off(r, cc));
+          *p = r < valid ? phi_chunk<FMAP>(*p) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&qphi[st]);
+      if (lane == 0) mbar_arrive(&ready[s]);
     }
   } else {
-    // --------------------------------------------------------------- epilogue
-    const int q = warp & 3;
-    const int r = 32 * q + lane;                    // token row in the tile
-    const bool leader = threadIdx.x == 192;
-    for (int li = 0; li < count; ++li) {
-      const long long item = begin + li;
-      const int bh = static_cast<int>(item / tiles), tile = static_cast<int>(item % tiles);
-      const int a = li & 1, ar = li >> 1;
-      if (leader) {
-        if (!mbar_wait(&accfull[a], ar & 1, status)) ep_abort = 1;
-        bulk_wait_group_read<1>();                  // staging buffer li&1 is free again
-      }
+    // ------------------------------------------- combine and output warps
+    // Warps kCombWarp0.. (4) copy the partial to shared memory; then they and
+    // the four output warps sum the cluster's partials; then the output warps
+    // write the phase-2 results.
+    const int ct = threadIdx.x - 32 * C::kCombWarp0;   // 0..255
+    const bool comb = warp < C::kEpiWarp0;
+    const bool leader = ct == 0;
+    const int q = warp & 3;                             // TMEM lane quarter
+    if (comb) {
+      // (1) partial (kv | ksum)^T -> own shared memory, bf16, image layout
+      bool ok = true;
+      if (leader && !mbar_wait(&p1full, 0, status)) comb_flag = 1;
       named_bar_sync(1, 128);
-      if (ep_abort) break;
-      tc_fence_after();
-      const uint32_t trow = tmem + a * C::kAccCols + (static_cast<uint32_t>(32 * q) << 16);
-      const float den = tmem_ld1(trow + D);
-      tmem_wait_ld();
-      const float inv = 1.0f / (den + eps);
-      uint8_t* ob = os + a * C::kTileBytes;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float v[32];
-        tmem_ld32(trow + c0, v);
-        tmem_wait_ld();
+      if (comb_flag) ok = false;
+      if (ok) {
+        tc_fence_after();
+        auto put_row = [&](int n, const float* v, int c0) {   // 32 values of row n from column c0
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t w[4];
+          for (int j = 0; j < 4; ++j) {
+            uint32_t w[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * j + 2 * i] * inv, v[8 * j + 2 * i + 1] * inv);
-            w[i] = *reinterpret_cast<uint32_t*>(&b);
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+              w[e] = *reinterpret_cast<uint32_t*>(&b);
+            }
+            const int c = c0 / 8 + j;
+            *reinterpret_cast<uint4*>(stage + (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(ob + swz_off(r, c0 / 8 + j)) = make_uint4(w[0], w[1], w[2], w[3]);
+        };
+        const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
+        // kv^T: M = 128 -> row = lane; M = 64 -> rows 16q..16q+15 in lanes 32q..32q+15
+        const bool valid = (D == 128) || lane < 16;
+        const int n = (D == 128) ? 32 * q + lane : 16 * q + lane;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + tq + c0, v);
+          tmem_wait_ld();
+          if (valid) put_row(n, v, c0);
+        }
+        // ksum^T is row 0 of the M = 64 product: lane 0 of quarter 0
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + tq + D + c0, v);
+          tmem_wait_ld();
+          if (q == 0 && lane == 0) put_row(D, v, c0);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p1empty);
+        fence_acq_rel_cluster();
+        named_bar_sync(1, 128);
+        if (leader) {
+          for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stage_ready), p));
+          if (!mbar_wait_cluster(&stage_ready, 0, status)) comb_flag = 1;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[a]);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
-#pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b) tma_store_3d(&tm_out, ob + b * kBoxBytes, 64 * b, tile * kTileTokens, bh);
-        bulk_commit_group();
-      }
     }
-    if (leader) bulk_wait_group<0>();
+    // (2) chunks [i0, i1) of rows 0..D of the image: the sum over the
+    // cluster's staged partials, in ascending CTA order, stored into every
+    // CTA's image.  Two chunks per thread and pass, all loads in flight.
+    named_bar_sync(3, 256);
+    const bool ok2 = comb_flag == 0;
+    if (ok2) {
+      constexpr int kChunks = (D + 1) * (D / 8);
+      const int i0 = rank * kChunks / S, i1 = (rank + 1) * kChunks / S;
+      const uint32_t stage_base = smem_u32(stage), blob_base = smem_u32(blob);
+      for (int i = i0 + ct; i < i1; i += 2 * 256) {
+        uint32_t off[2];
+        bool has[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int ii = i + h * 256;
+          has[h] = ii < i1;
+          const int n = ii / (D / 8), c = ii % (D / 8);
+          off[h] = (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4);
+        }
+        float acc[2][8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+        for (int p0 = 0; p0 < S; p0 += 4) {
+          uint32_t w[2][4][4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (has[h] && p0 + j < S) ld_cluster_v4(mapa_shared(stage_base + off[h], p0 + j), w[h][j]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (has[h] && p0 + j < S) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[h][j][e]));
+                  acc[h][2 * e] += x.x;
+                  acc[h][2 * e + 1] += x.y;
+                }
+              }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!has[h]) continue;
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(acc[h][2 * e], acc[h][2 * e + 1]);
+            o[e] = *reinterpret_cast<uint32_t*>(&b);
+          }
+          const uint4 val = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int p = 0; p < S; ++p) st_cluster_v4(mapa_shared(blob_base + off[h], p), val);
+        }
+      }
+      fence_acq_rel_cluster();
+    }
+    named_bar_sync(3, 256);
+    if (leader && ok2)
+      for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&blob_ready), p));
+    if (!comb) {
+      // (3) outputs of the CTA's Q tiles
+      const bool eleader = threadIdx.x == 32 * C::kEpiWarp0;
+      int prev_slot = -1;
+      for (int u = 0; u < T; ++u) {
+        const int s = (2 * T + u) % C::kSlots;
+        const int a = u & 1, ar = u >> 1;
+        if (eleader && !mbar_wait(&accfull[a], ar & 1, status)) ep_flag = 1;
+        named_bar_sync(2, 128);
+        if (ep_flag) break;
+        tc_fence_after();
+        const uint32_t trow = tmem + a * C::kAccStride + (static_cast<uint32_t>(32 * q) << 16);
+        const int r = 32 * q + lane;   // token row within the tile
+        const float den = tmem_ld1(trow + D);
+        tmem_wait_ld();
+        const float inv = 1.0f / (den + eps);
+        uint8_t* ob = slots + s * C::kSlotBytes;   // the MMA is done with this Q tile
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(trow + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * jj + 2 * e] * inv, v[8 * jj + 2 * e + 1] * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&b);
+            }
+            *reinterpret_cast<uint4*>(ob + swz_off(r, c0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[a]);
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (eleader) {
+#pragma unroll
+          for (int b = 0; b < C::kBoxes; ++b)
+            tma_store_3d(&tm_out, ob + b * kBoxBytes, 64 * b, (tile0 + u) * kTileTokens, bh);
+          bulk_commit_group();
+          if (prev_slot >= 0) {   // the previous tile's store has read its slot: hand it back
+            bulk_wait_group_read<1>();
+            mbar_arrive(&empty[prev_slot]);
+          }
+        }
+        prev_slot = s;
+      }
+      if (eleader) bulk_wait_group<0>();
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  cluster_sync_all();   // no CTA leaves while the cluster may still address its shared memory
 }
 
+// Largest cluster size S <= min(8, tiles) for which B*H clusters fit on the
+// device at once (one wave), per device and kernel; 1 when none does.
 template <typename K>
-cudaError_t set_smem(K kernel, uint32_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+int pick_cluster(K kern, uint32_t smem, int threads, long long BH, int tiles) {
+  static std::mutex mu;
+  static int cache[64][9];
+  static bool have[64][9] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 1;
+  }
+  const int smax = tiles < 8 ? tiles : 8;
+  for (int s = smax; s >= 2; --s) {
+    int n;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (!have[dev][s]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(s), 1);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int m = 0;
+        if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
+          cudaGetLastError();
+          m = 0;
+        }
+        cache[dev][s] = m;
+        have[dev][s] = true;
+      }
+      n = cache[dev][s];
+    }
+    if (n >= BH) return s;
+  }
+  return 1;
 }
 
 template <int D, int FMAP>
 cudaError_t run(const LaunchArgs& a) {
+  using C = Cfg<D>;
   const Plan& p = *a.p;
-  float* part = reinterpret_cast<float*>(a.ws + p.off_partial);
-  float* part_ksum = reinterpret_cast<float*>(a.ws + p.off_ksum_partial);
-  uint8_t* blobs = reinterpret_cast<uint8_t*>(a.ws + p.off_blob);
+  auto kern = fused_kernel<D, FMAP>;
+  cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  const int S = pick_cluster(kern, C::kSmemBytes, C::kThreads, p.BH, p.tiles);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(p.BH));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = a.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
-  cudaError_t err;
-
-  {
-    auto kern = kv_partial_kernel<D, FMAP>;
-    if ((err = set_smem(kern, PartialCfg<D>::kSmemBytes)) != cudaSuccess) return err;
-    dim3 grid(p.splits, static_cast<unsigned>(p.BH));
-    kern<<<grid, 192, PartialCfg<D>::kSmemBytes, a.stream>>>(*a.tm_k, *a.tm_v, part, part_ksum, status, p.N,
-                                                             p.tiles, p.tiles_per_split, p.splits);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  }
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(p.BH), p.Fe / 8);
-    cfg.blockDim = dim3(256);
-    cfg.stream = a.stream;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, kv_combine_kernel, static_cast<const float*>(part),
-                             static_cast<const float*>(part_ksum), blobs, p.D, p.Fe, p.splits, p.blob_bytes);
-    if (err != cudaSuccess) return err;
-  }
-  {
-    auto kern = apply_kernel<D, FMAP>;
-    if ((err = set_smem(kern, ApplyCfg<D>::kSmemBytes)) != cudaSuccess) return err;
-    const long long total = p.BH * p.tiles;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(total < p.num_sms ? total : p.num_sms));
-    cfg.blockDim = dim3(320);
-    cfg.dynamicSmemBytes = ApplyCfg<D>::kSmemBytes;
-    cfg.stream = a.stream;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_out, static_cast<const uint8_t*>(blobs), status, p.eps,
-                             p.tiles, total);
-  }
-  return err;
+  return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
 }
 
 }  // namespace

@@ -106,6 +106,10 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
       final_bytes = static_cast<size_t>(BH) * p->Fe * D * 4;
       final_ksum_bytes = static_cast<size_t>(BH) * p->Fe * 4;
     }
+  } else if (!causal && F == 0) {
+    // One thread-block cluster per head; the cluster size is chosen at launch
+    // from the device's cluster occupancy.  The combine runs through
+    // distributed shared memory, so only the workspace header is used.
   } else {
     const int tiles = std::max(p->tiles, 1);
     const long long want = std::max<long long>(1, p->num_sms / BH);
@@ -118,7 +122,8 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
     blob_total = static_cast<size_t>(BH) * p->blob_bytes;
   }
   size_t off = 0;
-  p->off_status = off;        off += 256;
+  p->off_status = off;        off += la::kStatusBytes;
+  p->off_sync = off;          off += la::kSyncBytes;
   p->off_partial = off;       off = align256(off + partial_floats * 4);
   p->off_ksum_partial = off;  off = align256(off + ksum_floats * 4);
   p->off_final = off;         off = align256(off + final_bytes);
@@ -178,6 +183,26 @@ void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int nu
 bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,
                           long long outer_stride_elems) {
   return encode_bf16_3d(m, base, outer, rows, cols, outer_stride_elems, 128);
+}
+
+cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes) {
+  static std::mutex mu;
+  static const void* done_fn[256];
+  static int done_dev[256];
+  static int n_done = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done_fn[i] == kernel && done_dev[i] == dev) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (err == cudaSuccess && n_done < 256) {
+    done_fn[n_done] = kernel;
+    done_dev[n_done] = dev;
+    ++n_done;
+  }
+  return err;
 }
 
 bool current_sm100(int* num_sms) {
@@ -245,10 +270,11 @@ la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
     return LA_OK;
   }
   if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return LA_ERR_MISALIGNED;
-  if (bytes < 256) return LA_ERR_WORKSPACE;
-  // Clear the device status word once, so that later reads see only errors
-  // of calls made with this workspace.
-  if (cudaMemset(ptr, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+  if (bytes < la::kHeaderBytes) return LA_ERR_WORKSPACE;
+  // Clear the status word and the barrier words once: later reads see only
+  // errors of calls made with this workspace, and every barrier count starts
+  // (and, after each completed barrier, returns) at zero.
+  if (cudaMemset(ptr, 0, la::kHeaderBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }
@@ -347,7 +373,8 @@ la_status_t la_sync_status(la_handle_t h, void* stream) {
     return LA_ERR_CUDA;
   }
   if (word == 0) return LA_OK;
-  if (cudaMemset(h->ws, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+  // An abandoned wait can leave barrier counts mid-way: clear the header.
+  if (cudaMemset(h->ws, 0, la::kHeaderBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }

@@ -15,6 +15,12 @@ constexpr int kDeviceTimeout = 6;                            // == LA_ERR_TIMEOU
 
 constexpr int kTileTokens = 128;   // tokens per tensor-core tile (MMA M or K)
 
+// Workspace header: a 256-byte status area, then barrier words for up to
+// 65536 heads (16 bytes each).  Zeroed when the workspace is bound.
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kSyncBytes = 65536 * 16;
+constexpr size_t kHeaderBytes = kStatusBytes + kSyncBytes;
+
 // Everything la_forward decides on the host, shared with la_workspace_bytes.
 struct Plan {
   int dtype;       // 0 f32, 1 bf16
@@ -27,8 +33,9 @@ struct Plan {
   int tiles_per_split;   // in 128-token tiles (bf16) or tokens per split (f32, see seg_len)
   int seg_len;     // tokens per split/segment
   int num_sms;
+  int heads_per_cta;   // bf16 non-causal: heads whose splits one CTA owns (1 or 2)
   // workspace layout (byte offsets from the workspace base, 256-aligned)
-  size_t off_status, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
+  size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
   size_t blob_bytes;   // bf16 B-operand image per head
 };
 
@@ -65,6 +72,9 @@ bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, lon
                           long long outer_stride_elems);
 // SM count of the current device; false unless it is an sm_100 device.
 bool current_sm100(int* num_sms);
+
+// Raise a kernel's dynamic shared-memory limit once per device (thread-safe).
+cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes);
 
 // f32 CUDA-core path (all modes).
 cudaError_t launch_f32(const LaunchArgs& a);

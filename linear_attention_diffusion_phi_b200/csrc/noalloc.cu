@@ -73,9 +73,11 @@ extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const vo
   void* scratch = nullptr;
   if (!scratch_address(&scratch)) return LA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents; only the status word must
-  // start at zero (every other byte the kernels read is written first).
-  if (cudaMemsetAsync(static_cast<char*>(scratch) + p.off_status, 0, 256, s) != cudaSuccess) {
+  // The array keeps the previous call's contents; the status word and this
+  // problem's barrier words must start at zero (every other byte the kernels
+  // read is written first).
+  if (cudaMemsetAsync(static_cast<char*>(scratch), 0, p.off_sync + static_cast<size_t>(p.BH) * 16, s) !=
+      cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }

@@ -234,6 +234,15 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 // ------------------------------------------------------------- feature maps
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Hardware base-2 exponential (approximate, flushes subnormals to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // elu(x)+1 with alpha = 1 (x + 1 for x > 0, exp(x) otherwise), or relu.
 template <int FMAP>
 __device__ __forceinline__ float phi_fast(float x) {
@@ -244,6 +253,165 @@ __device__ __forceinline__ float phi_fast(float x) {
 __device__ __forceinline__ float phi_accurate(float x, int fmap) {
   if (fmap == 0) return x > 0.f ? x + 1.f : expf(x);
   return fmaxf(x, 0.f);
+}
+
+}  // namespace la
+
+namespace la {
+
+// ------------------------------------------------------------------ clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of a cluster CTA (address from mapa_shared), with
+// release semantics at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with acquire semantics at cluster scope (remote arrivals).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(status, kDeviceTimeout);
+      return false;
+    }
+  }
+}
+
+// 16-byte store into a cluster CTA's shared memory.
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+// Split whole-cluster barrier: a relaxed arrive (no ordering of this thread's
+// earlier accesses, so outstanding TMA loads do not delay it) and an acquiring
+// wait.  Every thread of every CTA of the cluster takes part.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// Whole-cluster barrier (every thread of every CTA of the cluster).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared-memory descriptor without swizzle (core matrices of 8 rows x 16 B).
+// lbo: byte distance between core matrices along K; sbo: along M/N.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;   // layout type 0: no swizzle
+}
+
+}  // namespace la
+
+namespace la {
+
+// ------------------------------------------- grid-wide head barriers (global)
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Split-phase form of grid_barrier: arrive returns the generation to wait on
+// (taken before arriving, so it cannot have moved yet); the last of the n
+// arrivals resets the count and advances the generation.
+__device__ __forceinline__ unsigned grid_arrive(unsigned* count, unsigned* gen, unsigned n) {
+  const unsigned g = ld_acquire_gpu(gen);
+  const unsigned arrived = atom_add_acq_rel_gpu(count, 1u);
+  if (arrived == n - 1) {
+    st_relaxed_gpu(count, 0u);
+    red_add_release_gpu(gen, 1u);
+  }
+  return g;
+}
+
+// Bounded wait until the generation has moved past g.
+__device__ __forceinline__ bool grid_wait(unsigned* gen, unsigned g, int* status) {
+  if (ld_acquire_gpu(gen) != g) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(gen) == g) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(status, kDeviceTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Sense-reversing barrier among the `n` CTAs that share (count, gen); called
+// by one thread per CTA once the CTA's writes are complete.  `count` returns
+// to 0 every time the barrier completes; `gen` only grows.  All n CTAs must be
+// resident at once (cooperative launch).  Bounded: gives up after
+// kWaitLimitNs, records LA_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned n, int* status) {
+  const unsigned g = ld_acquire_gpu(gen);
+  const unsigned arrived = atom_add_acq_rel_gpu(count, 1u);
+  if (arrived == n - 1) {
+    st_relaxed_gpu(count, 0u);
+    red_add_release_gpu(gen, 1u);
+    return true;
+  }
+  if (ld_acquire_gpu(gen) != g) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(gen) == g) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(status, kDeviceTimeout);
+      return false;
+    }
+  }
+  return true;
 }
 
 }  // namespace la

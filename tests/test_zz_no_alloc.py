@@ -41,11 +41,21 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
         op.close()
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+def test_noalloc_rejects_bad_arguments_before_launching():
+    """Every rejection here happens on the host, before anything is enqueued,
+    so the (deliberately tiny) buffer is never read."""
     import torch
     la_build.build()
     dev = torch.device("cuda:0")
-    x = torch.empty(16, dtype=torch.bfloat16, device=dev)   # never read: rejected on the host
-    st = la.la_forward_noalloc(x.data_ptr(), x.data_ptr(), x.data_ptr(), x.data_ptr(),
-                               64, 24, 4608, 128, la.LA_PHI_ELU1, 1e-6, torch.cuda.current_stream().cuda_stream)
-    assert st == 4   # LA_ERR_WORKSPACE
+    x = torch.empty(64, dtype=torch.bfloat16, device=dev)
+    p = x.data_ptr()
+    s = torch.cuda.current_stream().cuda_stream
+    call = la.la_forward_noalloc
+    assert call(0, p, p, p, 1, 2, 128, 128, la.LA_PHI_ELU1, 1e-6, s) == 1         # null pointer
+    assert call(p + 2, p, p, p, 1, 2, 128, 128, la.LA_PHI_ELU1, 1e-6, s) == 3     # misaligned
+    assert call(p, p, p, p, 1, 2, 128, 96, la.LA_PHI_ELU1, 1e-6, s) == 2          # D not 64 / 128
+    assert call(p, p, p, p, 1, 2, 128, 128, 5, 1e-6, s) == 1                      # feature map
+    assert call(p, p, p, p, 1, 2, 128, 128, la.LA_PHI_ELU1, -1.0, s) == 1        # eps < 0
+    assert call(p, p, p, p, 300, 300, 128, 128, la.LA_PHI_ELU1, 1e-6, s) == 2    # B*H over the grid limit
+    assert call(p, p, p, p, 1, 2, 0, 128, la.LA_PHI_ELU1, 1e-6, s) == 0          # empty: nothing to do
+    torch.cuda.synchronize()
