@@ -53,7 +53,13 @@ struct Cfg {
   // 0..D), read by the cluster's CTAs.
   static constexpr uint32_t kStageBytes = kBlobBytes;
   static constexpr uint32_t kOnesBytes = 2048;                     // A of the ksum MMA (64 x 16)
-  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr int kSlots = D == 128 ? 4 : 8;                 // ring of tile slots
+  // During phase 1 the image and staging regions are idle; where a tile fits
+  // in them they serve as two more K/V slots.
+  static constexpr int kExtra = (kBlobBytes >= kSlotBytes) ? 2 : 0;
+  static constexpr int kRing1 = kSlots + kExtra;                   // phase-1 ring (K, V tiles)
+  // Phase 2 adds the staging region once the cluster has read it.
+  static constexpr int kRing2 = kSlots + kExtra / 2;
   static constexpr uint32_t kSmemBytes = kBlobBytes + kStageBytes + kOnesBytes + kSlots * kSlotBytes + 1024;
   static constexpr uint32_t kAccStride = D == 128 ? 256 : 128;    // TMEM columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccStride;
@@ -119,7 +125,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                  int* status, int N, int tiles, float eps) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[C::kSlots], ready[C::kSlots], empty[C::kSlots];
+  __shared__ __align__(8) uint64_t full[C::kRing1], ready[C::kRing1], empty[C::kRing1];
   // Tensor-memory accumulators a = 0, 1: phase 1 uses accumulator 0 once
   // (p1full / p1empty, consumed by the combine warps); phase-2 tile u uses
   // accumulator u & 1 (accfull / accempty, consumed by the output warps).
@@ -141,9 +147,22 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   uint8_t* stage = blob + C::kBlobBytes;
   uint8_t* ones = stage + C::kStageBytes;
   uint8_t* slots = ones + C::kOnesBytes;
+  // Physical slots 0..kSlots-1 are the ring, kSlots and kSlots+1 the image
+  // and staging regions.  Phase-1 use i (K, V of tile i / 2) takes slot
+  // i % kRing1; phase-2 use u (Q tile u) takes ring2(u % kRing2), the ring
+  // plus the staging region.  Every use of a slot completes one phase of its
+  // full / ready / empty barriers, so a use's phase parity is the number of
+  // earlier uses of that slot.
+  auto slot_ptr = [&](int phys) {
+    return phys < C::kSlots ? slots + phys * C::kSlotBytes : (phys == C::kSlots ? blob : stage);
+  };
+  auto uses1 = [&](int phys) { return (2 * T + C::kRing1 - 1 - phys) / C::kRing1; };   // phase-1 uses
+  auto ring2 = [&](int j) { return j < C::kSlots ? j : C::kSlots + 1; };
+  auto q_slot = [&](int u) { return ring2(u % C::kRing2); };
+  auto q_round = [&](int u) { return uses1(ring2(u % C::kRing2)) + u / C::kRing2; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kSlots; ++i) {
+    for (int i = 0; i < C::kRing1; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&ready[i], C::kPhiWarps);
       mbar_init(&empty[i], 1);
@@ -194,13 +213,21 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // Slot sequence: K, V of each phase-1 tile, then the Q tiles.  The first
   // round of slots is issued before the cluster handshake.
   int seq = 0;
+  bool staging_free = false;
   auto issue = [&](int upto) {
     while (seq < upto) {
-      const int s = seq % C::kSlots, round = seq / C::kSlots;
+      const bool p1 = seq < 2 * T;
+      const int s = p1 ? seq % C::kRing1 : q_slot(seq - 2 * T);
+      const int round = p1 ? seq / C::kRing1 : q_round(seq - 2 * T);
       if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, status)) return;
-      const CUtensorMap* m = seq >= 2 * T ? &tm_q : ((seq & 1) ? &tm_v : &tm_k);
-      const int tile = seq >= 2 * T ? seq - 2 * T : seq / 2;
-      uint8_t* dst = slots + s * C::kSlotBytes;
+      if (!p1 && s == C::kSlots + 1 && !staging_free) {
+        // the staging region is read by the whole cluster until the image is complete
+        if (!mbar_wait_cluster(&blob_ready, 0, status)) return;
+        staging_free = true;
+      }
+      const CUtensorMap* m = p1 ? ((seq & 1) ? &tm_v : &tm_k) : &tm_q;
+      const int tile = p1 ? seq / 2 : seq - 2 * T;
+      uint8_t* dst = slot_ptr(s);
       mbar_arrive_expect_tx(&full[s], C::kSlotBytes);
 #pragma unroll
       for (int b = 0; b < C::kBoxes; ++b)
@@ -211,7 +238,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // Every CTA's barriers exist (fence.mbarrier_init above) before any remote
   // arrival: relaxed arrive, first loads, then the acquiring wait.
   cluster_arrive_relaxed();
-  if (warp == 0 && lane == 0) issue(min(C::kSlots, 3 * T));
+  if (warp == 0 && lane == 0) issue(min(C::kRing1, 2 * T));
   cluster_wait();
 
   if (warp == 0) {
@@ -226,15 +253,15 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       bool ok = true;
       for (int t = 0; t < T; ++t) {
         const int qk = 2 * t, qv = 2 * t + 1;
-        const int sk = qk % C::kSlots, sv = qv % C::kSlots;
-        if (!mbar_wait(&ready[sk], (qk / C::kSlots) & 1, status) ||
-            !mbar_wait(&ready[sv], (qv / C::kSlots) & 1, status)) {
+        const int sk = qk % C::kRing1, sv = qv % C::kRing1;
+        if (!mbar_wait(&ready[sk], (qk / C::kRing1) & 1, status) ||
+            !mbar_wait(&ready[sv], (qv / C::kRing1) & 1, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ka = smem_u32(slots + sk * C::kSlotBytes);
-        const uint32_t va = smem_u32(slots + sv * C::kSlotBytes);
+        const uint32_t ka = smem_u32(slot_ptr(sk));
+        const uint32_t va = smem_u32(slot_ptr(sv));
 #pragma unroll
         for (int k = 0; k < kTileTokens / 16; ++k) {
           // kv^T: A = V^T (MN-major: values contiguous), B = phi(K) (MN-major:
@@ -253,14 +280,14 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         fence_proxy_async_smem();   // the cluster's stores into `blob` feed the tensor core
         const uint32_t ba = smem_u32(blob);
         for (int u = 0; u < T; ++u) {
-          const int qq = 2 * T + u, s = qq % C::kSlots;
+          const int s = q_slot(u);
           const int a = u & 1, ar = u >> 1;
-          bool got = mbar_wait(&ready[s], (qq / C::kSlots) & 1, status);
+          bool got = mbar_wait(&ready[s], q_round(u) & 1, status);
           if (got && ar == 0 && a == 0) got = mbar_wait(&p1empty, 0, status);   // freed by the combine warps
           if (got && ar > 0) got = mbar_wait(&accempty[a], (ar - 1) & 1, status);
           if (!got) break;
           tc_fence_after();
-          const uint32_t qa = smem_u32(slots + s * C::kSlotBytes);
+          const uint32_t qa = smem_u32(slot_ptr(s));
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             // A = phi(Q) and B = [kv | ksum]^T, both K-major (features contiguous).
@@ -282,10 +309,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     for (int seq = 0; seq < 3 * T; ++seq) {
       const bool in_kv = seq < 2 * T;
       const bool is_v = in_kv && (seq & 1);
-      const int s = seq % C::kSlots, round = seq / C::kSlots;
+      const int s = in_kv ? seq % C::kRing1 : q_slot(seq - 2 * T);
+      const int round = in_kv ? seq / C::kRing1 : q_round(seq - 2 * T);
       if (!warp_wait(&full[s], round & 1, status)) break;
       if (!is_v) {
-        uint8_t* tile = slots + s * C::kSlotBytes;
+        uint8_t* tile = slot_ptr(s);
         // key rows past the sequence end must not reach ksum
         const int valid = in_kv ? min(kTileTokens, N - (tile0 + seq / 2) * kTileTokens) : kTileTokens;
 #pragma unroll 4
@@ -349,10 +377,19 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           tmem_wait_ld();
           if (q == 0 && lane == 0) put_row(D, v, c0);
         }
+        if (C::kExtra) {   // the image region held K/V tiles: restore its zero padding rows
+          for (int i = ct; i < (D / 64) * (C::kNB - D - 1) * 8; i += 128) {
+            const int a = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
+            *reinterpret_cast<uint4*>(blob + a * C::kBlobAtomBytes + (D + 1 + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p1empty);
-        fence_acq_rel_cluster();
+        // The CTA barrier orders every thread's staging stores before the
+        // leader's release-arrive at cluster scope (release is cumulative).
         named_bar_sync(1, 128);
         if (leader) {
           for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stage_ready), p));
@@ -418,7 +455,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           for (int p = 0; p < S; ++p) st_cluster_v4(mapa_shared(blob_base + off[h], p), val);
         }
       }
-      fence_acq_rel_cluster();
     }
     named_bar_sync(3, 256);
     if (leader && ok2)
@@ -428,7 +464,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       const bool eleader = threadIdx.x == 32 * C::kEpiWarp0;
       int prev_slot = -1;
       for (int u = 0; u < T; ++u) {
-        const int s = (2 * T + u) % C::kSlots;
+        const int s = q_slot(u);
         const int a = u & 1, ar = u >> 1;
         if (eleader && !mbar_wait(&accfull[a], ar & 1, status)) ep_flag = 1;
         named_bar_sync(2, 128);
@@ -439,7 +475,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         const float den = tmem_ld1(trow + D);
         tmem_wait_ld();
         const float inv = 1.0f / (den + eps);
-        uint8_t* ob = slots + s * C::kSlotBytes;   // the MMA is done with this Q tile
+        uint8_t* ob = slot_ptr(s);   // the MMA is done with this Q tile
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           float v[32];
