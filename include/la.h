@@ -95,7 +95,7 @@ la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
  * la_feature_map_t; eps >= 0; causal is 0 or 1.
  * Supported: LA_F32: D <= 128, D % 4 == 0, F in {0, 256}.
  *            LA_BF16: D in {64, 128}; F in {0, 256} with D = 128 when F > 0;
- *            causal with F = 0.
+ *            causal with F = 0 and D = 64.
  * The result is deterministic: the same arguments give bitwise the same out. */
 la_status_t la_forward(la_handle_t handle, const void* q, const void* k, const void* v,
                        void* out, int B, int H, int N, int D, int F, int feature_map,

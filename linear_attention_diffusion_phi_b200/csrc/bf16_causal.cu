@@ -1,10 +1,553 @@
-// bf16_causal.cu -- tcgen05 tensor-core path for causal phi attention.
+// bf16_causal.cu -- tcgen05 tensor-core path for causal phi attention, bf16
+// storage and fp32 accumulation, D = 64, F = 0.
+//
+// Method (page "NNT Define Linear Attention", "The inputs": with causal set,
+// a token attends only to itself and earlier tokens; "How it works":
+// kv = phi(K)^T V and the normaliser 1/(phi(Q) . sum phi(K) + eps)).  Query i
+// sees keys j <= i:
+//   out_i = phi(q_i)^T S_i / (phi(q_i) . z_i + eps),
+//   S_i = sum_{j<=i} phi(k_j) v_j^T,  z_i = sum_{j<=i} phi(k_j).
+// Each head's sequence is cut into `splits` segments of whole 128-token
+// chunks, one CTA per (segment, head):
+//   causal_state_kernel  the sum S_seg^T, z_seg^T of every segment but the
+//                        last, as one MMA per 16 tokens: [V | 1]^T phi(K)
+//                        (M = 128: 64 value rows, a row of ones, zeros);
+//   causal_chunk_kernel  the segment's starting state is the sum of the
+//                        earlier segments' states (ascending order, fp32);
+//                        then chunk by chunk:
+//                          P  = phi(Q_c) phi(K_c)^T           (128 x 128)
+//                          Pm = P with j > i zeroed, bf16; r_i = sum_j Pm_ij
+//                          O  = phi(Q_c) [S_c | z_c] + Pm V_c  (numerator,
+//                               column 64: phi(q_i) . z_c)
+//                          out_i = O_i[0:64] / (O_i[64] + r_i + eps)
+//                          S_{c+1} = S_c + [V_c | 1]^T phi(K_c)
+//                        with the running state in fp32 registers of four
+//                        warps and each chunk's increment in tensor memory.
+// The chunk length (128) is a performance choice; the result depends on it
+// only through rounding.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "bf16_common.cuh"
 #include "la_internal.h"
+#include "sm100.cuh"
 
 namespace la {
+namespace {
 
-cudaError_t launch_bf16_causal(const LaunchArgs&) { return cudaErrorNotSupported; }
+constexpr int kD = 64;
+constexpr uint32_t kTile = 128u * kD * 2u;     // one 128-token tile of Q, K or V: 16 KB (one TMA box)
+constexpr int kStateRows = kD + 1;             // S^T rows, then z^T
+constexpr int kStateFloats = kStateRows * kD;  // per segment, fp32, row-major [65][64]
+constexpr int kImgRows = kD + 16;              // B operand [S | z | 0]^T: N = 80
+constexpr uint32_t kImgBytes = kImgRows * 128;
+
+// A-operand atom of ones: [128 tokens x 64] bf16 in the MN-major 128-byte
+// swizzled layout; element 0 of every token row is 1, the rest 0.  Placed as
+// the second M atom after a V tile, [V | ones]^T phi(K) has z^T in row 64.
+__device__ __forceinline__ void fill_ones_atom(uint8_t* p) {
+  for (int i = threadIdx.x; i < static_cast<int>(kTile / 16); i += blockDim.x) {
+    const int t = i >> 3, stored = i & 7;      // token row, stored 16-byte chunk
+    const uint32_t w = (stored == (t & 7)) ? 0x3F80u : 0u;   // logical chunk 0 lives at t & 7
+    *reinterpret_cast<uint4*>(p + i * 16) = make_uint4(w, 0u, 0u, 0u);
+  }
+}
+
+// phi on the 128 x 64 tile the 128 calling threads share (rows >= valid -> 0).
+template <int FMAP>
+__device__ __forceinline__ void phi_tile(uint8_t* tile, int pt, int valid) {
+  const int cc = pt >> 4, r0 = pt & 15;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int r = r0 + 16 * j;
+    uint4* p = reinterpret_cast<uint4*>(tile + swz_off(r, cc));
+    *p = r < valid ? phi_chunk<FMAP>(*p) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// ================================================= kernel 1: segment states
+
+constexpr int kStSlots = 8;
+constexpr uint32_t kStSmem = kStSlots * kTile + kTile + 1024;
+
+template <int FMAP>
+__global__ void __launch_bounds__(192, 1)
+    causal_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        float* __restrict__ state, int* status, int tps, int nseg) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kStSlots], ready[kStSlots], empty[kStSlots], accfull;
+  __shared__ uint32_t tmem_slot;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = blockIdx.x, bh = blockIdx.y;
+  const int tile0 = seg * tps, T = tps;   // never the last segment: always whole and inside N
+  uint8_t* slots = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ones = slots + kStSlots * kTile;   // above every slot: a positive atom stride
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&ready[i], 4);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(&accfull, 1);
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  fill_ones_atom(ones);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // producer: K_0, V_0, K_1, V_1, ...
+    if (lane == 0) {
+      for (int q = 0; q < 2 * T; ++q) {
+        const int s = q % kStSlots, round = q / kStSlots;
+        if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(&full[s], kTile);
+        tma_load_3d(slots + s * kTile, (q & 1) ? &tm_v : &tm_k, &full[s], 0, (tile0 + q / 2) * kTileTokens, bh);
+      }
+    }
+  } else if (warp == 1) {
+    // S'^T (128 x 64) += [V | ones]^T phi(K): A MN-major (atoms V, ones), B MN-major
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kD, 1, 1);
+      const uint32_t ones_a = smem_u32(ones);
+      for (int t = 0; t < T; ++t) {
+        const int qk = 2 * t, qv = qk + 1, sk = qk % kStSlots, sv = qv % kStSlots;
+        if (!mbar_wait(&ready[sk], (qk / kStSlots) & 1, status) ||
+            !mbar_wait(&ready[sv], (qv / kStSlots) & 1, status))
+          break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(slots + sk * kTile), va = smem_u32(slots + sv * kTile);
+#pragma unroll
+        for (int k = 0; k < kTileTokens / 16; ++k)
+          umma_bf16(tmem, smem_desc_sw128(va + k * 2048, ones_a - va, 1024),
+                    smem_desc_sw128(ka + k * 2048, kTile, 1024), idesc, (t > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[sk]);
+        umma_commit(&empty[sv]);
+      }
+      umma_commit(&accfull);
+    }
+  } else {
+    // phi on K, V passes through; then the readout of the state
+    const int pt = threadIdx.x - 64;
+    bool ok = true;
+    for (int q = 0; q < 2 * T; ++q) {
+      const int s = q % kStSlots;
+      if (!warp_wait(&full[s], (q / kStSlots) & 1, status)) {
+        ok = false;
+        break;
+      }
+      if (!(q & 1)) {
+        phi_tile<FMAP>(slots + s * kTile, pt, kTileTokens);
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[s]);
+    }
+    if (ok && warp_wait(&accfull, 0, status)) {
+      tc_fence_after();
+      const int qd = warp & 3, row = 32 * qd + lane;   // TMEM lane = row of S'^T
+      float* dst = state + (static_cast<size_t>(bh) * nseg + seg) * kStateFloats + row * kD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + c0, v);
+        tmem_wait_ld();
+        if (row < kStateRows) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 64);
+}
+
+// ====================================================== kernel 2: the chunks
+
+// Shared memory: Q ring of 3 tiles, K/V ring of 2 chunks, masked P (two
+// buffers of 32 KB), state images (two of 10 KB), the ones atom.
+constexpr int kQSlots = 3;
+constexpr int kSlots = kQSlots + 4;
+constexpr uint32_t kPmBytes = 2 * kBoxBytes;   // [128 x 128] bf16 as two 64-column boxes
+constexpr uint32_t kChSmem = kSlots * kTile + 2 * kPmBytes + 2 * kImgBytes + kTile + 1024;
+// Tensor-memory columns.
+constexpr uint32_t kColP = 0;        // P: two buffers of 128
+constexpr uint32_t kColO = 256;      // O: two buffers of 80, 96 apart
+constexpr uint32_t kOStride = 96;
+constexpr uint32_t kColD = 448;      // increment [V | 1]^T phi(K): 64 columns
+constexpr int kChThreads = 576;      // producer, MMA, 4 phi, 4 P, 4 state, 4 output warps
+
+__device__ __forceinline__ int q_slot(int c) { return c % kQSlots; }
+__device__ __forceinline__ int k_slot(int c) { return kQSlots + 2 * (c & 1); }
+__device__ __forceinline__ int v_slot(int c) { return kQSlots + 2 * (c & 1) + 1; }
+__device__ __forceinline__ uint32_t q_par(int c) { return static_cast<uint32_t>((c / kQSlots) & 1); }
+__device__ __forceinline__ uint32_t kv_par(int c) { return static_cast<uint32_t>((c >> 1) & 1); }
+
+template <int FMAP>
+__global__ void __launch_bounds__(kChThreads, 1)
+    causal_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                        const float* __restrict__ state, int* status, int N, int tiles, int tps, int nseg,
+                        float eps) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kSlots], ready[kSlots], empty[kSlots];
+  __shared__ __align__(8) uint64_t pfull[2], pempty[2], pmready[2], pmfree[2];
+  __shared__ __align__(8) uint64_t ofull[2], oempty[2], imgready[2], imgfree[2], dfull, dfree;
+  __shared__ float rowsum[4][128];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int flag_p, flag_s, flag_e;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = blockIdx.x, bh = blockIdx.y;
+  const int tile0 = seg * tps;
+  const int C = min(tiles, tile0 + tps) - tile0;   // chunks of this segment, >= 1
+  uint8_t* slots = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* pm = slots + kSlots * kTile;
+  uint8_t* img = pm + 2 * kPmBytes;
+  uint8_t* ones = img + 2 * kImgBytes;             // above every slot: a positive atom stride
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&ready[i], 4);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&pfull[i], 1);
+      mbar_init(&pempty[i], 4);
+      mbar_init(&pmready[i], 4);
+      mbar_init(&pmfree[i], 1);
+      mbar_init(&ofull[i], 1);
+      mbar_init(&oempty[i], 4);
+      mbar_init(&imgready[i], 4);
+      mbar_init(&imgfree[i], 1);
+    }
+    mbar_init(&dfull, 1);
+    mbar_init(&dfree, 4);
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_out);
+    flag_p = flag_s = flag_e = 0;
+  }
+  fill_ones_atom(ones);
+  // image rows 65..79 are the MMA's zero padding, in both buffers
+  constexpr int kPadChunks = (kImgRows - kStateRows) * 8;
+  for (int i = threadIdx.x; i < 2 * kPadChunks; i += blockDim.x) {
+    const int b = i / kPadChunks, rem = i % kPadChunks;
+    *reinterpret_cast<uint4*>(img + b * kImgBytes + (kStateRows + rem / 8) * 128 + (rem % 8) * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int c = 0; c < C; ++c) {
+        const int row = (tile0 + c) * kTileTokens;
+        const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
+        if (c >= kQSlots && !mbar_wait(&empty[sq], q_par(c) ^ 1u, status)) break;
+        mbar_arrive_expect_tx(&full[sq], kTile);
+        tma_load_3d(slots + sq * kTile, &tm_q, &full[sq], 0, row, bh);
+        if (c >= 2 && !mbar_wait(&empty[sk], kv_par(c) ^ 1u, status)) break;
+        mbar_arrive_expect_tx(&full[sk], kTile);
+        tma_load_3d(slots + sk * kTile, &tm_k, &full[sk], 0, row, bh);
+        if (c >= 2 && !mbar_wait(&empty[sv], kv_par(c) ^ 1u, status)) break;
+        mbar_arrive_expect_tx(&full[sv], kTile);
+        tma_load_3d(slots + sv * kTile, &tm_v, &full[sv], 0, row, bh);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);        // phi(Q) phi(K)^T
+      constexpr uint32_t id_qs = idesc_bf16_f32(128, kImgRows, 0, 0);  // phi(Q) [S | z | 0]
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);        // Pm V
+      constexpr uint32_t id_d = idesc_bf16_f32(128, kD, 1, 1);         // [V | 1]^T phi(K)
+      const uint32_t ones_a = smem_u32(ones);
+      for (int c = 0; c < C; ++c) {
+        const int b = c & 1, r2 = c >> 1;
+        const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
+        const uint32_t qa = smem_u32(slots + sq * kTile);
+        const uint32_t ka = smem_u32(slots + sk * kTile);
+        const uint32_t va = smem_u32(slots + sv * kTile);
+        // (1) P_b = phi(Q_c) phi(K_c)^T
+        if (!mbar_wait(&ready[sq], q_par(c), status) || !mbar_wait(&ready[sk], kv_par(c), status) ||
+            (r2 > 0 && !mbar_wait(&pempty[b], (r2 - 1) & 1, status)))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k)
+          umma_bf16(tmem + kColP + b * 128, smem_desc_sw128(qa + k * 32, 16, 1024),
+                    smem_desc_sw128(ka + k * 32, 16, 1024), id_p, k > 0 ? 1u : 0u);
+        umma_commit(&pfull[b]);
+        if (!mbar_wait(&ready[sv], kv_par(c), status)) break;
+        // (3) the increment for the next chunk's state (none after the last)
+        if (c + 1 < C) {
+          if (c > 0 && !mbar_wait(&dfree, (c - 1) & 1, status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kTileTokens / 16; ++k)
+            umma_bf16(tmem + kColD, smem_desc_sw128(va + k * 2048, ones_a - va, 1024),
+                      smem_desc_sw128(ka + k * 2048, kTile, 1024), id_d, k > 0 ? 1u : 0u);
+          umma_commit(&dfull);
+        }
+        umma_commit(&empty[sk]);
+        // (2) O_b = phi(Q_c) [S_c | z_c | 0] + Pm_b V_c
+        if (!mbar_wait(&pmready[b], r2 & 1, status) || !mbar_wait(&imgready[b], r2 & 1, status) ||
+            (r2 > 0 && !mbar_wait(&oempty[b], (r2 - 1) & 1, status)))
+          break;
+        tc_fence_after();
+        const uint32_t ocol = tmem + kColO + b * kOStride;
+        const uint32_t pa = smem_u32(pm + b * kPmBytes), ia = smem_u32(img + b * kImgBytes);
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k)
+          umma_bf16(ocol, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ia + k * 32, 16, 1024), id_qs,
+                    k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < kTileTokens / 16; ++k)
+          umma_bf16(ocol, smem_desc_sw128(pa + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024),
+                    smem_desc_sw128(va + k * 2048, kTile, 1024), id_pv, 1u);
+        umma_commit(&pmfree[b]);
+        umma_commit(&imgfree[b]);
+        umma_commit(&empty[sv]);
+        umma_commit(&ofull[b]);   // last: its arrival implies every MMA of the CTA so far is done
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------------------------- phi on Q and K; V passes through
+    const int pt = threadIdx.x - 64;
+    for (int c = 0; c < C; ++c) {
+      const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
+      if (!warp_wait(&full[sq], q_par(c), status)) break;
+      phi_tile<FMAP>(slots + sq * kTile, pt, kTileTokens);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[sq]);
+      if (!warp_wait(&full[sk], kv_par(c), status)) break;
+      // key rows past the sequence end must reach neither P nor the state
+      phi_tile<FMAP>(slots + sk * kTile, pt, min(kTileTokens, N - (tile0 + c) * kTileTokens));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[sk]);
+      if (!warp_wait(&full[sv], kv_par(c), status)) break;
+      if (lane == 0) mbar_arrive(&ready[sv]);
+    }
+  } else if (warp < 10) {
+    // ------------------ P warps: mask j > i, row sums, the bf16 A operand
+    const int qd = warp & 3, i = 32 * qd + lane;
+    const bool leader = threadIdx.x == 192;
+    for (int c = 0; c < C; ++c) {
+      const int b = c & 1, r2 = c >> 1;
+      if (leader) {
+        if (!mbar_wait(&pfull[b], r2 & 1, status) ||
+            (r2 > 0 && !mbar_wait(&pmfree[b], (r2 - 1) & 1, status)))
+          flag_p = 1;
+      }
+      named_bar_sync(1, 128);
+      if (flag_p) break;
+      tc_fence_after();
+      uint8_t* dst = pm + b * kPmBytes;
+      float rs = 0.f;
+#pragma unroll 1
+      for (int j0 = 0; j0 < 128; j0 += 32) {
+        if (j0 > 32 * qd) {   // wholly above the diagonal for this warp's rows
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            *reinterpret_cast<uint4*>(dst + swz_off(i, j0 / 8 + jj)) = make_uint4(0u, 0u, 0u, 0u);
+          continue;
+        }
+        float v[32];
+        tmem_ld32(tmem + kColP + b * 128 + (static_cast<uint32_t>(32 * qd) << 16) + j0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j0 + 8 * jj + 2 * e;
+            __nv_bfloat162 h = __floats2bfloat162_rn(j <= i ? v[8 * jj + 2 * e] : 0.f,
+                                                     j + 1 <= i ? v[8 * jj + 2 * e + 1] : 0.f);
+            const float2 g = __bfloat1622float2(h);
+            rs += g.x + g.y;
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(dst + swz_off(i, j0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      rowsum[c & 3][i] = rs;
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pempty[b]);
+        mbar_arrive(&pmready[b]);
+      }
+    }
+  } else if (warp < 14) {
+    // ------------- state warps: running S'^T row n in registers -> image
+    const int qd = warp & 3, n = 32 * qd + lane;   // TMEM lane = row of S'^T
+    const bool leader = threadIdx.x == 320;
+    const uint32_t trow = tmem + kColD + (static_cast<uint32_t>(32 * qd) << 16);
+    float S[kD];
+    // starting state: the sum of the earlier segments' states, ascending
+#pragma unroll
+    for (int e = 0; e < kD; ++e) S[e] = 0.f;
+    if (n < kStateRows) {
+      for (int s = 0; s < seg; ++s) {
+        const float* src = state + (static_cast<size_t>(bh) * nseg + s) * kStateFloats + n * kD;
+#pragma unroll
+        for (int e = 0; e < kD; e += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src + e);
+          S[e] += x.x; S[e + 1] += x.y; S[e + 2] += x.z; S[e + 3] += x.w;
+        }
+      }
+    }
+    for (int c = 0; c < C; ++c) {
+      const int b = c & 1, r2 = c >> 1;
+      if (leader) {
+        if ((c > 0 && !mbar_wait(&dfull, (c - 1) & 1, status)) ||
+            (r2 > 0 && !mbar_wait(&imgfree[b], (r2 - 1) & 1, status)))
+          flag_s = 1;
+      }
+      named_bar_sync(2, 128);
+      if (flag_s) break;
+      if (c > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+          tmem_ld32(trow + 32 * h, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) S[32 * h + e] += v[e];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dfree);
+      }
+      if (n < kStateRows) {
+        uint8_t* dst = img + b * kImgBytes + n * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < kD / 8; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(S[8 * c8 + 2 * e], S[8 * c8 + 2 * e + 1]);
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(dst + ((c8 ^ (n & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&imgready[b]);
+    }
+  } else {
+    // ------------------------------------------------------------ outputs
+    const int qd = warp & 3, i = 32 * qd + lane;
+    const bool leader = threadIdx.x == 448;
+    int prev = -1;
+    for (int c = 0; c < C; ++c) {
+      const int b = c & 1, r2 = c >> 1;
+      if (leader && !mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
+      named_bar_sync(3, 128);
+      if (flag_e) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + kColO + b * kOStride + (static_cast<uint32_t>(32 * qd) << 16);
+      const float zq = tmem_ld1(trow + kD);
+      tmem_wait_ld();
+      const float inv = 1.0f / (zq + rowsum[c & 3][i] + eps);
+      const int sq = q_slot(c);
+      uint8_t* ob = slots + sq * kTile;   // every MMA reading this Q tile is done
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float v[32];
+        tmem_ld32(trow + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * jj + 2 * e] * inv, v[8 * jj + 2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(ob + swz_off(i, c0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&oempty[b]);
+      named_bar_sync(3, 128);
+      if (leader) {
+        tma_store_3d(&tm_out, ob, 0, (tile0 + c) * kTileTokens, bh);
+        bulk_commit_group();
+        if (prev >= 0) {   // the previous chunk's store has read its Q slot: hand it back
+          bulk_wait_group_read<1>();
+          mbar_arrive(&empty[prev]);
+        }
+      }
+      prev = sq;
+    }
+    if (leader) bulk_wait_group<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int FMAP>
+cudaError_t run(const LaunchArgs& a) {
+  const Plan& p = *a.p;
+  float* state = reinterpret_cast<float*>(a.ws + p.off_partial);
+  int* status = reinterpret_cast<int*>(a.ws + p.off_status);
+  const unsigned bh = static_cast<unsigned>(p.BH);
+  cudaError_t err;
+  if (p.splits > 1) {
+    auto kern = causal_state_kernel<FMAP>;
+    if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kStSmem)) != cudaSuccess) return err;
+    kern<<<dim3(p.splits - 1, bh), 192, kStSmem, a.stream>>>(*a.tm_k, *a.tm_v, state, status,
+                                                              p.tiles_per_split, p.splits);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  auto kern = causal_chunk_kernel<FMAP>;
+  if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kChSmem)) != cudaSuccess) return err;
+  kern<<<dim3(p.splits, bh), kChThreads, kChSmem, a.stream>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, state, status,
+                                                               p.N, p.tiles, p.tiles_per_split, p.splits, p.eps);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bf16_causal(const LaunchArgs& a) {
+  const Plan& p = *a.p;
+  if (p.F != 0 || p.D != kD) return cudaErrorNotSupported;
+  return p.fmap == 0 ? run<0>(a) : run<1>(a);
+}
 
 }  // namespace la

@@ -31,13 +31,12 @@
 
 #include <mutex>
 
+#include "bf16_common.cuh"
 #include "la_internal.h"
 #include "sm100.cuh"
 
 namespace la {
 namespace {
-
-constexpr uint32_t kBoxBytes = 128 * 128;   // one TMA box: 128 rows x 64 bf16 (128 B)
 
 template <int D>
 struct Cfg {
@@ -72,51 +71,6 @@ struct Cfg {
   static constexpr int kEpiWarp0 = kCombWarp0 + 4;                 // 4 warps: outputs
   static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 };
-
-// Byte offset of (row r, logical 16-byte chunk cc) in a [128 x D] bf16 tile
-// held as D/64 TMA boxes with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz_off(int r, int cc) {
-  return static_cast<uint32_t>((cc >> 3) * kBoxBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
-}
-
-// phi on 8 bf16 values (one 16-byte chunk), branch-free and rounded once to
-// bf16.  elu(x)+1 = max(x, 0) + exp(min(x, 0)): for x > 0 the exponential is
-// exactly 1 and the bf16 add rounds x + 1 once; for x <= 0 the max is 0 and
-// the sum is the bf16-rounded exponential.  exp(y) = 2^(y log2 e) uses the
-// hardware ex2 on fp32.  relu = max(x, 0) is exact in bf16.
-template <int FMAP>
-__device__ __forceinline__ uint32_t phi_pair(uint32_t w) {
-  const __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&w);
-  const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
-  __nv_bfloat162 r = __hmax2(x, zero);
-  if (FMAP == 0) {
-    const float2 n = __bfloat1622float2(__hmin2(x, zero));
-    const __nv_bfloat162 e = __floats2bfloat162_rn(ex2_approx(n.x * kLog2e), ex2_approx(n.y * kLog2e));
-    r = __hadd2(r, e);
-  }
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
-template <int FMAP>
-__device__ __forceinline__ uint4 phi_chunk(uint4 x) {
-  return make_uint4(phi_pair<FMAP>(x.x), phi_pair<FMAP>(x.y), phi_pair<FMAP>(x.z), phi_pair<FMAP>(x.w));
-}
-
-// Lane 0 waits, the verdict is broadcast so the warp stays converged.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
-}
-
-// 16-byte load from a cluster CTA's shared memory.
-__device__ __forceinline__ void ld_cluster_v4(uint32_t cluster_addr, uint32_t (&v)[4]) {
-  asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-               : "r"(cluster_addr)
-               : "memory");
-}
 
 template <int D, int FMAP>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)

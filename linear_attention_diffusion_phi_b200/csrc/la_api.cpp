@@ -74,7 +74,7 @@ la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F,
   } else {
     if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
     if (F != 0 && (F != 256 || D != 128)) return LA_ERR_UNSUPPORTED;
-    if (causal && F != 0) return LA_ERR_UNSUPPORTED;
+    if (causal && (F != 0 || D != 64)) return LA_ERR_UNSUPPORTED;
   }
   return LA_OK;
 }
@@ -110,6 +110,15 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
     // One thread-block cluster per head; the cluster size is chosen at launch
     // from the device's cluster occupancy.  The combine runs through
     // distributed shared memory, so only the workspace header is used.
+  } else if (causal) {
+    // Segments of whole 128-token chunks, about one CTA per SM in all; every
+    // segment but the last leaves its state sum, [D + 1][D] fp32.
+    const int tiles = std::max(p->tiles, 1);
+    const long long want = std::max<long long>(1, p->num_sms / BH);
+    p->tiles_per_split = static_cast<int>(cdiv(tiles, std::min<long long>(want, tiles)));
+    p->splits = static_cast<int>(cdiv(tiles, p->tiles_per_split));
+    p->seg_len = p->tiles_per_split * la::kTileTokens;
+    partial_floats = static_cast<size_t>(BH) * p->splits * (D + 1) * D;
   } else {
     const int tiles = std::max(p->tiles, 1);
     const long long want = std::max<long long>(1, p->num_sms / BH);

@@ -92,6 +92,7 @@ def test_forward_argument_validation(handles):
     assert fwd(b16, D=64, F=256) == 2
     assert fwd(b16, D=128, F=512) == 2
     assert fwd(b16, D=128, F=256, causal=1) == 2
+    assert fwd(b16, D=128, causal=1) == 2   # bf16 causal: D = 64 only
     assert fwd(f32, B=300, H=300) == 2      # B*H beyond the grid limit
     # empty problems are a no-op
     assert fwd(f32, N=0, ptr=0, out=0) == 0
@@ -128,6 +129,9 @@ def test_workspace_bytes_and_binding(handles):
     n = la.la_workspace_bytes(h, 1, 24, 4608, 128, 0, 0)
     assert n == 256 + (1 << 20)
     assert la.la_workspace_bytes(h, 1, 24, 4608, 128, 256, 0) >= n
+    # bf16 causal: the header plus one [D + 1][D] fp32 state per (segment, head)
+    nc = la.la_workspace_bytes(h, 4, 8, 32768, 64, 0, 1)
+    assert nc >= 256 + (1 << 20) + 32 * 2 * 65 * 64 * 4 and nc < 64 << 20
     assert la.la_set_workspace(h, 0x1010, 4096) == 3          # not 256-aligned
     assert la.la_set_workspace(h, None, 0) == 0
     assert la.la_sync_status(h, None) == 4                    # no workspace bound

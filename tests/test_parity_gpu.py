@@ -189,6 +189,76 @@ def test_bf16_constant_values():
     np.testing.assert_allclose(got, np.broadcast_to(as_float64(v[0, 0, 0]), got.shape), atol=2e-2)
 
 
+# ----------------------------------------------------------- bf16 causal path
+
+BF16_CAUSAL_CASES = [
+    dict(N=1), dict(N=127), dict(N=128, fmap="relu"), dict(N=129), dict(N=300, fmap="relu"),
+    dict(N=4607), dict(N=2048, B=3, H=5), dict(N=1000, B=2, H=74), dict(N=4000, B=1, H=37, fmap="relu"),
+]
+
+
+@pytest.mark.parametrize("case", BF16_CAUSAL_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_causal_shapes(case):
+    """Every output element against the oracle's token-by-token recurrence.
+    The shapes give one chunk, ragged tails, one segment per chunk (B*H = 2),
+    one segment of many chunks (B*H = 148) and several multi-chunk segments."""
+    case = dict(case)
+    B, H = case.pop("B", 1), case.pop("H", 2)
+    w = Workload("bf16causal", B=B, H=H, D=64, causal=True, seed=89, **case)
+    check_workload(w)
+
+
+def test_causal32k_sampled_rows():
+    """The long causal workload (B=4, H=8, N=32768, D=64) in the launch
+    configuration the benchmark times; rows at the start, at chunk and segment
+    boundaries, at the end and at random, for heads spread over the batch,
+    each against the definition row by row."""
+    w = WORKLOADS["causal32k"]
+    q, k, v, _ = make_inputs(w)
+    got = run_gpu(w, q, k, v)
+    assert torch_isfinite(got)
+    qf, kf, vf = as_float64(q), as_float64(k), as_float64(v)
+    rng = np.random.default_rng(7)
+    fixed = list(range(0, 130)) + [255, 256, 257]
+    for b0 in (8192, 16384, 24576):
+        fixed += list(range(b0 - 2, b0 + 3))
+    fixed += list(range(w.N - 130, w.N))
+    for b, h in ((0, 0), (1, 5), (2, 2), (3, 7)):
+        idx = sorted(set(fixed) | set(rng.integers(0, w.N, 64).tolist()))
+        ref = ora.rows(qf, kf, vf, b, h, idx, w.fmap, w.eps, True)
+        assert_parity(as_float64(got[b, h])[idx], ref, "bf16")
+
+
+def test_bf16_causal_weights_property():
+    """N = D and V = I: row i holds the normalised weights of keys 0..i, so
+    every entry above the diagonal is exactly zero and rows sum to ~1."""
+    import torch
+    w = Workload("cweights", B=1, H=2, N=64, D=64, causal=True, seed=19)
+    q, k, _, _ = make_inputs(w)
+    v = torch.eye(64).expand(1, 2, 64, 64).contiguous().to(torch.bfloat16)
+    got = as_float64(run_gpu(w, q, k, v))
+    upper = np.triu(np.ones((64, 64), dtype=bool), 1)
+    assert np.all(got[:, :, upper] == 0.0)
+    assert got.min() >= 0.0
+    np.testing.assert_allclose(got.sum(axis=-1), 1.0, atol=2e-2)
+    assert_parity(got, oracle_full(w, q, k, v, None), "bf16")
+
+
+def test_bf16_causal_last_row_is_noncausal():
+    """The last query sees every key, so its causal row equals the
+    non-causal row (two different kernels, compared within bf16 rounding)."""
+    w = Workload("clast", B=2, H=3, N=3000, D=64, causal=True, seed=21)
+    q, k, v, _ = make_inputs(w)
+    c = as_float64(run_gpu(w, q, k, v))[:, :, -1]
+    n = as_float64(run_gpu(w.with_(causal=False), q, k, v))[:, :, -1]
+    assert np.abs(c - n).max() <= 1e-2
+
+
+def torch_isfinite(t):
+    import torch
+    return bool(torch.isfinite(t.float()).all())
+
+
 def test_host_buffer_entry_point_matches_device_path():
     import torch
     w = Workload("e2e", B=1, H=4, N=1000, D=128, seed=12)
