@@ -67,6 +67,21 @@ def algorithmic_flops(w):
     return per_head * w.B * w.H
 
 
+def kernels_per_step(w, sms):
+    """(description, launches) of the library's kernels for one forward."""
+    if w.dtype == "bf16" and not w.F and not w.causal:
+        return "fused_kernel (one cluster launch per step)", 1
+    if w.dtype == "bf16" and w.causal:
+        tiles = max(1, -(-w.N // 128))
+        want = max(1, sms // (w.B * w.H))
+        tps = -(-tiles // min(want, tiles))
+        splits = -(-tiles // tps)
+        if splits > 1:
+            return "causal_state_kernel + causal_chunk_kernel (two launches per step)", 2
+        return "causal_chunk_kernel (one launch per step)", 1
+    return "library kernels", None
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
 
@@ -340,10 +355,10 @@ def main():
     hbm, tflops, src = peaks()
     abytes = algorithmic_bytes(w)
     achieved = abytes / per_step_s / 1e9
+    kdesc, launches = kernels_per_step(w, torch.cuda.get_device_properties(dev).multi_processor_count)
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": None, "peak_source": f"{src} hbm_gbs",
-            "kernel": "fused_kernel (one launch per step)",
-            "algorithmic_bytes_per_launch": abytes}
+            "traffic": None, "peak_source": f"{src} hbm_gbs", "kernel": kdesc,
+            "algorithmic_bytes_per_step": abytes}
     if w.F:
         af = algorithmic_flops(w)
         roof["tensor"] = {"achieved": af / per_step_s / 1e12, "peak": tflops, "unit": "TFLOP/s",
@@ -360,7 +375,7 @@ def main():
                        "global_batch": w.B * ws, "seq_len": w.N, "parallelism": f"replicas{ws}",
                        "l2": f"{nsets} rotating input sets, {nsets * set_bytes / 2**20:.0f} MiB > 3x L2"},
             "hbm_gbs": achieved, "roofline": roof, "clocks": clocks, "e2e": e2e,
-            "gpu_launches": args.steps, "launch": "cuda-graph" if not args.no_graph else "host"}
+            "gpu_launches": None if launches is None else launches * args.steps, "launch": "cuda-graph" if not args.no_graph else "host"}
     if not args.no_cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)

@@ -57,13 +57,7 @@ __device__ __forceinline__ void fill_ones_atom(uint8_t* p) {
 // phi on the 128 x 64 tile the 128 calling threads share (rows >= valid -> 0).
 template <int FMAP>
 __device__ __forceinline__ void phi_tile(uint8_t* tile, int pt, int valid) {
-  const int cc = pt >> 4, r0 = pt & 15;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int r = r0 + 16 * j;
-    uint4* p = reinterpret_cast<uint4*>(tile + swz_off(r, cc));
-    *p = r < valid ? phi_chunk<FMAP>(*p) : make_uint4(0u, 0u, 0u, 0u);
-  }
+  phi_rows<FMAP, 8, 16>(tile, pt >> 4, pt & 15, valid);
 }
 
 // ================================================= kernel 1: segment states
@@ -178,24 +172,23 @@ __global__ void __launch_bounds__(192, 1)
 
 // ====================================================== kernel 2: the chunks
 
-// Shared memory: Q ring of 3 tiles, K/V ring of 2 chunks, masked P (two
-// buffers of 32 KB), state images (two of 10 KB), the ones atom.
-constexpr int kQSlots = 3;
-constexpr int kSlots = kQSlots + 4;
-constexpr uint32_t kPmBytes = 2 * kBoxBytes;   // [128 x 128] bf16 as two 64-column boxes
-constexpr uint32_t kChSmem = kSlots * kTile + 2 * kPmBytes + 2 * kImgBytes + kTile + 1024;
+// Shared memory: a ring of three chunks (Q, K, V tiles), state images (two of
+// 10 KB), the ones atom, output staging (two tiles).
+constexpr int kRing = 3;                        // chunks in flight
+constexpr int kTiles = 3 * kRing;
+constexpr uint32_t kOffImg = kTiles * kTile;
+constexpr uint32_t kOffOnes = kOffImg + 2 * kImgBytes;
+constexpr uint32_t kOffOut = kOffOnes + kTile;
+constexpr uint32_t kChSmem = kOffOut + 2 * kTile + 1024;
 // Tensor-memory columns.
-constexpr uint32_t kColP = 0;        // P: two buffers of 128
+constexpr uint32_t kColP = 0;        // P (fp32) and, in place, masked P (bf16, 64 columns): two buffers of 128
 constexpr uint32_t kColO = 256;      // O: two buffers of 80, 96 apart
 constexpr uint32_t kOStride = 96;
 constexpr uint32_t kColD = 448;      // increment [V | 1]^T phi(K): 64 columns
 constexpr int kChThreads = 576;      // producer, MMA, 4 phi, 4 P, 4 state, 4 output warps
 
-__device__ __forceinline__ int q_slot(int c) { return c % kQSlots; }
-__device__ __forceinline__ int k_slot(int c) { return kQSlots + 2 * (c & 1); }
-__device__ __forceinline__ int v_slot(int c) { return kQSlots + 2 * (c & 1) + 1; }
-__device__ __forceinline__ uint32_t q_par(int c) { return static_cast<uint32_t>((c / kQSlots) & 1); }
-__device__ __forceinline__ uint32_t kv_par(int c) { return static_cast<uint32_t>((c >> 1) & 1); }
+__device__ __forceinline__ int tile_of(int c, int kind) { return 3 * (c % kRing) + kind; }   // kind: 0 Q, 1 K, 2 V
+__device__ __forceinline__ uint32_t ring_par(int c) { return static_cast<uint32_t>((c / kRing) & 1); }
 
 template <int FMAP>
 __global__ void __launch_bounds__(kChThreads, 1)
@@ -204,8 +197,8 @@ __global__ void __launch_bounds__(kChThreads, 1)
                         const float* __restrict__ state, int* status, int N, int tiles, int tps, int nseg,
                         float eps) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kSlots], ready[kSlots], empty[kSlots];
-  __shared__ __align__(8) uint64_t pfull[2], pempty[2], pmready[2], pmfree[2];
+  __shared__ __align__(8) uint64_t full[kTiles], ready[kTiles], empty[kTiles];
+  __shared__ __align__(8) uint64_t pfull[2], pmready[2], pmfree[2];
   __shared__ __align__(8) uint64_t ofull[2], oempty[2], imgready[2], imgfree[2], dfull, dfree;
   __shared__ float rowsum[4][128];
   __shared__ uint32_t tmem_slot;
@@ -215,20 +208,20 @@ __global__ void __launch_bounds__(kChThreads, 1)
   const int seg = blockIdx.x, bh = blockIdx.y;
   const int tile0 = seg * tps;
   const int C = min(tiles, tile0 + tps) - tile0;   // chunks of this segment, >= 1
-  uint8_t* slots = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* pm = slots + kSlots * kTile;
-  uint8_t* img = pm + 2 * kPmBytes;
-  uint8_t* ones = img + 2 * kImgBytes;             // above every slot: a positive atom stride
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* img = smem + kOffImg;
+  uint8_t* ones = smem + kOffOnes;             // above every tile: a positive atom stride
+  uint8_t* outbuf = smem + kOffOut;
+  auto tile_ptr = [&](int c, int kind) { return smem + tile_of(c, kind) * kTile; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < kTiles; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&ready[i], 4);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&pfull[i], 1);
-      mbar_init(&pempty[i], 4);
       mbar_init(&pmready[i], 4);
       mbar_init(&pmfree[i], 1);
       mbar_init(&ofull[i], 1);
@@ -266,18 +259,19 @@ __global__ void __launch_bounds__(kChThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int c = 0; c < C; ++c) {
+      const CUtensorMap* maps[3] = {&tm_q, &tm_k, &tm_v};
+      bool ok = true;
+      for (int c = 0; c < C && ok; ++c) {
         const int row = (tile0 + c) * kTileTokens;
-        const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
-        if (c >= kQSlots && !mbar_wait(&empty[sq], q_par(c) ^ 1u, status)) break;
-        mbar_arrive_expect_tx(&full[sq], kTile);
-        tma_load_3d(slots + sq * kTile, &tm_q, &full[sq], 0, row, bh);
-        if (c >= 2 && !mbar_wait(&empty[sk], kv_par(c) ^ 1u, status)) break;
-        mbar_arrive_expect_tx(&full[sk], kTile);
-        tma_load_3d(slots + sk * kTile, &tm_k, &full[sk], 0, row, bh);
-        if (c >= 2 && !mbar_wait(&empty[sv], kv_par(c) ^ 1u, status)) break;
-        mbar_arrive_expect_tx(&full[sv], kTile);
-        tma_load_3d(slots + sv * kTile, &tm_v, &full[sv], 0, row, bh);
+        for (int kind = 0; kind < 3; ++kind) {
+          const int t = tile_of(c, kind);
+          if (c >= kRing && !mbar_wait(&empty[t], ring_par(c) ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[t], kTile);
+          tma_load_3d(smem + t * kTile, maps[kind], &full[t], 0, row, bh);
+        }
       }
     }
   } else if (warp == 1) {
@@ -285,26 +279,28 @@ __global__ void __launch_bounds__(kChThreads, 1)
     if (lane == 0) {
       constexpr uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);        // phi(Q) phi(K)^T
       constexpr uint32_t id_qs = idesc_bf16_f32(128, kImgRows, 0, 0);  // phi(Q) [S | z | 0]
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);        // Pm V
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);        // Pm V (Pm in tensor memory)
       constexpr uint32_t id_d = idesc_bf16_f32(128, kD, 1, 1);         // [V | 1]^T phi(K)
       const uint32_t ones_a = smem_u32(ones);
       for (int c = 0; c < C; ++c) {
         const int b = c & 1, r2 = c >> 1;
-        const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
-        const uint32_t qa = smem_u32(slots + sq * kTile);
-        const uint32_t ka = smem_u32(slots + sk * kTile);
-        const uint32_t va = smem_u32(slots + sv * kTile);
-        // (1) P_b = phi(Q_c) phi(K_c)^T
-        if (!mbar_wait(&ready[sq], q_par(c), status) || !mbar_wait(&ready[sk], kv_par(c), status) ||
-            (r2 > 0 && !mbar_wait(&pempty[b], (r2 - 1) & 1, status)))
+        const int tq = tile_of(c, 0), tk = tq + 1, tv = tq + 2;
+        const uint32_t par = ring_par(c);
+        const uint32_t qa = smem_u32(smem + tq * kTile);
+        const uint32_t ka = smem_u32(smem + tk * kTile);
+        const uint32_t va = smem_u32(smem + tv * kTile);
+        const uint32_t pcol = tmem + kColP + b * 128;
+        // (1) P_b = phi(Q_c) phi(K_c)^T, once the PV of chunk c - 2 has read buffer b
+        if (!mbar_wait(&ready[tq], par, status) || !mbar_wait(&ready[tk], par, status) ||
+            (r2 > 0 && !mbar_wait(&pmfree[b], (r2 - 1) & 1, status)))
           break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kD / 16; ++k)
-          umma_bf16(tmem + kColP + b * 128, smem_desc_sw128(qa + k * 32, 16, 1024),
-                    smem_desc_sw128(ka + k * 32, 16, 1024), id_p, k > 0 ? 1u : 0u);
+          umma_bf16(pcol, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ka + k * 32, 16, 1024), id_p,
+                    k > 0 ? 1u : 0u);
         umma_commit(&pfull[b]);
-        if (!mbar_wait(&ready[sv], kv_par(c), status)) break;
+        if (!mbar_wait(&ready[tv], par, status)) break;
         // (3) the increment for the next chunk's state (none after the last)
         if (c + 1 < C) {
           if (c > 0 && !mbar_wait(&dfree, (c - 1) & 1, status)) break;
@@ -315,25 +311,25 @@ __global__ void __launch_bounds__(kChThreads, 1)
                       smem_desc_sw128(ka + k * 2048, kTile, 1024), id_d, k > 0 ? 1u : 0u);
           umma_commit(&dfull);
         }
-        umma_commit(&empty[sk]);
+        umma_commit(&empty[tk]);
         // (2) O_b = phi(Q_c) [S_c | z_c | 0] + Pm_b V_c
         if (!mbar_wait(&pmready[b], r2 & 1, status) || !mbar_wait(&imgready[b], r2 & 1, status) ||
             (r2 > 0 && !mbar_wait(&oempty[b], (r2 - 1) & 1, status)))
           break;
         tc_fence_after();
         const uint32_t ocol = tmem + kColO + b * kOStride;
-        const uint32_t pa = smem_u32(pm + b * kPmBytes), ia = smem_u32(img + b * kImgBytes);
+        const uint32_t ia = smem_u32(img + b * kImgBytes);
 #pragma unroll
         for (int k = 0; k < kD / 16; ++k)
           umma_bf16(ocol, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ia + k * 32, 16, 1024), id_qs,
                     k > 0 ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < kTileTokens / 16; ++k)
-          umma_bf16(ocol, smem_desc_sw128(pa + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024),
-                    smem_desc_sw128(va + k * 2048, kTile, 1024), id_pv, 1u);
+          umma_bf16_ta(ocol, pcol + 8 * k, smem_desc_sw128(va + k * 2048, kTile, 1024), id_pv, 1u);
         umma_commit(&pmfree[b]);
         umma_commit(&imgfree[b]);
-        umma_commit(&empty[sv]);
+        umma_commit(&empty[tq]);
+        umma_commit(&empty[tv]);
         umma_commit(&ofull[b]);   // last: its arrival implies every MMA of the CTA so far is done
       }
     }
@@ -341,71 +337,63 @@ __global__ void __launch_bounds__(kChThreads, 1)
     // ---------------------------------- phi on Q and K; V passes through
     const int pt = threadIdx.x - 64;
     for (int c = 0; c < C; ++c) {
-      const int sq = q_slot(c), sk = k_slot(c), sv = v_slot(c);
-      if (!warp_wait(&full[sq], q_par(c), status)) break;
-      phi_tile<FMAP>(slots + sq * kTile, pt, kTileTokens);
+      const int tq = tile_of(c, 0);
+      const uint32_t par = ring_par(c);
+      if (!warp_wait(&full[tq], par, status)) break;
+      phi_tile<FMAP>(smem + tq * kTile, pt, kTileTokens);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[sq]);
-      if (!warp_wait(&full[sk], kv_par(c), status)) break;
+      if (lane == 0) mbar_arrive(&ready[tq]);
+      if (!warp_wait(&full[tq + 1], par, status)) break;
       // key rows past the sequence end must reach neither P nor the state
-      phi_tile<FMAP>(slots + sk * kTile, pt, min(kTileTokens, N - (tile0 + c) * kTileTokens));
+      phi_tile<FMAP>(smem + (tq + 1) * kTile, pt, min(kTileTokens, N - (tile0 + c) * kTileTokens));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[sk]);
-      if (!warp_wait(&full[sv], kv_par(c), status)) break;
-      if (lane == 0) mbar_arrive(&ready[sv]);
+      if (lane == 0) mbar_arrive(&ready[tq + 1]);
+      if (!warp_wait(&full[tq + 2], par, status)) break;
+      if (lane == 0) mbar_arrive(&ready[tq + 2]);
     }
   } else if (warp < 10) {
-    // ------------------ P warps: mask j > i, row sums, the bf16 A operand
+    // -- P warps: mask j > i, row sums, masked P back to tensor memory as bf16
     const int qd = warp & 3, i = 32 * qd + lane;
     const bool leader = threadIdx.x == 192;
+    const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
     for (int c = 0; c < C; ++c) {
       const int b = c & 1, r2 = c >> 1;
-      if (leader) {
-        if (!mbar_wait(&pfull[b], r2 & 1, status) ||
-            (r2 > 0 && !mbar_wait(&pmfree[b], (r2 - 1) & 1, status)))
-          flag_p = 1;
-      }
+      if (leader && !mbar_wait(&pfull[b], r2 & 1, status)) flag_p = 1;
       named_bar_sync(1, 128);
       if (flag_p) break;
       tc_fence_after();
-      uint8_t* dst = pm + b * kPmBytes;
+      const uint32_t pcol = tmem + kColP + b * 128 + lanes;
       float rs = 0.f;
+      // block j0 (32 keys) is read from columns j0.. and written, packed, to
+      // columns j0 / 2..: always columns of blocks already read
 #pragma unroll 1
       for (int j0 = 0; j0 < 128; j0 += 32) {
+        uint32_t w[16];
         if (j0 > 32 * qd) {   // wholly above the diagonal for this warp's rows
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            *reinterpret_cast<uint4*>(dst + swz_off(i, j0 / 8 + jj)) = make_uint4(0u, 0u, 0u, 0u);
-          continue;
-        }
-        float v[32];
-        tmem_ld32(tmem + kColP + b * 128 + (static_cast<uint32_t>(32 * qd) << 16) + j0, v);
-        tmem_wait_ld();
+          for (int e = 0; e < 16; ++e) w[e] = 0u;
+        } else {
+          float v[32];
+          tmem_ld32(pcol + j0, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = j0 + 8 * jj + 2 * e;
-            __nv_bfloat162 h = __floats2bfloat162_rn(j <= i ? v[8 * jj + 2 * e] : 0.f,
-                                                     j + 1 <= i ? v[8 * jj + 2 * e + 1] : 0.f);
+          for (int e = 0; e < 16; ++e) {
+            const int j = j0 + 2 * e;
+            __nv_bfloat162 h = __floats2bfloat162_rn(j <= i ? v[2 * e] : 0.f, j + 1 <= i ? v[2 * e + 1] : 0.f);
             const float2 g = __bfloat1622float2(h);
             rs += g.x + g.y;
             w[e] = *reinterpret_cast<uint32_t*>(&h);
           }
-          *reinterpret_cast<uint4*>(dst + swz_off(i, j0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        tmem_st16(pcol + j0 / 2, w);
       }
+      tmem_wait_st();
       rowsum[c & 3][i] = rs;
       tc_fence_before();
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&pempty[b]);
-        mbar_arrive(&pmready[b]);
-      }
+      if (lane == 0) mbar_arrive(&pmready[b]);
     }
   } else if (warp < 14) {
     // ------------- state warps: running S'^T row n in registers -> image
@@ -470,10 +458,12 @@ __global__ void __launch_bounds__(kChThreads, 1)
     // ------------------------------------------------------------ outputs
     const int qd = warp & 3, i = 32 * qd + lane;
     const bool leader = threadIdx.x == 448;
-    int prev = -1;
     for (int c = 0; c < C; ++c) {
       const int b = c & 1, r2 = c >> 1;
-      if (leader && !mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
+      if (leader) {
+        if (!mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
+        bulk_wait_group_read<1>();   // the store of chunk c - 2 has read staging buffer b
+      }
       named_bar_sync(3, 128);
       if (flag_e) break;
       tc_fence_after();
@@ -481,8 +471,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
       const float zq = tmem_ld1(trow + kD);
       tmem_wait_ld();
       const float inv = 1.0f / (zq + rowsum[c & 3][i] + eps);
-      const int sq = q_slot(c);
-      uint8_t* ob = slots + sq * kTile;   // every MMA reading this Q tile is done
+      uint8_t* ob = outbuf + b * kTile;
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
@@ -507,12 +496,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
       if (leader) {
         tma_store_3d(&tm_out, ob, 0, (tile0 + c) * kTileTokens, bh);
         bulk_commit_group();
-        if (prev >= 0) {   // the previous chunk's store has read its Q slot: hand it back
-          bulk_wait_group_read<1>();
-          mbar_arrive(&empty[prev]);
-        }
       }
-      prev = sq;
     }
     if (leader) bulk_wait_group<0>();
   }

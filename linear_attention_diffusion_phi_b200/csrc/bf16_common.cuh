@@ -40,6 +40,22 @@ __device__ __forceinline__ uint4 phi_chunk(uint4 x) {
   return make_uint4(phi_pair<FMAP>(x.x), phi_pair<FMAP>(x.y), phi_pair<FMAP>(x.z), phi_pair<FMAP>(x.w));
 }
 
+// phi in place on NR 16-byte chunks of one swizzled tile: column chunk cc,
+// rows r0, r0 + RS, ...; rows >= valid become 0.  Every load is issued first,
+// then the arithmetic, then every store, so that the loads overlap instead of
+// each waiting behind the previous row's store.
+template <int FMAP, int NR, int RS>
+__device__ __forceinline__ void phi_rows(uint8_t* tile, int cc, int r0, int valid) {
+  uint4 x[NR];
+#pragma unroll
+  for (int j = 0; j < NR; ++j) x[j] = *reinterpret_cast<const uint4*>(tile + swz_off(r0 + RS * j, cc));
+#pragma unroll
+  for (int j = 0; j < NR; ++j)
+    x[j] = (r0 + RS * j < valid) ? phi_chunk<FMAP>(x[j]) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int j = 0; j < NR; ++j) *reinterpret_cast<uint4*>(tile + swz_off(r0 + RS * j, cc)) = x[j];
+}
+
 // Lane 0 waits, the verdict is broadcast so the warp stays converged.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status) {
   int ok = 1;

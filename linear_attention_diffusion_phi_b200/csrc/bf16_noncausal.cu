@@ -270,12 +270,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         uint8_t* tile = slot_ptr(s);
         // key rows past the sequence end must not reach ksum
         const int valid = in_kv ? min(kTileTokens, N - (tile0 + seq / 2) * kTileTokens) : kTileTokens;
-#pragma unroll 4
-        for (int j = 0; j < C::kRowsPerThread; ++j) {
-          const int r = r0 + j * C::kThreadsPerChunk;
-          uint4* p = reinterpret_cast<uint4*>(tile + swz_off(r, cc));
-          *p = r < valid ? phi_chunk<FMAP>(*p) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        phi_rows<FMAP, C::kRowsPerThread, C::kThreadsPerChunk>(tile, cc, r0, valid);
         fence_proxy_async_smem();
       }
       __syncwarp();
