@@ -17,9 +17,9 @@
 //                        then chunk by chunk:
 //                          P  = phi(Q_c) phi(K_c)^T           (128 x 128)
 //                          Pm = P with j > i zeroed, bf16; r_i = sum_j Pm_ij
-//                          O  = phi(Q_c) [S_c | z_c] + Pm V_c  (numerator,
-//                               column 64: phi(q_i) . z_c)
-//                          out_i = O_i[0:64] / (O_i[64] + r_i + eps)
+//                          O  = phi(Q_c) [S_c | z_c] + Pm [V_c | 1]
+//                               (numerator; column 64: phi(q_i) . z_c + r_i)
+//                          out_i = O_i[0:64] / (O_i[64] + eps)
 //                          S_{c+1} = S_c + [V_c | 1]^T phi(K_c)
 //                        with the running state in fp32 registers of four
 //                        warps and each chunk's increment in tensor memory.
@@ -122,10 +122,14 @@ __global__ void __launch_bounds__(192, 1)
           break;
         tc_fence_after();
         const uint32_t ka = smem_u32(slots + sk * kTile), va = smem_u32(slots + sv * kTile);
+        const uint64_t a = smem_desc_sw128(va, ones_a - va, 1024), bk = smem_desc_sw128(ka, kTile, 1024);
+        if (t == 0)
+          umma_ss<0>(tmem, a, bk, idesc);
+        else
+          umma_ss<1>(tmem, a, bk, idesc);
 #pragma unroll
-        for (int k = 0; k < kTileTokens / 16; ++k)
-          umma_bf16(tmem, smem_desc_sw128(va + k * 2048, ones_a - va, 1024),
-                    smem_desc_sw128(ka + k * 2048, kTile, 1024), idesc, (t > 0 || k > 0) ? 1u : 0u);
+        for (int k = 1; k < kTileTokens / 16; ++k)
+          umma_ss<1>(tmem, desc_add(a, 2048 * k), desc_add(bk, 2048 * k), idesc);
         umma_commit(&empty[sk]);
         umma_commit(&empty[sv]);
       }
@@ -172,23 +176,22 @@ __global__ void __launch_bounds__(192, 1)
 
 // ====================================================== kernel 2: the chunks
 
-// Shared memory: a ring of three chunks (Q, K, V tiles), state images (two of
-// 10 KB), the ones atom, output staging (two tiles).
-constexpr int kRing = 3;                        // chunks in flight
-constexpr int kTiles = 3 * kRing;
-constexpr uint32_t kOffImg = kTiles * kTile;
+// Shared memory: rings of Q, K and V tiles, state images (two of 10 KB), the
+// ones atom.  phi(Q) goes straight to tensor memory, so a Q tile is free once
+// phi has read it; a chunk's output is staged in its K tile, free once both
+// MMAs that read phi(K) are done.
+constexpr int kRQ = 3, kRK = 4, kRV = 4;
+constexpr uint32_t kOffK = kRQ * kTile;
+constexpr uint32_t kOffV = kOffK + kRK * kTile;
+constexpr uint32_t kOffImg = kOffV + kRV * kTile;
 constexpr uint32_t kOffOnes = kOffImg + 2 * kImgBytes;
-constexpr uint32_t kOffOut = kOffOnes + kTile;
-constexpr uint32_t kChSmem = kOffOut + 2 * kTile + 1024;
-// Tensor-memory columns.
-constexpr uint32_t kColP = 0;        // P (fp32) and, in place, masked P (bf16, 64 columns): two buffers of 128
-constexpr uint32_t kColO = 256;      // O: two buffers of 80, 96 apart
-constexpr uint32_t kOStride = 96;
-constexpr uint32_t kColD = 448;      // increment [V | 1]^T phi(K): 64 columns
-constexpr int kChThreads = 576;      // producer, MMA, 4 phi, 4 P, 4 state, 4 output warps
-
-__device__ __forceinline__ int tile_of(int c, int kind) { return 3 * (c % kRing) + kind; }   // kind: 0 Q, 1 K, 2 V
-__device__ __forceinline__ uint32_t ring_par(int c) { return static_cast<uint32_t>((c / kRing) & 1); }
+constexpr uint32_t kChSmem = kOffOnes + kTile + 1024;
+// Tensor-memory columns, two buffers each.  P (fp32, 128 columns) becomes, in
+// place, masked P (bf16, columns 0..63); O then takes columns 64..143.
+__device__ __forceinline__ constexpr uint32_t col_p(int b) { return 160u * b; }
+__device__ __forceinline__ constexpr uint32_t col_q(int b) { return 320u + 32u * b; }   // phi(Q), bf16: 32 columns
+constexpr uint32_t kColD = 384;             // increment [V | 1]^T phi(K): 64 columns
+constexpr int kChThreads = 576;             // producer, MMA, 4 phi, 4 P, 4 state, 4 output warps
 
 template <int FMAP>
 __global__ void __launch_bounds__(kChThreads, 1)
@@ -197,10 +200,10 @@ __global__ void __launch_bounds__(kChThreads, 1)
                         const float* __restrict__ state, int* status, int N, int tiles, int tps, int nseg,
                         float eps) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kTiles], ready[kTiles], empty[kTiles];
-  __shared__ __align__(8) uint64_t pfull[2], pmready[2], pmfree[2];
-  __shared__ __align__(8) uint64_t ofull[2], oempty[2], imgready[2], imgfree[2], dfull, dfree;
-  __shared__ float rowsum[4][128];
+  __shared__ __align__(8) uint64_t qfull[kRQ], qempty[kRQ], kfull[kRK], kready[kRK], kempty[kRK];
+  __shared__ __align__(8) uint64_t vfull[kRV], vempty[kRV];
+  __shared__ __align__(8) uint64_t qready[2], qfree[2], pfull[2], pmready[2], ofull[2], oempty[2];
+  __shared__ __align__(8) uint64_t imgready[2], imgfree[2], dfull, dfree;
   __shared__ uint32_t tmem_slot;
   __shared__ int flag_p, flag_s, flag_e;
 
@@ -210,20 +213,30 @@ __global__ void __launch_bounds__(kChThreads, 1)
   const int C = min(tiles, tile0 + tps) - tile0;   // chunks of this segment, >= 1
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* img = smem + kOffImg;
-  uint8_t* ones = smem + kOffOnes;             // above every tile: a positive atom stride
-  uint8_t* outbuf = smem + kOffOut;
-  auto tile_ptr = [&](int c, int kind) { return smem + tile_of(c, kind) * kTile; };
+  uint8_t* ones = smem + kOffOnes;   // above every V tile: a positive atom stride
+  auto q_tile = [&](int c) { return smem + (c % kRQ) * kTile; };
+  auto k_tile = [&](int c) { return smem + kOffK + (c % kRK) * kTile; };
+  auto v_tile = [&](int c) { return smem + kOffV + (c % kRV) * kTile; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTiles; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&ready[i], 4);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < kRQ; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 4);
+    }
+    for (int i = 0; i < kRK; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kready[i], 4);
+      mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < kRV; ++i) {
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&qready[i], 4);
+      mbar_init(&qfree[i], 1);
       mbar_init(&pfull[i], 1);
       mbar_init(&pmready[i], 4);
-      mbar_init(&pmfree[i], 1);
       mbar_init(&ofull[i], 1);
       mbar_init(&oempty[i], 4);
       mbar_init(&imgready[i], 4);
@@ -259,102 +272,140 @@ __global__ void __launch_bounds__(kChThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const CUtensorMap* maps[3] = {&tm_q, &tm_k, &tm_v};
-      bool ok = true;
-      for (int c = 0; c < C && ok; ++c) {
+      for (int c = 0; c < C; ++c) {
         const int row = (tile0 + c) * kTileTokens;
-        for (int kind = 0; kind < 3; ++kind) {
-          const int t = tile_of(c, kind);
-          if (c >= kRing && !mbar_wait(&empty[t], ring_par(c) ^ 1u, status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[t], kTile);
-          tma_load_3d(smem + t * kTile, maps[kind], &full[t], 0, row, bh);
-        }
+        if (c >= kRQ && !mbar_wait(&qempty[c % kRQ], ((c / kRQ) - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(&qfull[c % kRQ], kTile);
+        tma_load_3d(q_tile(c), &tm_q, &qfull[c % kRQ], 0, row, bh);
+        if (c >= kRK && !mbar_wait(&kempty[c % kRK], ((c / kRK) - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(&kfull[c % kRK], kTile);
+        tma_load_3d(k_tile(c), &tm_k, &kfull[c % kRK], 0, row, bh);
+        if (c >= kRV && !mbar_wait(&vempty[c % kRV], ((c / kRV) - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(&vfull[c % kRV], kTile);
+        tma_load_3d(v_tile(c), &tm_v, &vfull[c % kRV], 0, row, bh);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);        // phi(Q) phi(K)^T
-      constexpr uint32_t id_qs = idesc_bf16_f32(128, kImgRows, 0, 0);  // phi(Q) [S | z | 0]
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);        // Pm V (Pm in tensor memory)
+      constexpr uint32_t id_o = idesc_bf16_f32(128, kImgRows, 0, 0);   // phi(Q) [S | z | 0]
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, kImgRows, 0, 1);  // Pm [V | 1]
       constexpr uint32_t id_d = idesc_bf16_f32(128, kD, 1, 1);         // [V | 1]^T phi(K)
       const uint32_t ones_a = smem_u32(ones);
-      for (int c = 0; c < C; ++c) {
+      auto kmajor = [&](const uint8_t* p) { return smem_desc_sw128(smem_u32(p), 16, 1024); };
+      // [V | ones] as an MN-major operand: the ones atom is the second atom
+      auto v_ones = [&](const uint8_t* p) { return smem_desc_sw128(smem_u32(p), ones_a - smem_u32(p), 1024); };
+      // inputs of P for chunk c: phi(Q_c), phi(K_c), and buffer b read out by the epilogue of c - 2
+      auto p_inputs = [&](int c, bool block) -> bool {
         const int b = c & 1, r2 = c >> 1;
-        const int tq = tile_of(c, 0), tk = tq + 1, tv = tq + 2;
-        const uint32_t par = ring_par(c);
-        const uint32_t qa = smem_u32(smem + tq * kTile);
-        const uint32_t ka = smem_u32(smem + tk * kTile);
-        const uint32_t va = smem_u32(smem + tv * kTile);
-        const uint32_t pcol = tmem + kColP + b * 128;
-        // (1) P_b = phi(Q_c) phi(K_c)^T, once the PV of chunk c - 2 has read buffer b
-        if (!mbar_wait(&ready[tq], par, status) || !mbar_wait(&ready[tk], par, status) ||
-            (r2 > 0 && !mbar_wait(&pmfree[b], (r2 - 1) & 1, status)))
-          break;
+        const uint32_t pq = r2 & 1, pk = (c / kRK) & 1, po = (r2 - 1) & 1;
+        if (!block)
+          return mbar_test(&qready[b], pq) && mbar_test(&kready[c % kRK], pk) && (r2 == 0 || mbar_test(&oempty[b], po));
+        return mbar_wait(&qready[b], pq, status) && mbar_wait(&kready[c % kRK], pk, status) &&
+               (r2 == 0 || mbar_wait(&oempty[b], po, status));
+      };
+      // (1) P_b = phi(Q_c) phi(K_c)^T
+      auto issue_p = [&](int c) {
+        const int b = c & 1;
         tc_fence_after();
+        const uint64_t bk = kmajor(k_tile(c));
+        const uint32_t d = tmem + col_p(b), a = tmem + col_q(b);
+        umma_ts<0>(d, a, bk, id_p);
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k)
-          umma_bf16(pcol, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ka + k * 32, 16, 1024), id_p,
-                    k > 0 ? 1u : 0u);
+        for (int k = 1; k < kD / 16; ++k) umma_ts<1>(d, a + 8 * k, desc_add(bk, 32 * k), id_p);
         umma_commit(&pfull[b]);
-        if (!mbar_wait(&ready[tv], par, status)) break;
-        // (3) the increment for the next chunk's state (none after the last)
-        if (c + 1 < C) {
-          if (c > 0 && !mbar_wait(&dfree, (c - 1) & 1, status)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < kTileTokens / 16; ++k)
-            umma_bf16(tmem + kColD, smem_desc_sw128(va + k * 2048, ones_a - va, 1024),
-                      smem_desc_sw128(ka + k * 2048, kTile, 1024), id_d, k > 0 ? 1u : 0u);
-          umma_commit(&dfull);
-        }
-        umma_commit(&empty[tk]);
-        // (2) O_b = phi(Q_c) [S_c | z_c | 0] + Pm_b V_c
-        if (!mbar_wait(&pmready[b], r2 & 1, status) || !mbar_wait(&imgready[b], r2 & 1, status) ||
-            (r2 > 0 && !mbar_wait(&oempty[b], (r2 - 1) & 1, status)))
-          break;
+      };
+      // (3) the increment [V_c | 1]^T phi(K_c) for the next chunk's state
+      auto issue_d = [&](int c) -> bool {
+        if (!mbar_wait(&vfull[c % kRV], (c / kRV) & 1, status) || (c > 0 && !mbar_wait(&dfree, (c - 1) & 1, status)))
+          return false;
         tc_fence_after();
-        const uint32_t ocol = tmem + kColO + b * kOStride;
-        const uint32_t ia = smem_u32(img + b * kImgBytes);
+        const uint64_t a = v_ones(v_tile(c)), bk = smem_desc_sw128(smem_u32(k_tile(c)), kTile, 1024);
+        umma_ss<0>(tmem + kColD, a, bk, id_d);
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k)
-          umma_bf16(ocol, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ia + k * 32, 16, 1024), id_qs,
-                    k > 0 ? 1u : 0u);
+        for (int k = 1; k < kTileTokens / 16; ++k)
+          umma_ss<1>(tmem + kColD, desc_add(a, 2048 * k), desc_add(bk, 2048 * k), id_d);
+        umma_commit(&dfull);
+        return true;
+      };
+      // (2) O_b = phi(Q_c) [S_c | z_c | 0] + Pm_b [V_c | 1], columns 64.. of buffer b
+      auto issue_o = [&](int c) -> bool {
+        const int b = c & 1, r2 = c >> 1;
+        if (!mbar_wait(&vfull[c % kRV], (c / kRV) & 1, status) || !mbar_wait(&pmready[b], r2 & 1, status) ||
+            !mbar_wait(&imgready[b], r2 & 1, status))
+          return false;
+        tc_fence_after();
+        const uint32_t d = tmem + col_p(b) + 64, aq = tmem + col_q(b), pm = tmem + col_p(b);
+        const uint64_t bi = kmajor(img + b * kImgBytes), bv = v_ones(v_tile(c));
+        umma_ts<0>(d, aq, bi, id_o);
 #pragma unroll
-        for (int k = 0; k < kTileTokens / 16; ++k)
-          umma_bf16_ta(ocol, pcol + 8 * k, smem_desc_sw128(va + k * 2048, kTile, 1024), id_pv, 1u);
-        umma_commit(&pmfree[b]);
+        for (int k = 1; k < kD / 16; ++k) umma_ts<1>(d, aq + 8 * k, desc_add(bi, 32 * k), id_o);
+#pragma unroll
+        for (int k = 0; k < kTileTokens / 16; ++k) umma_ts<1>(d, pm + 8 * k, desc_add(bv, 2048 * k), id_pv);
+        umma_commit(&qfree[b]);
         umma_commit(&imgfree[b]);
-        umma_commit(&empty[tq]);
-        umma_commit(&empty[tv]);
+        umma_commit(&vempty[c % kRV]);
         umma_commit(&ofull[b]);   // last: its arrival implies every MMA of the CTA so far is done
+        return true;
+      };
+      bool ok = p_inputs(0, true);
+      if (ok) issue_p(0);
+      for (int c = 0; c < C && ok; ++c) {
+        const bool more = c + 1 < C;
+        if (more && !issue_d(c)) break;
+        // P of chunk c + 1 ahead of the output MMAs of chunk c when its inputs are there already
+        bool early = false;
+        if (more && p_inputs(c + 1, false)) {
+          issue_p(c + 1);
+          early = true;
+        }
+        if (!issue_o(c)) break;
+        if (more && !early) {
+          if (!p_inputs(c + 1, true)) break;
+          issue_p(c + 1);
+        }
       }
     }
   } else if (warp < 6) {
-    // ---------------------------------- phi on Q and K; V passes through
+    // -------- phi: Q rows into tensor memory, K in place; V needs nothing
+    const int qd = warp & 3, i = 32 * qd + lane;   // Q row = tensor-memory lane
     const int pt = threadIdx.x - 64;
+    const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
     for (int c = 0; c < C; ++c) {
-      const int tq = tile_of(c, 0);
-      const uint32_t par = ring_par(c);
-      if (!warp_wait(&full[tq], par, status)) break;
-      phi_tile<FMAP>(smem + tq * kTile, pt, kTileTokens);
-      fence_proxy_async_smem();
+      const int b = c & 1, r2 = c >> 1;
+      if (!warp_wait(&qfull[c % kRQ], (c / kRQ) & 1, status)) break;
+      if (r2 > 0 && !warp_wait(&qfree[b], (r2 - 1) & 1, status)) break;
+      {
+        const uint8_t* src = q_tile(c) + i * 128;
+        uint4 x[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) x[cc] = *reinterpret_cast<const uint4*>(src + ((cc ^ (i & 7)) << 4));
+        uint32_t w[32];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 y = phi_chunk<FMAP>(x[cc]);
+          w[4 * cc] = y.x; w[4 * cc + 1] = y.y; w[4 * cc + 2] = y.z; w[4 * cc + 3] = y.w;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + col_q(b) + lanes, w);
+        tmem_wait_st();
+        tc_fence_before();
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[tq]);
-      if (!warp_wait(&full[tq + 1], par, status)) break;
+      if (lane == 0) {
+        mbar_arrive(&qempty[c % kRQ]);
+        mbar_arrive(&qready[b]);
+      }
+      if (!warp_wait(&kfull[c % kRK], (c / kRK) & 1, status)) break;
       // key rows past the sequence end must reach neither P nor the state
-      phi_tile<FMAP>(smem + (tq + 1) * kTile, pt, min(kTileTokens, N - (tile0 + c) * kTileTokens));
+      phi_tile<FMAP>(k_tile(c), pt, min(kTileTokens, N - (tile0 + c) * kTileTokens));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[tq + 1]);
-      if (!warp_wait(&full[tq + 2], par, status)) break;
-      if (lane == 0) mbar_arrive(&ready[tq + 2]);
+      if (lane == 0) mbar_arrive(&kready[c % kRK]);
     }
   } else if (warp < 10) {
-    // -- P warps: mask j > i, row sums, masked P back to tensor memory as bf16
+    // -- P warps: mask j > i, masked P back to tensor memory as bf16
     const int qd = warp & 3, i = 32 * qd + lane;
     const bool leader = threadIdx.x == 192;
     const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
@@ -364,8 +415,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
       named_bar_sync(1, 128);
       if (flag_p) break;
       tc_fence_after();
-      const uint32_t pcol = tmem + kColP + b * 128 + lanes;
-      float rs = 0.f;
+      const uint32_t pcol = tmem + col_p(b) + lanes;
       // block j0 (32 keys) is read from columns j0.. and written, packed, to
       // columns j0 / 2..: always columns of blocks already read
 #pragma unroll 1
@@ -378,19 +428,19 @@ __global__ void __launch_bounds__(kChThreads, 1)
           float v[32];
           tmem_ld32(pcol + j0, v);
           tmem_wait_ld();
+          if (j0 == 32 * qd) {   // the diagonal block: keys j <= i only
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = (j0 + e <= i) ? v[e] : 0.f;
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int j = j0 + 2 * e;
-            __nv_bfloat162 h = __floats2bfloat162_rn(j <= i ? v[2 * e] : 0.f, j + 1 <= i ? v[2 * e + 1] : 0.f);
-            const float2 g = __bfloat1622float2(h);
-            rs += g.x + g.y;
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
             w[e] = *reinterpret_cast<uint32_t*>(&h);
           }
         }
         tmem_st16(pcol + j0 / 2, w);
       }
       tmem_wait_st();
-      rowsum[c & 3][i] = rs;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&pmready[b]);
@@ -458,45 +508,48 @@ __global__ void __launch_bounds__(kChThreads, 1)
     // ------------------------------------------------------------ outputs
     const int qd = warp & 3, i = 32 * qd + lane;
     const bool leader = threadIdx.x == 448;
+    int prev = -1;   // K ring slot whose store is still reading it
     for (int c = 0; c < C; ++c) {
       const int b = c & 1, r2 = c >> 1;
-      if (leader) {
-        if (!mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
-        bulk_wait_group_read<1>();   // the store of chunk c - 2 has read staging buffer b
-      }
+      if (leader && !mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
       named_bar_sync(3, 128);
       if (flag_e) break;
       tc_fence_after();
-      const uint32_t trow = tmem + kColO + b * kOStride + (static_cast<uint32_t>(32 * qd) << 16);
-      const float zq = tmem_ld1(trow + kD);
+      const uint32_t trow = tmem + col_p(b) + 64 + (static_cast<uint32_t>(32 * qd) << 16);
+      float v[2][32];
+      tmem_ld32(trow, v[0]);
+      tmem_ld32(trow + 32, v[1]);
+      const float den = tmem_ld1(trow + kD);   // phi(q_i) . z_c + sum_j Pm_ij
       tmem_wait_ld();
-      const float inv = 1.0f / (zq + rowsum[c & 3][i] + eps);
-      uint8_t* ob = outbuf + b * kTile;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
-        float v[32];
-        tmem_ld32(trow + c0, v);
-        tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&oempty[b]);
+      const float inv = 1.0f / (den + eps);
+      uint8_t* ob = k_tile(c);   // every MMA reading this K tile is done
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * jj + 2 * e] * inv, v[8 * jj + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<uint32_t*>(&h);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(v[h][8 * jj + 2 * e] * inv, v[h][8 * jj + 2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<uint32_t*>(&hv);
           }
-          *reinterpret_cast<uint4*>(ob + swz_off(i, c0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ob + swz_off(i, 4 * h + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      tc_fence_before();
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&oempty[b]);
       named_bar_sync(3, 128);
       if (leader) {
         tma_store_3d(&tm_out, ob, 0, (tile0 + c) * kTileTokens, bh);
         bulk_commit_group();
+        if (prev >= 0) {   // the previous chunk's store has read its K tile: hand it back
+          bulk_wait_group_read<1>();
+          mbar_arrive(&kempty[prev]);
+        }
       }
+      prev = c % kRK;
     }
     if (leader) bulk_wait_group<0>();
   }

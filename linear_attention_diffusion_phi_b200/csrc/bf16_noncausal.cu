@@ -216,15 +216,22 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         tc_fence_after();
         const uint32_t ka = smem_u32(slot_ptr(sk));
         const uint32_t va = smem_u32(slot_ptr(sv));
+        // kv^T: A = V^T (MN-major: values contiguous), B = phi(K) (MN-major:
+        // features contiguous); ksum^T: A = ones block, same B.  16 tokens
+        // per MMA, 2048 bytes apart.
+        const uint64_t vdesc = smem_desc_sw128(va, kBoxBytes, 1024);
+        const uint64_t kdesc = smem_desc_sw128(ka, kBoxBytes, 1024);
+        if (t == 0) {
+          umma_ss<0>(tmem, vdesc, kdesc, idesc_kv);
+          umma_ss<0>(tmem + D, ones_desc, kdesc, idesc_ks);
+        } else {
+          umma_ss<1>(tmem, vdesc, kdesc, idesc_kv);
+          umma_ss<1>(tmem + D, ones_desc, kdesc, idesc_ks);
+        }
 #pragma unroll
-        for (int k = 0; k < kTileTokens / 16; ++k) {
-          // kv^T: A = V^T (MN-major: values contiguous), B = phi(K) (MN-major:
-          // features contiguous); ksum^T: A = ones block, same B.
-          const uint64_t vdesc = smem_desc_sw128(va + k * 2048, kBoxBytes, 1024);
-          const uint64_t kdesc = smem_desc_sw128(ka + k * 2048, kBoxBytes, 1024);
-          const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
-          umma_bf16(tmem, vdesc, kdesc, idesc_kv, acc);
-          umma_bf16(tmem + D, ones_desc, kdesc, idesc_ks, acc);
+        for (int k = 1; k < kTileTokens / 16; ++k) {
+          umma_ss<1>(tmem, desc_add(vdesc, 2048 * k), desc_add(kdesc, 2048 * k), idesc_kv);
+          umma_ss<1>(tmem + D, ones_desc, desc_add(kdesc, 2048 * k), idesc_ks);
         }
         umma_commit(&empty[sk]);
         umma_commit(&empty[sv]);
@@ -242,13 +249,15 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           if (!got) break;
           tc_fence_after();
           const uint32_t qa = smem_u32(slot_ptr(s));
+          // A = phi(Q) and B = [kv | ksum]^T, both K-major (features contiguous)
+          const uint64_t adesc = smem_desc_sw128(qa, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(ba, 16, 1024);
+          const uint32_t d = tmem + a * C::kAccStride;
+          umma_ss<0>(d, adesc, bdesc, idesc_ap);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            // A = phi(Q) and B = [kv | ksum]^T, both K-major (features contiguous).
-            const uint64_t adesc = smem_desc_sw128(qa + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(ba + (k >> 2) * C::kBlobAtomBytes + (k & 3) * 32, 16, 1024);
-            umma_bf16(tmem + a * C::kAccStride, adesc, bdesc, idesc_ap, k > 0 ? 1u : 0u);
-          }
+          for (int k = 1; k < D / 16; ++k)
+            umma_ss<1>(d, desc_add(adesc, (k >> 2) * kBoxBytes + (k & 3) * 32),
+                       desc_add(bdesc, (k >> 2) * C::kBlobAtomBytes + (k & 3) * 32), idesc_ap);
           umma_commit(&accfull[a]);
         }
       }
