@@ -54,19 +54,24 @@ __device__ __forceinline__ void fill_ones_atom(uint8_t* p) {
   }
 }
 
-// phi on the 128 x 64 tile the 128 calling threads share (rows >= valid -> 0).
+// phi on the 128 x 64 tile the 256 calling threads (8 warps, two per
+// sub-partition) share: column chunk pt / 32, rows pt % 32 + 32 j.
 template <int FMAP>
 __device__ __forceinline__ void phi_tile(uint8_t* tile, int pt, int valid) {
-  phi_rows<FMAP, 8, 16>(tile, pt >> 4, pt & 15, valid);
+  phi_rows<FMAP, 4, 32>(tile, pt >> 5, pt & 31, valid);
 }
+
+constexpr int kPhiWarps = 8;
 
 // ================================================= kernel 1: segment states
 
 constexpr int kStSlots = 8;
 constexpr uint32_t kStSmem = kStSlots * kTile + kTile + 1024;
 
+constexpr int kStThreads = 64 + 32 * kPhiWarps;   // producer, MMA, phi warps
+
 template <int FMAP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kStThreads, 1)
     causal_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         float* __restrict__ state, int* status, int tps, int nseg) {
   extern __shared__ uint8_t smem_raw[];
@@ -81,7 +86,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStSlots; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&ready[i], 4);
+      mbar_init(&ready[i], kPhiWarps);
       mbar_init(&empty[i], 1);
     }
     mbar_init(&accfull, 1);
@@ -152,7 +157,8 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ready[s]);
     }
-    if (ok && warp_wait(&accfull, 0, status)) {
+    // warps 2..5 cover the four lane quarters of tensor memory
+    if (ok && warp < 6 && warp_wait(&accfull, 0, status)) {
       tc_fence_after();
       const int qd = warp & 3, row = 32 * qd + lane;   // TMEM lane = row of S'^T
       float* dst = state + (static_cast<size_t>(bh) * nseg + seg) * kStateFloats + row * kD;
@@ -191,7 +197,7 @@ constexpr uint32_t kChSmem = kOffOnes + kTile + 1024;
 __device__ __forceinline__ constexpr uint32_t col_p(int b) { return 160u * b; }
 __device__ __forceinline__ constexpr uint32_t col_q(int b) { return 320u + 32u * b; }   // phi(Q), bf16: 32 columns
 constexpr uint32_t kColD = 384;             // increment [V | 1]^T phi(K): 64 columns
-constexpr int kChThreads = 576;             // producer, MMA, 4 phi, 4 P, 4 state, 4 output warps
+constexpr int kChThreads = 64 + 32 * kPhiWarps + 256;   // producer, MMA, phi, 4 P + output, 4 state warps
 
 template <int FMAP>
 __global__ void __launch_bounds__(kChThreads, 1)
@@ -205,7 +211,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
   __shared__ __align__(8) uint64_t qready[2], qfree[2], pfull[2], pmready[2], ofull[2], oempty[2];
   __shared__ __align__(8) uint64_t imgready[2], imgfree[2], dfull, dfree;
   __shared__ uint32_t tmem_slot;
-  __shared__ int flag_p, flag_s, flag_e;
+  __shared__ int flag_p, flag_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = blockIdx.x, bh = blockIdx.y;
@@ -221,11 +227,11 @@ __global__ void __launch_bounds__(kChThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRQ; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], 4);
+      mbar_init(&qempty[i], kPhiWarps);
     }
     for (int i = 0; i < kRK; ++i) {
       mbar_init(&kfull[i], 1);
-      mbar_init(&kready[i], 4);
+      mbar_init(&kready[i], kPhiWarps);
       mbar_init(&kempty[i], 1);
     }
     for (int i = 0; i < kRV; ++i) {
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
       mbar_init(&vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&qready[i], 4);
+      mbar_init(&qready[i], kPhiWarps);
       mbar_init(&qfree[i], 1);
       mbar_init(&pfull[i], 1);
       mbar_init(&pmready[i], 4);
@@ -249,7 +255,7 @@ __global__ void __launch_bounds__(kChThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_out);
-    flag_p = flag_s = flag_e = 0;
+    flag_p = flag_s = 0;
   }
   fill_ones_atom(ones);
   // image rows 65..79 are the MMA's zero padding, in both buffers
@@ -367,9 +373,11 @@ __global__ void __launch_bounds__(kChThreads, 1)
         }
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kPhiWarps) {
     // -------- phi: Q rows into tensor memory, K in place; V needs nothing
-    const int qd = warp & 3, i = 32 * qd + lane;   // Q row = tensor-memory lane
+    // Two warps per lane quarter: Q row i = tensor-memory lane, each warp one
+    // half of the 64 features.
+    const int qd = warp & 3, half = (warp - 2) >> 2, i = 32 * qd + lane;
     const int pt = threadIdx.x - 64;
     const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
     for (int c = 0; c < C; ++c) {
@@ -378,17 +386,17 @@ __global__ void __launch_bounds__(kChThreads, 1)
       if (r2 > 0 && !warp_wait(&qfree[b], (r2 - 1) & 1, status)) break;
       {
         const uint8_t* src = q_tile(c) + i * 128;
-        uint4 x[8];
+        uint4 x[4];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) x[cc] = *reinterpret_cast<const uint4*>(src + ((cc ^ (i & 7)) << 4));
-        uint32_t w[32];
+        for (int m = 0; m < 4; ++m) x[m] = *reinterpret_cast<const uint4*>(src + (((4 * half + m) ^ (i & 7)) << 4));
+        uint32_t w[16];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint4 y = phi_chunk<FMAP>(x[cc]);
-          w[4 * cc] = y.x; w[4 * cc + 1] = y.y; w[4 * cc + 2] = y.z; w[4 * cc + 3] = y.w;
+        for (int m = 0; m < 4; ++m) {
+          const uint4 y = phi_chunk<FMAP>(x[m]);
+          w[4 * m] = y.x; w[4 * m + 1] = y.y; w[4 * m + 2] = y.z; w[4 * m + 3] = y.w;
         }
         tc_fence_after();
-        tmem_st32(tmem + col_q(b) + lanes, w);
+        tmem_st16(tmem + col_q(b) + 16 * half + lanes, w);
         tmem_wait_st();
         tc_fence_before();
       }
@@ -404,51 +412,99 @@ __global__ void __launch_bounds__(kChThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&kready[c % kRK]);
     }
-  } else if (warp < 10) {
-    // -- P warps: mask j > i, masked P back to tensor memory as bf16
+  } else if (warp < 14) {
+    // ---- P and output warps: masked P of chunk c, then the output of c - 1
     const int qd = warp & 3, i = 32 * qd + lane;
-    const bool leader = threadIdx.x == 192;
+    const bool leader = threadIdx.x == 64 + 32 * kPhiWarps;
     const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
-    for (int c = 0; c < C; ++c) {
-      const int b = c & 1, r2 = c >> 1;
-      if (leader && !mbar_wait(&pfull[b], r2 & 1, status)) flag_p = 1;
-      named_bar_sync(1, 128);
-      if (flag_p) break;
-      tc_fence_after();
-      const uint32_t pcol = tmem + col_p(b) + lanes;
-      // block j0 (32 keys) is read from columns j0.. and written, packed, to
-      // columns j0 / 2..: always columns of blocks already read
+    int prev = -1;   // K ring slot whose store is still reading it
+    for (int c = 0; c <= C; ++c) {
+      if (c < C) {
+        // mask j > i, masked P back to tensor memory as bf16
+        const int b = c & 1, r2 = c >> 1;
+        if (leader && !mbar_wait(&pfull[b], r2 & 1, status)) flag_p = 1;
+        named_bar_sync(1, 128);
+        if (flag_p) break;
+        tc_fence_after();
+        const uint32_t pcol = tmem + col_p(b) + lanes;
+        // block j0 (32 keys) is read from columns j0.. and written, packed, to
+        // columns j0 / 2..: always columns of blocks already read
 #pragma unroll 1
-      for (int j0 = 0; j0 < 128; j0 += 32) {
-        uint32_t w[16];
-        if (j0 > 32 * qd) {   // wholly above the diagonal for this warp's rows
+        for (int j0 = 0; j0 < 128; j0 += 32) {
+          uint32_t w[16];
+          if (j0 > 32 * qd) {   // wholly above the diagonal for this warp's rows
 #pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = 0u;
-        } else {
-          float v[32];
-          tmem_ld32(pcol + j0, v);
-          tmem_wait_ld();
-          if (j0 == 32 * qd) {   // the diagonal block: keys j <= i only
+            for (int e = 0; e < 16; ++e) w[e] = 0u;
+          } else {
+            float v[32];
+            tmem_ld32(pcol + j0, v);
+            tmem_wait_ld();
+            if (j0 == 32 * qd) {   // the diagonal block: keys j <= i only
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (j0 + e <= i) ? v[e] : 0.f;
+              for (int e = 0; e < 32; ++e) v[e] = (j0 + e <= i) ? v[e] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+              w[e] = *reinterpret_cast<uint32_t*>(&h);
+            }
           }
+          tmem_st16(pcol + j0 / 2, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pmready[b]);
+      }
+      if (c > 0) {
+        // output of chunk e = c - 1
+        const int e = c - 1, b = e & 1, r2 = e >> 1;
+        if (leader && !mbar_wait(&ofull[b], r2 & 1, status)) flag_p = 1;
+        named_bar_sync(1, 128);
+        if (flag_p) break;
+        tc_fence_after();
+        const uint32_t trow = tmem + col_p(b) + 64 + lanes;
+        float v[2][32];
+        tmem_ld32(trow, v[0]);
+        tmem_ld32(trow + 32, v[1]);
+        const float den = tmem_ld1(trow + kD);   // phi(q_i) . z_e + sum_j Pm_ij
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&oempty[b]);
+        const float inv = 1.0f / (den + eps);
+        uint8_t* ob = k_tile(e);   // every MMA reading this K tile is done
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-            w[e] = *reinterpret_cast<uint32_t*>(&h);
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint32_t w[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              __nv_bfloat162 hv = __floats2bfloat162_rn(v[h][8 * jj + 2 * t] * inv, v[h][8 * jj + 2 * t + 1] * inv);
+              w[t] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(ob + swz_off(i, 4 * h + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-        tmem_st16(pcol + j0 / 2, w);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          tma_store_3d(&tm_out, ob, 0, (tile0 + e) * kTileTokens, bh);
+          bulk_commit_group();
+          if (prev >= 0) {   // the previous chunk's store has read its K tile: hand it back
+            bulk_wait_group_read<1>();
+            mbar_arrive(&kempty[prev]);
+          }
+        }
+        prev = e % kRK;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&pmready[b]);
     }
-  } else if (warp < 14) {
+    if (leader) bulk_wait_group<0>();
+  } else {
     // ------------- state warps: running S'^T row n in registers -> image
     const int qd = warp & 3, n = 32 * qd + lane;   // TMEM lane = row of S'^T
-    const bool leader = threadIdx.x == 320;
+    const bool leader = threadIdx.x == 64 + 32 * kPhiWarps + 128;
     const uint32_t trow = tmem + kColD + (static_cast<uint32_t>(32 * qd) << 16);
     float S[kD];
     // starting state: the sum of the earlier segments' states, ascending
@@ -504,54 +560,6 @@ __global__ void __launch_bounds__(kChThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&imgready[b]);
     }
-  } else {
-    // ------------------------------------------------------------ outputs
-    const int qd = warp & 3, i = 32 * qd + lane;
-    const bool leader = threadIdx.x == 448;
-    int prev = -1;   // K ring slot whose store is still reading it
-    for (int c = 0; c < C; ++c) {
-      const int b = c & 1, r2 = c >> 1;
-      if (leader && !mbar_wait(&ofull[b], r2 & 1, status)) flag_e = 1;
-      named_bar_sync(3, 128);
-      if (flag_e) break;
-      tc_fence_after();
-      const uint32_t trow = tmem + col_p(b) + 64 + (static_cast<uint32_t>(32 * qd) << 16);
-      float v[2][32];
-      tmem_ld32(trow, v[0]);
-      tmem_ld32(trow + 32, v[1]);
-      const float den = tmem_ld1(trow + kD);   // phi(q_i) . z_c + sum_j Pm_ij
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&oempty[b]);
-      const float inv = 1.0f / (den + eps);
-      uint8_t* ob = k_tile(c);   // every MMA reading this K tile is done
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 hv = __floats2bfloat162_rn(v[h][8 * jj + 2 * e] * inv, v[h][8 * jj + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<uint32_t*>(&hv);
-          }
-          *reinterpret_cast<uint4*>(ob + swz_off(i, 4 * h + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(3, 128);
-      if (leader) {
-        tma_store_3d(&tm_out, ob, 0, (tile0 + c) * kTileTokens, bh);
-        bulk_commit_group();
-        if (prev >= 0) {   // the previous chunk's store has read its K tile: hand it back
-          bulk_wait_group_read<1>();
-          mbar_arrive(&kempty[prev]);
-        }
-      }
-      prev = c % kRK;
-    }
-    if (leader) bulk_wait_group<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -568,7 +576,7 @@ cudaError_t run(const LaunchArgs& a) {
   if (p.splits > 1) {
     auto kern = causal_state_kernel<FMAP>;
     if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kStSmem)) != cudaSuccess) return err;
-    kern<<<dim3(p.splits - 1, bh), 192, kStSmem, a.stream>>>(*a.tm_k, *a.tm_v, state, status,
+    kern<<<dim3(p.splits - 1, bh), kStThreads, kStSmem, a.stream>>>(*a.tm_k, *a.tm_v, state, status,
                                                               p.tiles_per_split, p.splits);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
