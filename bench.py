@@ -67,6 +67,31 @@ def algorithmic_flops(w):
     return per_head * w.B * w.H
 
 
+# DRAM traffic per step (dram__bytes_read.sum + dram__bytes_write.sum summed
+# over the step's launches, one ncu --set full capture each; the summaries are
+# in profiles/).  Reported only while the kernel sources still hash to what
+# was captured; otherwise null.
+NCU_TRAFFIC = {
+    "flux1024": (88_507_648, ("bf16_noncausal.cu", "bf16_common.cuh", "sm100.cuh", "la_internal.h"),
+                 "36acf9208342a632"),
+    "causal32k": (720_156_416, ("bf16_causal.cu", "bf16_common.cuh", "sm100.cuh", "la_internal.h"),
+                  "7a22c532fe7c9d4c"),
+}
+
+
+def captured_traffic(w):
+    import hashlib
+    entry = NCU_TRAFFIC.get(w.name)
+    if entry is None:
+        return None
+    nbytes, files, digest = entry
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "linear_attention_diffusion_phi_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return nbytes if h.hexdigest()[:16] == digest else None
+
+
 def kernels_per_step(w, sms):
     """(description, launches) of the library's kernels for one forward."""
     if w.dtype == "bf16" and not w.F and not w.causal:
@@ -357,7 +382,7 @@ def main():
     achieved = abytes / per_step_s / 1e9
     kdesc, launches = kernels_per_step(w, torch.cuda.get_device_properties(dev).multi_processor_count)
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": None, "peak_source": f"{src} hbm_gbs", "kernel": kdesc,
+            "traffic": captured_traffic(w), "peak_source": f"{src} hbm_gbs", "frac_of": src, "kernel": kdesc,
             "algorithmic_bytes_per_step": abytes}
     if w.F:
         af = algorithmic_flops(w)
