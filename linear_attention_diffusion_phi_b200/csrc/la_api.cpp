@@ -120,14 +120,21 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
     p->seg_len = p->tiles_per_split * la::kTileTokens;
     partial_floats = static_cast<size_t>(BH) * p->splits * (D + 1) * D;
   } else {
+    // Projected (D = 128, F = 256): state CTAs per (split, head, feature
+    // half), about one per SM; apply CTAs about one per SM. Partials are fp32
+    // kv^T [D][F/2] and ksum [F/2] per (head, split, half); the image is the
+    // apply's bf16 [kv | ksum | 0]^T operand, [D + 16][F] per head.
     const int tiles = std::max(p->tiles, 1);
-    const long long want = std::max<long long>(1, p->num_sms / BH);
+    const long long want = std::max<long long>(1, p->num_sms / (2 * BH));
     p->tiles_per_split = static_cast<int>(cdiv(tiles, std::min<long long>(want, tiles)));
     p->splits = static_cast<int>(cdiv(tiles, p->tiles_per_split));
     p->seg_len = p->tiles_per_split * la::kTileTokens;
+    const long long want3 = std::max<long long>(1, p->num_sms / BH);
+    p->apply_tps = static_cast<int>(cdiv(tiles, std::min<long long>(want3, tiles)));
+    p->apply_ctas = static_cast<int>(cdiv(tiles, p->apply_tps));
     partial_floats = static_cast<size_t>(BH) * p->splits * p->Fe * D;
     ksum_floats = static_cast<size_t>(BH) * p->splits * p->Fe;
-    p->blob_bytes = la::blob_bytes_for(D, p->Fe);
+    p->blob_bytes = static_cast<size_t>(D + 16) * p->Fe * 2;
     blob_total = static_cast<size_t>(BH) * p->blob_bytes;
   }
   size_t off = 0;
@@ -336,7 +343,7 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
       if (!encode_bf16_3d(&tw, h->W, nW, D, F, ws, 128)) return LA_ERR_CUDA;
       a.tm_w = &tw;
     }
-    err = causal ? la::launch_bf16_causal(a) : la::launch_bf16_noncausal(a);
+    err = causal ? la::launch_bf16_causal(a) : (F > 0 ? la::launch_bf16_projected(a) : la::launch_bf16_noncausal(a));
   }
   if (err == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
   if (err != cudaSuccess) {

@@ -34,6 +34,7 @@ struct Plan {
   int seg_len;     // tokens per split/segment
   int num_sms;
   int heads_per_cta;   // bf16 non-causal: heads whose splits one CTA owns (1 or 2)
+  int apply_ctas, apply_tps;   // bf16 projected: apply CTAs per head, 128-token tiles each
   // workspace layout (byte offsets from the workspace base, 256-aligned)
   size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
   size_t blob_bytes;   // bf16 B-operand image per head
@@ -81,5 +82,6 @@ cudaError_t launch_f32(const LaunchArgs& a);
 // bf16 tensor-core paths.
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a);
 cudaError_t launch_bf16_causal(const LaunchArgs& a);
+cudaError_t launch_bf16_projected(const LaunchArgs& a);
 
 }  // namespace la

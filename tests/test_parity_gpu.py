@@ -189,6 +189,47 @@ def test_bf16_constant_values():
     np.testing.assert_allclose(got, np.broadcast_to(as_float64(v[0, 0, 0]), got.shape), atol=2e-2)
 
 
+# -------------------------------------------------------- bf16 projected path
+
+BF16_PROJ_CASES = [
+    dict(N=1), dict(N=127), dict(N=129, fmap="relu"), dict(N=300), dict(N=1000, fmap="relu"),
+    dict(N=4607), dict(N=2048, B=3, H=5),
+]
+
+
+@pytest.mark.parametrize("case", BF16_PROJ_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_projected_shapes(case):
+    """phi(x) = fmap(x W_h) with D = 128, F = 256 (one W per head), every
+    output element against the oracle."""
+    case = dict(case)
+    B, H = case.pop("B", 1), case.pop("H", 2)
+    w = Workload("bf16proj", B=B, H=H, D=128, F=256, seed=90, **case)
+    check_workload(w)
+
+
+def test_proj256_full():
+    """The projected-feature workload (B=1, H=24, N=4608, D=128, F=256,
+    elu(xW)+1), every output element."""
+    check_workload(WORKLOADS["proj256"])
+
+
+def test_bf16_projected_shared_matrix():
+    """One W for all heads (head stride 0) equals passing it per head."""
+    import torch
+    w = Workload("bf16projshared", B=2, H=3, N=700, D=128, F=256, seed=91)
+    q, k, v, W = make_inputs(w)
+    W1 = W[:1].contiguous()
+    dev = torch.device("cuda:0")
+    per_head = run_gpu(w, q, k, v, W1.expand(3, 128, 256).contiguous())
+    assert_parity(per_head, oracle_full(w, q, k, v, W1.expand(3, 128, 256).contiguous()), "bf16")
+    shared = la.LinearAttention(torch.bfloat16, w.fmap, w.eps, False, W1[0].to(dev))   # [D, F]: every head
+    got = shared(q.to(dev), k.to(dev), v.to(dev)).cpu()
+    torch.cuda.synchronize()
+    assert shared.sync_status() == la.LA_OK
+    assert torch.equal(got, per_head)
+    shared.close()
+
+
 # ----------------------------------------------------------- bf16 causal path
 
 BF16_CAUSAL_CASES = [
