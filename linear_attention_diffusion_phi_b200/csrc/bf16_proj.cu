@@ -14,8 +14,8 @@
 //                        warps into shared memory (bf16), then
 //                        kv^T += V^T phi(K) (M = D, N = 128) and
 //                        ksum += phi(K)^T 1 (M = 128 features, N = 16).
-//   proj_combine_kernel  grid (B H): sums the splits in ascending order (fp32)
-//                        and writes the apply's B operand [kv | ksum | 0]^T as
+//   image_combine_kernel (bf16_split.cu) sums the splits in ascending order
+//                        (fp32) into the apply's B operand [kv | ksum | 0]^T,
 //                        bf16, K-major, 128-byte swizzle (144 rows x 256).
 //   proj_apply_kernel    grid (ctas, B H): W_h and the image stay in shared
 //                        memory; per tile, Q W one feature half at a time,
@@ -256,45 +256,6 @@ __global__ void __launch_bounds__(kS1Threads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// ==================================================== kernel 2: the combine
-
-// One block per head: image[n][f] = sum over splits (ascending) of kv^T[n][f]
-// (n < 128), ksum[f] (n = 128), 0 (n = 129..143); bf16, K-major, 128-byte
-// swizzle, four 64-feature atoms of 144 rows.
-__global__ void __launch_bounds__(256)
-    proj_combine_kernel(const float* __restrict__ part_kv, const float* __restrict__ part_ks,
-                        uint8_t* __restrict__ image, int nsplit) {
-  const int bh = blockIdx.x;
-  uint8_t* img = image + static_cast<size_t>(bh) * kImgBytes;
-  for (int idx = threadIdx.x; idx < kNB * (kF / 8); idx += blockDim.x) {
-    const int n = idx / (kF / 8), f0 = (idx % (kF / 8)) * 8;
-    const int fh = f0 / kFH, fl = f0 % kFH;
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    if (n <= kD) {
-      for (int s = 0; s < nsplit; ++s) {
-        const size_t part = (static_cast<size_t>(bh) * nsplit + s) * 2 + fh;
-        const float* src = n < kD ? part_kv + part * (kD * kFH) + static_cast<size_t>(n) * kFH + fl
-                                  : part_ks + part * kFH + fl;
-        const float4 a = *reinterpret_cast<const float4*>(src);
-        const float4 b = *reinterpret_cast<const float4*>(src + 4);
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-      }
-    }
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-      w[e] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    const int atom = f0 >> 6, cc = (f0 & 63) >> 3;
-    *reinterpret_cast<uint4*>(img + atom * kImgAtom + n * 128 + ((cc ^ (n & 7)) << 4)) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 // ====================================================== kernel 3: the apply
 
 constexpr uint32_t kS3OffW = 0;                          // W: four 64-feature atoms [128 d][64 f]
@@ -444,29 +405,29 @@ __global__ void __launch_bounds__(kS3Threads, 1)
       const float den = tmem_ld1(trow + kD);   // phi(q_i) . ksum
       tmem_wait_ld();
       const float inv = 1.0f / (den + eps);
-      const int row = (tile0 + t) * kTileTokens + i;
-      uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + min(row, N - 1)) * kD);
-#pragma unroll 1
+      // the whole row is packed to bf16 in registers first, so that O is
+      // handed back to the next tile's apply before the global stores
+      uint32_t w[kD / 2];
+#pragma unroll
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
         tmem_ld32(trow + c0, v);
         tmem_wait_ld();
-        if (row < N) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 hv = __floats2bfloat162_rn(v[8 * c + 2 * e] * inv, v[8 * c + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            dst[c0 / 8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * e] * inv, v[2 * e + 1] * inv);
+          w[c0 / 2 + e] = *reinterpret_cast<uint32_t*>(&hv);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&oempty);
+      const int row = (tile0 + t) * kTileTokens + i;
+      if (row < N) {
+        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + row) * kD);
+#pragma unroll
+        for (int c = 0; c < kD / 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      }
     }
   }
   tc_fence_before();
@@ -492,8 +453,8 @@ cudaError_t run(const LaunchArgs& a) {
                                                                     p.tiles_per_split);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  proj_combine_kernel<<<bh, 256, 0, a.stream>>>(part_kv, part_ks, image, p.splits);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = launch_image_combine(part_kv, part_ks, image, p.BH, p.splits, kD, kFH, 2, a.stream)) != cudaSuccess)
+    return err;
   {
     auto kern = proj_apply_kernel<FMAP>;
     if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kS3Smem)) != cudaSuccess) return err;

@@ -190,10 +190,22 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 namespace la {
 
+// Plan of the fused cluster kernel (la_forward_noalloc): the combine runs
+// through distributed shared memory, so the workspace is only the header
+// (status word and per-head barrier words).
 void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p) {
-  la_handle_s h = {};
-  h.dtype = LA_BF16;
-  make_plan(&h, B, H, N, D, 0, fmap, eps, 0, num_sms, p);
+  memset(p, 0, sizeof(*p));
+  p->dtype = LA_BF16;
+  p->B = B; p->H = H; p->N = N; p->D = D; p->F = 0; p->Fe = D;
+  p->fmap = fmap; p->causal = 0; p->eps = eps;
+  p->BH = static_cast<long long>(B) * H;
+  p->tiles = static_cast<int>(cdiv(N, la::kTileTokens));
+  p->num_sms = num_sms > 0 ? num_sms : 148;
+  size_t off = 0;
+  p->off_status = off;        off += la::kStatusBytes;
+  p->off_sync = off;          off += la::kSyncBytes;
+  p->off_partial = p->off_ksum_partial = p->off_final = p->off_final_ksum = p->off_blob = off;
+  p->bytes = off;
 }
 
 bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,

@@ -83,5 +83,9 @@ cudaError_t launch_f32(const LaunchArgs& a);
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a);
 cudaError_t launch_bf16_causal(const LaunchArgs& a);
 cudaError_t launch_bf16_projected(const LaunchArgs& a);
+// Sums fp32 partials (kv^T [D][fpart] and ksum [fpart] per (head, split, part))
+// into the apply's bf16 [kv | ksum | 0]^T image, K-major, D + 16 rows.
+cudaError_t launch_image_combine(const float* part_kv, const float* part_ks, uint8_t* image, long long BH,
+                                 int nsplit, int D, int fpart, int parts, cudaStream_t stream);
 
 }  // namespace la
