@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       ++seq;
     }
   };
+  // Programmatic dependent launch: this grid may have started while the
+  // previous launch on the stream still ran.  Nothing above touched global
+  // memory; wait for that launch to complete before the first load, and let
+  // the next launch begin its own set-up as this grid's CTAs leave.
+  pdl_wait();
+  pdl_launch_dependents();
   // Every CTA's barriers exist (fence.mbarrier_init above) before any remote
   // arrival: relaxed arrive, first loads, then the acquiring wait.
   cluster_arrive_relaxed();
@@ -528,18 +534,20 @@ cudaError_t run(const LaunchArgs& a) {
   cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
   const int S = pick_cluster(kern, C::kSmemBytes, C::kThreads, p.BH, p.tiles);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(p.BH));
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = a.stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
   return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
 }
