@@ -69,27 +69,31 @@ def algorithmic_flops(w):
 
 # DRAM traffic per step (dram__bytes_read.sum + dram__bytes_write.sum summed
 # over the step's launches, one ncu --set full capture each; the summaries are
-# in profiles/).  Reported only while the kernel sources still hash to what
-# was captured; otherwise null.
+# in profiles/).  Reported only while the device code (the kernel file and the
+# device headers it includes) still hashes to what was captured; else null.
+DEVICE_HEADERS = ("bf16_common.cuh", "sm100.cuh")
 NCU_TRAFFIC = {
-    "flux1024": (88_507_648, ("bf16_noncausal.cu", "bf16_common.cuh", "sm100.cuh", "la_internal.h"),
-                 "36acf9208342a632"),
-    "causal32k": (720_156_416, ("bf16_causal.cu", "bf16_common.cuh", "sm100.cuh", "la_internal.h"),
-                  "7a22c532fe7c9d4c"),
+    "flux1024": (89_110_272, ("bf16_noncausal.cu",), "5d5b55b9fa575f59"),
+    "causal32k": (720_138_752, ("bf16_causal.cu",), "9f1af53b6a66f758"),
+    "proj256": (101_737_216, ("bf16_proj.cu", "bf16_image.cu"), "fc1fb88d621ca2f1"),
 }
 
 
-def captured_traffic(w):
+def source_hash(kernel_files):
     import hashlib
+    h = hashlib.sha256()
+    for f in tuple(kernel_files) + DEVICE_HEADERS:
+        with open(os.path.join(ROOT, "linear_attention_diffusion_phi_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(w):
     entry = NCU_TRAFFIC.get(w.name)
     if entry is None:
         return None
-    nbytes, files, digest = entry
-    h = hashlib.sha256()
-    for f in files:
-        with open(os.path.join(ROOT, "linear_attention_diffusion_phi_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return nbytes if h.hexdigest()[:16] == digest else None
+    nbytes, kernel_files, digest = entry
+    return nbytes if source_hash(kernel_files) == digest else None
 
 
 def kernels_per_step(w, sms):

@@ -104,6 +104,10 @@ __global__ void __launch_bounds__(kStThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // programmatic dependent launch: no global access before the previous
+  // launch on the stream has completed; the chunk kernel may launch now
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // producer: K_0, V_0, K_1, V_1, ...
@@ -274,6 +278,10 @@ __global__ void __launch_bounds__(kChThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // the segment states come from the previous launch: wait for it before any
+  // global access; the next launch may begin its set-up
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -573,18 +581,30 @@ cudaError_t run(const LaunchArgs& a) {
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
   const unsigned bh = static_cast<unsigned>(p.BH);
   cudaError_t err;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = a.stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   if (p.splits > 1) {
     auto kern = causal_state_kernel<FMAP>;
     if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kStSmem)) != cudaSuccess) return err;
-    kern<<<dim3(p.splits - 1, bh), kStThreads, kStSmem, a.stream>>>(*a.tm_k, *a.tm_v, state, status,
-                                                              p.tiles_per_split, p.splits);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    cfg.gridDim = dim3(p.splits - 1, bh);
+    cfg.blockDim = dim3(kStThreads);
+    cfg.dynamicSmemBytes = kStSmem;
+    if ((err = cudaLaunchKernelEx(&cfg, kern, *a.tm_k, *a.tm_v, state, status, p.tiles_per_split, p.splits)) !=
+        cudaSuccess)
+      return err;
   }
   auto kern = causal_chunk_kernel<FMAP>;
   if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kChSmem)) != cudaSuccess) return err;
-  kern<<<dim3(p.splits, bh), kChThreads, kChSmem, a.stream>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, state, status,
-                                                               p.N, p.tiles, p.tiles_per_split, p.splits, p.eps);
-  return cudaGetLastError();
+  cfg.gridDim = dim3(p.splits, bh);
+  cfg.blockDim = dim3(kChThreads);
+  cfg.dynamicSmemBytes = kChSmem;
+  return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, static_cast<const float*>(state),
+                            status, p.N, p.tiles, p.tiles_per_split, p.splits, p.eps);
 }
 
 }  // namespace

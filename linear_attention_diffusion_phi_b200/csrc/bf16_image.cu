@@ -24,6 +24,8 @@ namespace {
 __global__ void __launch_bounds__(256)
     image_combine_kernel(const float* __restrict__ part_kv, const float* __restrict__ part_ks,
                          uint8_t* __restrict__ image, int nsplit, int D, int fpart, int parts) {
+  pdl_wait();                // the partials come from the previous launch
+  pdl_launch_dependents();   // the apply may begin its set-up
   const int bh = blockIdx.x;
   const int F = fpart * parts, chunks_per_row = F / 8;
   const int rows = D + 16, atom = rows * 128;
@@ -75,9 +77,16 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_image_combine(const float* part_kv, const float* part_ks, uint8_t* image, long long BH, int nsplit,
                                  int D, int fpart, int parts, cudaStream_t stream) {
   const int chunks = (D + 16) * fpart * parts / 8;
-  const dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((chunks + 255) / 256));
-  image_combine_kernel<<<grid, 256, 0, stream>>>(part_kv, part_ks, image, nsplit, D, fpart, parts);
-  return cudaGetLastError();
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(BH), static_cast<unsigned>((chunks + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, image_combine_kernel, part_kv, part_ks, image, nsplit, D, fpart, parts);
 }
 
 }  // namespace la

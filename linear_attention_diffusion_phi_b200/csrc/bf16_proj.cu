@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(kS1Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // programmatic dependent launch: no global access before the previous
+  // launch has completed; the combine may launch now
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -307,6 +311,9 @@ __global__ void __launch_bounds__(kS3Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // the image comes from the previous launch: wait before any global access
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -445,24 +452,33 @@ cudaError_t run(const LaunchArgs& a) {
   const unsigned bh = static_cast<unsigned>(p.BH);
   const int w_per_head = a.w_head_stride != 0;
   cudaError_t err;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = a.stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   {
     auto kern = proj_state_kernel<FMAP>;
     if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kS1Smem)) != cudaSuccess) return err;
-    kern<<<dim3(p.splits, bh, 2), kS1Threads, kS1Smem, a.stream>>>(*a.tm_k, *a.tm_v, *a.tm_w, part_kv, part_ks,
-                                                                    status, p.N, p.H, w_per_head, p.tiles,
-                                                                    p.tiles_per_split);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    cfg.gridDim = dim3(p.splits, bh, 2);
+    cfg.blockDim = dim3(kS1Threads);
+    cfg.dynamicSmemBytes = kS1Smem;
+    if ((err = cudaLaunchKernelEx(&cfg, kern, *a.tm_k, *a.tm_v, *a.tm_w, part_kv, part_ks, status, p.N, p.H,
+                                  w_per_head, p.tiles, p.tiles_per_split)) != cudaSuccess)
+      return err;
   }
   if ((err = launch_image_combine(part_kv, part_ks, image, p.BH, p.splits, kD, kFH, 2, a.stream)) != cudaSuccess)
     return err;
-  {
-    auto kern = proj_apply_kernel<FMAP>;
-    if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kS3Smem)) != cudaSuccess) return err;
-    kern<<<dim3(p.apply_ctas, bh), kS3Threads, kS3Smem, a.stream>>>(
-        *a.tm_q, *a.tm_w, image, static_cast<__nv_bfloat16*>(a.out), status, p.N, p.H, w_per_head, p.tiles,
-        p.apply_tps, p.eps);
-  }
-  return cudaGetLastError();
+  auto kern = proj_apply_kernel<FMAP>;
+  if ((err = ensure_smem_attr(reinterpret_cast<const void*>(kern), kS3Smem)) != cudaSuccess) return err;
+  cfg.gridDim = dim3(p.apply_ctas, bh);
+  cfg.blockDim = dim3(kS3Threads);
+  cfg.dynamicSmemBytes = kS3Smem;
+  return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_w, static_cast<const uint8_t*>(image),
+                            static_cast<__nv_bfloat16*>(a.out), status, p.N, p.H, w_per_head, p.tiles, p.apply_tps,
+                            p.eps);
 }
 
 }  // namespace
