@@ -203,6 +203,27 @@ def dist_env():
     return ws, rank, local
 
 
+def input_seed(w, i, rank):
+    """Seed of input set i on `rank`: every rank streams its own replica."""
+    return w.seed + 7919 * i + 104729 * rank
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank float values over the process group (the
+    job's time is its slowest rank's); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(tokens_per_rank, world_size, steps, ms_total):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world_size / (ms_total / 1e3 / steps)
+
+
 def run_reference(args, w):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -276,7 +297,7 @@ def main():
     nsets = max(2, -(-3 * L2_BYTES // set_bytes))
     sets = []
     for i in range(nsets):
-        q, k, v, W = make_inputs(w, seed=w.seed + 7919 * i + 104729 * rank)
+        q, k, v, W = make_inputs(w, seed=input_seed(w, i, rank))
         sets.append((q.to(dev), k.to(dev), v.to(dev), torch.empty_like(q, device=dev)))
     Wd = None if W is None else W.to(dev)
     op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, Wd)
@@ -371,10 +392,7 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = ev0.elapsed_time(ev1)
 
-    t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
     if ws > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -382,7 +400,7 @@ def main():
 
     tokens = w.tokens * ws
     per_step_s = ms / 1e3 / args.steps
-    value = tokens / per_step_s
+    value = job_throughput(w.tokens, ws, args.steps, ms)
     hbm, tflops, src = peaks()
     abytes = algorithmic_bytes(w)
     achieved = abytes / per_step_s / 1e9

@@ -19,6 +19,8 @@ LA_PHI_ELU1, LA_PHI_RELU = 0, 1
 FEATURE_MAPS = {"elu": LA_PHI_ELU1, "relu": LA_PHI_RELU}
 
 LA_OK = 0
+(LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_MISALIGNED, LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_TIMEOUT,
+ LA_ERR_NO_DEVICE) = range(1, 8)
 STATUS_NAMES = {
     0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_MISALIGNED",
     4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT", 7: "LA_ERR_NO_DEVICE",
