@@ -37,15 +37,8 @@ struct Plan {
   int apply_ctas, apply_tps;   // bf16 projected: apply CTAs per head, 128-token tiles each
   // workspace layout (byte offsets from the workspace base, 256-aligned)
   size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
-  size_t blob_bytes;   // bf16 B-operand image per head
+  size_t blob_bytes;   // bf16 [kv | ksum | 0]^T image per head (projected path)
 };
-
-// Per-head layout of the bf16 [kv | ksum | 0] B-operand image used by the
-// apply kernels: MN-major, 128-byte swizzle, N atoms of 64 columns.
-__host__ __device__ constexpr int blob_atoms(int D) { return (D + 16 + 63) / 64; }
-__host__ __device__ constexpr size_t blob_bytes_for(int D, int Fe) {
-  return static_cast<size_t>(blob_atoms(D)) * Fe * 128;
-}
 
 struct LaunchArgs {
   const Plan* p;
