@@ -28,6 +28,12 @@
  *
  * Asynchrony.  la_forward only enqueues kernels on the given stream (a
  * cudaStream_t passed as void*, NULL = legacy default stream) and returns.
+ * The bf16 kernels are launched with programmatic dependent launch: they may
+ * start their set-up while earlier work on the stream is finishing, but touch
+ * no global memory before it has completed; they also let the next launch on
+ * the stream start early, so a following kernel that is itself launched with
+ * programmatic serialization must wait (griddepcontrol.wait) before it reads
+ * out.  Ordinary launches are ordered as usual.
  *
  * Errors.  Argument errors are detected on the host before anything is
  * enqueued; out is then untouched.  Launch failures return LA_ERR_CUDA.
