@@ -133,8 +133,8 @@ la_status_t la_sync_status(la_handle_t handle, void* stream);
  * pages have no counterpart; this entry point exists only for such callers.
  * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward; D is 64
  * or 128.  No handle is used and nothing is allocated, on host or device.
- * The scratch this path needs (a status word and per-head barrier words,
- * about 1 MiB) does not grow with N, so every supported shape fits; a plan
+ * The scratch this path needs (its status word, 256 bytes) does not grow
+ * with the problem, so every supported shape fits; a plan
  * that needed more than the array would return LA_ERR_WORKSPACE before
  * anything is enqueued.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first

@@ -139,7 +139,6 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
   }
   size_t off = 0;
   p->off_status = off;        off += la::kStatusBytes;
-  p->off_sync = off;          off += la::kSyncBytes;
   p->off_partial = off;       off = align256(off + partial_floats * 4);
   p->off_ksum_partial = off;  off = align256(off + ksum_floats * 4);
   p->off_final = off;         off = align256(off + final_bytes);
@@ -191,8 +190,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 namespace la {
 
 // Plan of the fused cluster kernel (la_forward_noalloc): the combine runs
-// through distributed shared memory, so the workspace is only the header
-// (status word and per-head barrier words).
+// through distributed shared memory, so the workspace is only the status word.
 void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p) {
   memset(p, 0, sizeof(*p));
   p->dtype = LA_BF16;
@@ -203,7 +201,6 @@ void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int nu
   p->num_sms = num_sms > 0 ? num_sms : 148;
   size_t off = 0;
   p->off_status = off;        off += la::kStatusBytes;
-  p->off_sync = off;          off += la::kSyncBytes;
   p->off_partial = p->off_ksum_partial = p->off_final = p->off_final_ksum = p->off_blob = off;
   p->bytes = off;
 }
@@ -299,9 +296,8 @@ la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
   }
   if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return LA_ERR_MISALIGNED;
   if (bytes < la::kHeaderBytes) return LA_ERR_WORKSPACE;
-  // Clear the status word and the barrier words once: later reads see only
-  // errors of calls made with this workspace, and every barrier count starts
-  // (and, after each completed barrier, returns) at zero.
+  // Clear the status word once: later reads see only errors of calls made
+  // with this workspace.
   if (cudaMemset(ptr, 0, la::kHeaderBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;

@@ -15,11 +15,9 @@ constexpr int kDeviceTimeout = 6;                            // == LA_ERR_TIMEOU
 
 constexpr int kTileTokens = 128;   // tokens per tensor-core tile (MMA M or K)
 
-// Workspace header: a 256-byte status area, then barrier words for up to
-// 65536 heads (16 bytes each).  Zeroed when the workspace is bound.
+// Workspace header: a 256-byte status area, zeroed when the workspace is bound.
 constexpr size_t kStatusBytes = 256;
-constexpr size_t kSyncBytes = 65536 * 16;
-constexpr size_t kHeaderBytes = kStatusBytes + kSyncBytes;
+constexpr size_t kHeaderBytes = kStatusBytes;
 
 // Everything la_forward decides on the host, shared with la_workspace_bytes.
 struct Plan {
@@ -33,10 +31,9 @@ struct Plan {
   int tiles_per_split;   // in 128-token tiles (bf16) or tokens per split (f32, see seg_len)
   int seg_len;     // tokens per split/segment
   int num_sms;
-  int heads_per_cta;   // bf16 non-causal: heads whose splits one CTA owns (1 or 2)
   int apply_ctas, apply_tps;   // bf16 projected: apply CTAs per head, 128-token tiles each
   // workspace layout (byte offsets from the workspace base, 256-aligned)
-  size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
+  size_t off_status, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
   size_t blob_bytes;   // bf16 [kv | ksum | 0]^T image per head (projected path)
 };
 

@@ -19,8 +19,7 @@ namespace {
 
 constexpr size_t kScratchBytes = LA_NOALLOC_SCRATCH_BYTES;
 
-// Scratch for la_forward_noalloc: partial states, per-head operand images and
-// the status word.  In host code this name is only a handle for
+// Scratch for la_forward_noalloc: the status word of its kernel.  In host code this name is only a handle for
 // cudaGetSymbolAddress, never a device address.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -73,10 +72,9 @@ extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const vo
   void* scratch = nullptr;
   if (!scratch_address(&scratch)) return LA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents; the status word and this
-  // problem's barrier words must start at zero (every other byte the kernels
-  // read is written first).
-  if (cudaMemsetAsync(static_cast<char*>(scratch), 0, p.off_sync + static_cast<size_t>(p.BH) * 16, s) !=
+  // The array keeps the previous call's contents; the status word must start
+  // at zero (the kernel reads nothing else from it).
+  if (cudaMemsetAsync(static_cast<char*>(scratch), 0, p.off_status + la::kStatusBytes, s) !=
       cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;

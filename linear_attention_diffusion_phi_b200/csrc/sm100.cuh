@@ -168,17 +168,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate).
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on `bar` once every previously issued tcgen05.mma of this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -213,9 +202,11 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-// The same two MMAs with the accumulate flag as an immediate (ACC = 0
-// overwrites D, 1 accumulates) and descriptors the caller precomputes: the
-// issuing thread then spends a few cycles per MMA instead of several tens.
+// D[tmem] (+)= A * B, kind::f16 (bf16 inputs, fp32 accumulate), A and B in
+// shared memory (umma_ss) or A in tensor memory (umma_ts).  The accumulate
+// flag is an immediate (ACC = 0 overwrites D, 1 accumulates) and the caller
+// precomputes the descriptors: the issuing thread then spends a few cycles
+// per MMA instead of several tens.
 template <int ACC>
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
   asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, %4;" ::"r"(d_tmem), "l"(adesc), "l"(bdesc),
@@ -223,6 +214,9 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_
                : "memory");
 }
 
+// A in tensor memory (M = 128): row m in lane m, the 16-bit K elements two
+// per 32-bit column, element k in the low half of column k / 2 when k is
+// even; one K step of 16 reads 8 columns.
 template <int ACC>
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
   asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, %4;" ::"r"(d_tmem), "r"(a_tmem),
@@ -258,19 +252,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// D[tmem] (+)= A[tmem] * B[smem], kind::f16.  A (M = 128) sits with row m in
-// lane m and its 16-bit K elements two per 32-bit column, element k in the
-// low half of column k / 2 when k is even; one K step of 16 reads 8 columns.
-__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // ---------------------------------------------------- descriptors (sm_100 UMMA)
 
@@ -321,21 +302,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// elu(x)+1 with alpha = 1 (x + 1 for x > 0, exp(x) otherwise), or relu.
-template <int FMAP>
-__device__ __forceinline__ float phi_fast(float x) {
-  if (FMAP == 0) return x > 0.f ? x + 1.f : __expf(x);
-  return fmaxf(x, 0.f);
-}
-
+// elu(x)+1 with alpha = 1 (x + 1 for x > 0, exp(x) otherwise), or relu, with
+// the accurate expf (the fp32 path).
 __device__ __forceinline__ float phi_accurate(float x, int fmap) {
   if (fmap == 0) return x > 0.f ? x + 1.f : expf(x);
   return fmaxf(x, 0.f);
 }
-
-}  // namespace la
-
-namespace la {
 
 // ------------------------------------------------------------------ clusters
 
@@ -390,7 +362,6 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v) {
                : "memory");
 }
 
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 // Split whole-cluster barrier: a relaxed arrive (no ordering of this thread's
 // earlier accesses, so outstanding TMA loads do not delay it) and an acquiring
@@ -414,82 +385,6 @@ __device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   return d;   // layout type 0: no swizzle
-}
-
-}  // namespace la
-
-namespace la {
-
-// ------------------------------------------- grid-wide head barriers (global)
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Split-phase form of grid_barrier: arrive returns the generation to wait on
-// (taken before arriving, so it cannot have moved yet); the last of the n
-// arrivals resets the count and advances the generation.
-__device__ __forceinline__ unsigned grid_arrive(unsigned* count, unsigned* gen, unsigned n) {
-  const unsigned g = ld_acquire_gpu(gen);
-  const unsigned arrived = atom_add_acq_rel_gpu(count, 1u);
-  if (arrived == n - 1) {
-    st_relaxed_gpu(count, 0u);
-    red_add_release_gpu(gen, 1u);
-  }
-  return g;
-}
-
-// Bounded wait until the generation has moved past g.
-__device__ __forceinline__ bool grid_wait(unsigned* gen, unsigned g, int* status) {
-  if (ld_acquire_gpu(gen) != g) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(gen) == g) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(status, kDeviceTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-
-// Sense-reversing barrier among the `n` CTAs that share (count, gen); called
-// by one thread per CTA once the CTA's writes are complete.  `count` returns
-// to 0 every time the barrier completes; `gen` only grows.  All n CTAs must be
-// resident at once (cooperative launch).  Bounded: gives up after
-// kWaitLimitNs, records LA_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned n, int* status) {
-  const unsigned g = ld_acquire_gpu(gen);
-  const unsigned arrived = atom_add_acq_rel_gpu(count, 1u);
-  if (arrived == n - 1) {
-    st_relaxed_gpu(count, 0u);
-    red_add_release_gpu(gen, 1u);
-    return true;
-  }
-  if (ld_acquire_gpu(gen) != g) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(gen) == g) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(status, kDeviceTimeout);
-      return false;
-    }
-  }
-  return true;
 }
 
 }  // namespace la

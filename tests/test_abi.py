@@ -120,18 +120,18 @@ def test_projection_validation(handles):
 def test_workspace_bytes_and_binding(handles):
     for name, h in handles.items():
         n = la.la_workspace_bytes(h, 1, 24, 4608, 128 if name == "bf16" else 64, 0, 0)
-        assert n > 256 and n % 256 == 0
+        assert n >= 256 and n % 256 == 0
         assert n < 64 << 20
         assert la.la_workspace_bytes(h, 1, 24, 4608, 130, 0, 0) == 0
     h = handles["bf16"]
     # the bf16 non-causal F = 0 path reduces states in distributed shared
-    # memory: only the header (status word + barrier words) is needed
+    # memory: only the header (the status word) is needed
     n = la.la_workspace_bytes(h, 1, 24, 4608, 128, 0, 0)
-    assert n == 256 + (1 << 20)
+    assert n == 256
     assert la.la_workspace_bytes(h, 1, 24, 4608, 128, 256, 0) >= n
     # bf16 causal: the header plus one [D + 1][D] fp32 state per (segment, head)
     nc = la.la_workspace_bytes(h, 4, 8, 32768, 64, 0, 1)
-    assert nc >= 256 + (1 << 20) + 32 * 2 * 65 * 64 * 4 and nc < 64 << 20
+    assert nc >= 256 + 32 * 3 * 65 * 64 * 4 and nc < 64 << 20
     assert la.la_set_workspace(h, 0x1010, 4096) == 3          # not 256-aligned
     assert la.la_set_workspace(h, None, 0) == 0
     assert la.la_sync_status(h, None) == 4                    # no workspace bound
