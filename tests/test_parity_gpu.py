@@ -320,3 +320,95 @@ def test_host_buffer_entry_point_matches_device_path():
     assert st == la.LA_OK
     torch.cuda.synchronize()
     assert torch.equal(oh, ref)
+
+
+# ------------------------------------------- many heads, up to the grid limit
+
+MANY_HEAD_CASES = [
+    # more heads than clusters of two CTAs fit at once: one CTA per head, in waves
+    dict(B=2, H=100, N=1000, D=128),
+    dict(B=1, H=150, N=4607, D=64, fmap="relu"),
+    # causal and projected: one segment / split per head, in waves
+    dict(B=2, H=100, N=700, D=64, causal=True),
+    dict(B=2, H=90, N=300, D=128, F=256),
+    # B*H = 65535, the largest the library accepts (a grid's y extent)
+    dict(B=3, H=21845, N=3, D=64),
+    dict(B=3, H=21845, N=3, D=64, causal=True, fmap="relu"),
+]
+
+
+@pytest.mark.parametrize("case", MANY_HEAD_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_many_heads(case):
+    """More heads than the device holds at once, up to B*H = 65535; every
+    output element against the oracle."""
+    w = Workload("bf16heads", seed=93, **case)
+    check_workload(w)
+
+
+def test_bf16_projected_grid_limit_shared_matrix():
+    """Projected path at B*H = 65535 with one W for every head."""
+    import torch
+    w = Workload("bf16projmax", B=1, H=65535, N=3, D=128, seed=94)
+    q, k, v, _ = make_inputs(w)
+    _, _, _, W = make_inputs(Workload("bf16projW", B=1, H=1, N=1, D=128, F=256, seed=95))
+    W0 = W[0]
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, "elu", w.eps, False, W0.to(dev))
+    got = op(q.to(dev), k.to(dev), v.to(dev)).cpu()
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    ref = ora.forward(as_float64(q), as_float64(k), as_float64(v), "elu", w.eps, False, as_float64(W0))
+    assert_parity(got, ref, "bf16")
+
+
+# ------------------------------------- degenerate rows and a closed form
+
+EMPTY_ROW_CASES = [dict(D=128), dict(D=64, causal=True), dict(D=128, F=256)]
+
+
+@pytest.mark.parametrize("case", EMPTY_ROW_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_relu_empty_rows(case):
+    """Under relu a query with no positive feature has no weight on any key,
+    so its output row is exactly 0 (0 / eps); the other rows follow the
+    oracle.  A zero query row is such a query with or without a projection."""
+    import torch
+    w = Workload("bf16empty", B=1, H=2, N=700, fmap="relu", seed=96, **case)
+    q, k, v, W = make_inputs(w)
+    rows = [0, 127, 128, 699]
+    q[:, :, rows] = 0
+    if not w.F:
+        q[0, 1, 300] = -q[0, 1, 300].abs()
+        rows_h1 = rows + [300]
+    else:
+        rows_h1 = rows
+    got = run_gpu(w, q, k, v, W)
+    assert torch.all(got[0, 0, rows] == 0) and torch.all(got[0, 1, rows_h1] == 0)
+    assert_parity(got, oracle_full(w, q, k, v, W), "bf16")
+
+
+CLOSED_FORM_CASES = [dict(D=128), dict(D=64, causal=True), dict(D=128, F=256)]
+
+
+@pytest.mark.parametrize("case", CLOSED_FORM_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_zero_qk_closed_form(case):
+    """Q = K = 0 under elu+1 makes every feature elu(0) + 1 = 1, with or
+    without a projection, so every weight is F and out_i is the mean of the
+    values row i sees, times s_i / (s_i + eps) with s_i = F * (keys seen): the
+    mean of all rows, or causally the running mean.  Computed here from that
+    closed form, not by the oracle."""
+    import torch
+    w = Workload("bf16closed", B=2, H=2, N=1500, seed=97, **case)
+    _, _, v, W = make_inputs(w)
+    q = torch.zeros_like(v)
+    got = as_float64(run_gpu(w, q, q.clone(), v, W))
+    vf = as_float64(v)
+    fe = w.F or w.D
+    if w.causal:
+        seen = np.arange(1, w.N + 1, dtype=np.float64)[None, None, :, None]
+        mean = np.cumsum(vf, axis=2) / seen
+    else:
+        seen = float(w.N)
+        mean = np.broadcast_to(vf.mean(axis=2, keepdims=True), vf.shape)
+    s = fe * seen
+    assert_parity(got, mean * (s / (s + w.eps)), "bf16")
