@@ -334,11 +334,15 @@ MANY_HEAD_CASES = [
     # B*H = 65535, the largest the library accepts (a grid's y extent)
     dict(B=3, H=21845, N=3, D=64),
     dict(B=3, H=21845, N=3, D=64, causal=True, fmap="relu"),
+    # the fp32 path at the same limits
+    dict(B=3, H=21845, N=3, D=36, dtype="f32"),
+    dict(B=3, H=21845, N=5, D=16, causal=True, fmap="relu", dtype="f32"),
+    dict(B=2, H=100, N=300, D=64, F=256, causal=True, dtype="f32"),
 ]
 
 
 @pytest.mark.parametrize("case", MANY_HEAD_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
-def test_bf16_many_heads(case):
+def test_many_heads(case):
     """More heads than the device holds at once, up to B*H = 65535; every
     output element against the oracle."""
     w = Workload("bf16heads", seed=93, **case)
