@@ -22,7 +22,10 @@
  * device that is current when la_forward is called.
  *
  * Layout.  q, k, v and out are dense row-major [B, H, N, D] tensors (D
- * innermost), all of the handle's dtype; out never aliases q, k or v.
+ * innermost), all of the handle's dtype.  q, k and v are only read and may
+ * coincide; out shares no byte with q, k, v, the part of W the call reads or
+ * the workspace, nor the workspace with q, k, v or W (la_forward checks the
+ * address ranges and returns LA_ERR_INVALID_ARG otherwise).
  * W is [H, D, F] row-major (F innermost) with head stride head_stride
  * elements (0: one matrix shared by all heads).
  *
@@ -56,7 +59,8 @@ typedef struct la_handle_s* la_handle_t;
 
 typedef enum {
   LA_OK = 0,
-  LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, eps < 0, bad enum */
+  LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, eps < 0, bad enum,
+                               an output overlapping an input                  */
   LA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape/dtype this build runs   */
   LA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
   LA_ERR_WORKSPACE = 4,     /* no workspace bound, or it is too small         */
@@ -109,8 +113,10 @@ la_status_t la_forward(la_handle_t handle, const void* q, const void* k, const v
 
 /* End-to-end variant over HOST buffers: copies q, k, v (host, pinned for
  * asynchrony) into the caller's device buffers dq, dk, dv, runs la_forward into
- * dout and copies dout back to out_host, all enqueued on `stream`.  The host
- * buffers must stay valid until the stream reaches the end of the copies. */
+ * dout and copies dout back to out_host, all enqueued on `stream`.  dq, dk, dv
+ * and dout are [B, H, N, D] device buffers that share no byte (else
+ * LA_ERR_INVALID_ARG).  The host buffers must stay valid until the stream
+ * reaches the end of the copies. */
 la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* k_host,
                             const void* v_host, void* out_host, void* dq, void* dk, void* dv,
                             void* dout, int B, int H, int N, int D, int F, int feature_map,
@@ -131,8 +137,8 @@ la_status_t la_sync_status(la_handle_t handle, void* stream);
  * F = 0 forward of la_forward, with its scratch in a static device array of
  * LA_NOALLOC_SCRATCH_BYTES inside this library instead of a workspace.  The
  * pages have no counterpart; this entry point exists only for such callers.
- * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward; D is 64
- * or 128.  No handle is used and nothing is allocated, on host or device.
+ * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward (out
+ * overlapping q, k or v gives LA_ERR_INVALID_ARG); D is 64 or 128.  No handle is used and nothing is allocated, on host or device.
  * The scratch this path needs (its status word, 256 bytes) does not grow
  * with the problem, so every supported shape fits; a plan
  * that needed more than the array would return LA_ERR_WORKSPACE before

@@ -179,10 +179,30 @@ class LinearAttention:
             self._ws = self.torch.empty(need, dtype=self.torch.uint8, device=device)
             check(la_set_workspace(self.handle, self._ws.data_ptr(), self._ws.numel()), "la_set_workspace")
 
+    def _check_tensors(self, q, k, v, out):
+        # the library sees only base pointers: every tensor must be a dense
+        # [B, H, N, D] array of the operator's dtype on one CUDA device
+        if q.dim() != 4:
+            raise ValueError(f"q: expected [B, H, N, D], got shape {tuple(q.shape)}")
+        ts = (("q", q), ("k", k), ("v", v), ("out", out))
+        for name, t in ts:
+            if t.shape != q.shape:
+                raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(q.shape)}")
+        for name, t in ts:
+            if t.dtype != self.dtype:
+                raise ValueError(f"{name}: dtype {t.dtype}, the operator's is {self.dtype}")
+        for name, t in ts:
+            if not t.is_contiguous():
+                raise ValueError(f"{name}: must be contiguous (row-major [B, H, N, D])")
+        for name, t in ts:
+            if t.device.type != "cuda" or t.device != q.device:
+                raise ValueError(f"{name}: on {t.device}, expected one CUDA device for all tensors")
+
     def __call__(self, q, k, v, out=None, stream=None):
-        B, H, N, D = q.shape
         if out is None:
             out = self.torch.empty_like(q)
+        self._check_tensors(q, k, v, out)
+        B, H, N, D = q.shape
         self._bind_workspace(B, H, N, D, q.device)
         s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
         check(la_forward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),

@@ -230,6 +230,11 @@ cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes) {
   return err;
 }
 
+bool overlap(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return an != 0 && bn != 0 && x < y + bn && y < x + an;
+}
+
 bool current_sm100(int* num_sms) {
   DeviceInfo di;
   if (!device_info(&di) || di.major != 10 || di.minor != 0) return false;
@@ -319,6 +324,24 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
     if (!h->W) return LA_ERR_INVALID_ARG;
     if (h->wD != D || h->wF != F || (h->w_head_stride != 0 && h->wH < H)) return LA_ERR_INVALID_ARG;
   }
+  // The kernels write out and the workspace while q, k, v and W are still
+  // being read, so neither may share a byte with them or with each other; q,
+  // k and v are only read and may coincide.
+  {
+    const size_t es = h->dtype == LA_F32 ? 4 : 2;
+    const size_t nb = static_cast<size_t>(B) * H * N * D * es;
+    const size_t wb = F == 0 ? 0
+                      : (h->w_head_stride ? static_cast<size_t>(H - 1) * h->w_head_stride : 0) * es +
+                            static_cast<size_t>(D) * F * es;
+    const void* ins[3] = {q, k, v};
+    for (const void* x : ins) {
+      if (la::overlap(out, nb, x, nb)) return LA_ERR_INVALID_ARG;
+      if (h->ws && la::overlap(h->ws, h->ws_bytes, x, nb)) return LA_ERR_INVALID_ARG;
+    }
+    if (F > 0 && la::overlap(out, nb, h->W, wb)) return LA_ERR_INVALID_ARG;
+    if (h->ws && (la::overlap(h->ws, h->ws_bytes, out, nb) || (F > 0 && la::overlap(h->ws, h->ws_bytes, h->W, wb))))
+      return LA_ERR_INVALID_ARG;
+  }
   DeviceInfo di;
   if (!device_info(&di)) return LA_ERR_NO_DEVICE;
   if (di.major != 10 || di.minor != 0) return LA_ERR_NO_DEVICE;   // kernels are built for sm_100a
@@ -370,6 +393,12 @@ la_status_t la_forward_host(la_handle_t h, const void* q_host, const void* k_hos
   const size_t n = static_cast<size_t>(B) * H * N * D * (h->dtype == LA_F32 ? 4 : 2);
   if (n == 0) return LA_OK;
   if (!q_host || !k_host || !v_host || !out_host) return LA_ERR_INVALID_ARG;
+  if (!dq || !dk || !dv || !dout) return LA_ERR_INVALID_ARG;
+  // dq, dk and dv are copy destinations and dout the output: all disjoint
+  void* const dev[4] = {dq, dk, dv, dout};
+  for (int i = 0; i < 4; ++i)
+    for (int j = i + 1; j < 4; ++j)
+      if (la::overlap(dev[i], n, dev[j], n)) return LA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||

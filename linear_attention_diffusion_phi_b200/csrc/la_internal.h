@@ -63,6 +63,8 @@ bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, lon
                           long long outer_stride_elems);
 // SM count of the current device; false unless it is an sm_100 device.
 bool current_sm100(int* num_sms);
+// The byte ranges [a, a + an) and [b, b + bn) share at least one byte.
+bool overlap(const void* a, size_t an, const void* b, size_t bn);
 
 // Raise a kernel's dynamic shared-memory limit once per device (thread-safe).
 cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes);

@@ -62,6 +62,10 @@ extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const vo
   if (static_cast<long long>(B) * H * N == 0) return LA_OK;
   if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_MISALIGNED;
+  // out is written while q, k and v are still being read
+  const size_t nb = static_cast<size_t>(B) * H * N * D * 2;
+  if (la::overlap(out, nb, q, nb) || la::overlap(out, nb, k, nb) || la::overlap(out, nb, v, nb))
+    return LA_ERR_INVALID_ARG;
 
   int sms = 0;
   if (!la::current_sm100(&sms)) return LA_ERR_NO_DEVICE;

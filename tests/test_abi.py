@@ -70,7 +70,7 @@ def handles():
         la.la_destroy(h)
 
 
-def fwd(h, B=1, H=2, N=256, D=64, F=0, fmap=0, eps=1e-6, causal=0, ptr=0x1000, out=0x2000):
+def fwd(h, B=1, H=2, N=256, D=64, F=0, fmap=0, eps=1e-6, causal=0, ptr=0x1000, out=0x4000_0000):
     return la.la_forward(h, ptr, ptr, ptr, out, B, H, N, D, F, fmap, eps, causal, None)
 
 
@@ -105,6 +105,33 @@ def test_forward_argument_validation(handles):
     assert fwd(b16, D=128, F=256) == 1
 
 
+def test_outputs_may_not_overlap_inputs(handles):
+    """Checked on the host before anything is enqueued (the addresses here
+    are never dereferenced).  The default problem is 131072 bytes per tensor
+    in fp32, 65536 in bf16."""
+    f32, b16 = handles["f32"], handles["bf16"]
+    nb = 1 * 2 * 256 * 64 * 4
+    assert fwd(f32, ptr=0x1000, out=0x1000) == 1                 # in place
+    assert fwd(f32, ptr=0x1000, out=0x1000 + nb - 16) == 1       # last 16 bytes shared
+    assert fwd(f32, ptr=0x1000 + nb - 16, out=0x1000) == 1
+    assert fwd(f32, ptr=0x1000, out=0x1000 + nb) not in (1, 0)    # adjacent: accepted, then no device / workspace
+    assert fwd(f32, ptr=0x1000 + nb, out=0x1000) not in (1, 0)
+    assert fwd(b16, ptr=0x1000, out=0x1000 + nb // 2 - 16) == 1
+    # q, k and v are only read and may coincide: fwd passes one pointer for all three
+    # la_forward_host: the four device buffers are pairwise disjoint
+    h = 0x9000_0000
+    host = lambda dq, dk, dv, do: la.la_forward_host(f32, h, h, h, h, dq, dk, dv, do, 1, 2, 256, 64, 0, 0, 1e-6, 0,
+                                                    None)
+    assert host(0x1000, 0x1000, 0x100000, 0x200000) == 1
+    assert host(0x1000, 0x100000, 0x200000, 0x200000 + nb - 16) == 1
+    assert host(0, 0x100000, 0x200000, 0x300000) == 1
+    # la_forward_noalloc: out vs q, k, v
+    nbb = 1 * 2 * 256 * 128 * 2
+    call = lambda q, k, v, o: la.la_forward_noalloc(q, k, v, o, 1, 2, 256, 128, 0, 1e-6, None)
+    assert call(0x1000, 0x100000, 0x200000, 0x1000) == 1
+    assert call(0x1000, 0x100000, 0x200000, 0x200000 + nbb - 16) == 1
+
+
 def test_projection_validation(handles):
     h = handles["bf16"]
     assert la.la_set_projection(h, 0x1000, 24, 128, 255, 0) == 1
@@ -113,6 +140,11 @@ def test_projection_validation(handles):
     assert la.la_set_projection(h, 0x1008, 24, 128, 256, 0) == 3
     assert la.la_set_projection(h, 0x1000, 24, 128, 256, 128 * 256) == 0
     assert fwd(h, D=64, F=256) == 2
+    # out may not overlap the part of W the call reads: heads 0..H-1 at the
+    # bound stride, bf16 (two heads here: 2 * 128 * 256 * 2 bytes from 0x1000)
+    wend = 0x1000 + 2 * 128 * 256 * 2
+    assert fwd(h, D=128, F=256, ptr=0x8000_0000, out=wend - 16) == 1
+    assert fwd(h, D=128, F=256, ptr=0x8000_0000, out=wend) not in (1, 0)
     assert la.la_set_projection(h, None, 0, 0, 0, 0) == 0
     assert fwd(h, D=128, F=256) == 1
 
@@ -149,3 +181,24 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(la, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         la.la_version()
+
+
+def test_binding_checks_tensors_before_calling():
+    """The binding hands the library base pointers only, so it refuses
+    tensors that are not dense [B, H, N, D] arrays of its dtype on one CUDA
+    device (all checks on the host; nothing reaches the library)."""
+    torch = pytest.importorskip("torch")
+    op = la.LinearAttention(torch.bfloat16)
+    x = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="expected \\[B, H, N, D\\]"):
+        op(x[0], x[0], x[0])
+    with pytest.raises(ValueError, match="k: shape"):
+        op(x, x[:, :1], x)
+    with pytest.raises(ValueError, match="v: dtype"):
+        op(x, x, x.float())
+    with pytest.raises(ValueError, match="q: must be contiguous"):
+        t = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16).transpose(1, 2)
+        op(t, x, x, out=x.clone())
+    with pytest.raises(ValueError, match="CUDA device"):
+        op(x, x, x)
+    op.close()

@@ -416,3 +416,32 @@ def test_bf16_zero_qk_closed_form(case):
         mean = np.broadcast_to(vf.mean(axis=2, keepdims=True), vf.shape)
     s = fe * seen
     assert_parity(got, mean * (s / (s + w.eps)), "bf16")
+
+
+def test_overlapping_output_is_refused_before_launch():
+    """out on top of q, or inside the bound workspace, is refused on the host
+    with LA_ERR_INVALID_ARG; nothing is enqueued, so every buffer keeps its
+    contents and the next proper call is unaffected."""
+    import torch
+    w = Workload("alias", B=1, H=2, N=1000, D=128, seed=13)
+    q, k, v, _ = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, "elu", w.eps)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    ref = op(qd, kd, vd).clone()
+    ws = op._ws
+    ws_before = ws.clone()
+    s = torch.cuda.current_stream().cuda_stream
+    args = (1, 2, 1000, 128, 0, la.LA_PHI_ELU1, w.eps, 0, s)
+    assert la.la_forward(op.handle, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), qd.data_ptr(), *args) == \
+        la.LA_ERR_INVALID_ARG
+    big = torch.empty(2 * qd.numel() + ws.numel(), dtype=torch.bfloat16, device=dev)
+    op2 = la.LinearAttention(torch.bfloat16, "elu", w.eps)
+    assert la.la_set_workspace(op2.handle, big.data_ptr(), 256) == la.LA_OK
+    assert la.la_forward(op2.handle, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), big.data_ptr(), *args) == \
+        la.LA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.equal(qd.cpu(), q) and torch.equal(ws, ws_before)
+    assert torch.equal(op(qd, kd, vd), ref)
+    op.close()
+    op2.close()
