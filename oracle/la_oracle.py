@@ -14,7 +14,7 @@ groups the product as phi(Q) (phi(K)^T V) and normalises by
 weighted sum, and the grouped form is implemented separately so that each can
 be checked against the other.
 
-Readings of the pages taken here (each one is listed in the design doc):
+Readings taken here where the pages leave a step open:
   * elu is the standard ELU with alpha = 1, so elu(x)+1 is x+1 for x > 0 and
     exp(x) for x <= 0 (page "NNT Define Linear Attention", "The inputs").
   * eps is added once per query row to the summed weights (same page, "How it
