@@ -89,3 +89,33 @@ def test_oracle_module_spec_is_standalone():
         src = fh.read()
     assert "linear_attention_diffusion_phi_b200" not in src
     assert spec is not None
+
+
+def test_grouped_form_equals_definition_on_random_shapes():
+    """The identity the fast path rests on, sum_j (phi(q).phi(k_j)) v_j =
+    phi(q)^T (sum_j phi(k_j) v_j^T), over random shapes the fixed pins do not
+    reach: one token, value width unlike the key width, odd feature counts,
+    eps from 0 to large (eps = 0 only under elu+1, whose weights are > 0)."""
+    import numpy as np
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=80, deadline=None, database=None, derandomize=True)
+    @given(N=st.integers(1, 24), D=st.integers(1, 8), Dv=st.integers(1, 8), F=st.sampled_from([0, 3, 16]),
+           fmap=st.sampled_from(["elu", "relu"]), causal=st.booleans(), eps=st.sampled_from([0.0, 1e-6, 0.5]),
+           shared_w=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
+    def check(N, D, Dv, F, fmap, causal, eps, shared_w, seed):
+        if eps == 0.0 and fmap == "relu":
+            eps = 1e-6
+        rng = np.random.default_rng(seed)
+        q = rng.standard_normal((1, 2, N, D))
+        k = rng.standard_normal((1, 2, N, D))
+        v = rng.standard_normal((1, 2, N, Dv))
+        W = None
+        if F:
+            W = rng.standard_normal((D, F) if shared_w else (2, D, F)) / np.sqrt(D)
+        a = la_oracle.forward(q, k, v, fmap, eps, causal, W)
+        b = la_oracle.brute_force(q, k, v, fmap, eps, causal, W)
+        assert a.shape == (1, 2, N, Dv)
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+
+    check()
