@@ -118,7 +118,8 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
     p->tiles_per_split = static_cast<int>(cdiv(tiles, std::min<long long>(want, tiles)));
     p->splits = static_cast<int>(cdiv(tiles, p->tiles_per_split));
     p->seg_len = p->tiles_per_split * la::kTileTokens;
-    partial_floats = static_cast<size_t>(BH) * p->splits * (D + 1) * D;
+    // with one segment per head no state is written or read
+    if (p->splits > 1) partial_floats = static_cast<size_t>(BH) * p->splits * (D + 1) * D;
   } else {
     // Projected (D = 128, F = 256): state CTAs per (split, head, feature
     // half), about one per SM; apply CTAs about one per SM. Partials are fp32

@@ -164,6 +164,9 @@ def test_workspace_bytes_and_binding(handles):
     # bf16 causal: the header plus one [D + 1][D] fp32 state per (segment, head)
     nc = la.la_workspace_bytes(h, 4, 8, 32768, 64, 0, 1)
     assert nc >= 256 + 32 * 3 * 65 * 64 * 4 and nc < 64 << 20
+    # one segment per head (at least as many heads as SMs): no state at all
+    assert la.la_workspace_bytes(h, 3, 21845, 3, 64, 0, 1) == 256
+    assert la.la_workspace_bytes(h, 2, 100, 700, 64, 0, 1) == 256
     assert la.la_set_workspace(h, 0x1010, 4096) == 3          # not 256-aligned
     assert la.la_set_workspace(h, None, 0) == 0
     assert la.la_sync_status(h, None) == 4                    # no workspace bound
