@@ -164,6 +164,26 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def percentiles_ms(times_ms):
+    """p10 / p50 / p90 of per-call device times (ms)."""
+    t = np.asarray(times_ms, dtype=np.float64)
+    p10, p50, p90 = np.percentile(t, [10, 50, 90])
+    return {"p10": float(p10), "p50": float(p50), "p90": float(p90), "calls": int(t.size)}
+
+
+def per_call_ms(run_one, n, stream):
+    """Device time of each of n single steps, each between its own pair of
+    CUDA events on the launching stream (outside the timed region)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        run_one(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
 def cpu_baseline(w, budget_s=10.0):
     """The float64 oracle, as it stands, on the host cores: whole-problem
     forwards of the same workload until ~budget_s of CPU time has passed."""
@@ -364,6 +384,14 @@ def main():
     clocks = sampler.stop()
     assert op.sync_status() == la.LA_OK, "device-side error during the timed region"
 
+    # distribution of single calls (this rank's), informational: the value
+    # above is the mean over the bracketed steps
+    try:
+        one = (lambda i: step(i)) if args.no_graph else (lambda i: g_one[i % nsets].replay())
+        per_call = percentiles_ms(per_call_ms(one, max(10, min(args.steps, 100)), stream))
+    except Exception as e:   # never let the extra figure cost the bench line
+        per_call = {"error": f"{type(e).__name__}: {e}"[:200]}
+
     # end to end through the host-buffer entry point: pinned host inputs,
     # H2D copies, forward, D2H copy of the result, every step
     qh = [s[0].cpu().pin_memory() for s in sets[:2]]
@@ -428,7 +456,7 @@ def main():
                        "feature_map": w.fmap, "eps": w.eps, "causal": w.causal,
                        "global_batch": w.B * ws, "seq_len": w.N, "parallelism": f"replicas{ws}",
                        "l2": f"{nsets} rotating input sets, {nsets * set_bytes / 2**20:.0f} MiB > 3x L2"},
-            "hbm_gbs": achieved, "roofline": roof, "clocks": clocks, "e2e": e2e,
+            "hbm_gbs": achieved, "roofline": roof, "clocks": clocks, "e2e": e2e, "per_call_ms": per_call,
             "gpu_launches": None if launches is None else launches * args.steps, "launch": "cuda-graph" if not args.no_graph else "host"}
     if not args.no_cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(w)

@@ -70,3 +70,37 @@ def test_two_gloo_ranks(tmp_path):
     assert r[1]["ref_out"] == ""
     line = json.loads(r[0]["ref_out"].strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+def test_per_call_percentiles_and_event_pairing(monkeypatch):
+    """bench.py's per-call figure: one event pair around each single step, read
+    after one synchronize, then p10 / p50 / p90 (CUDA events faked on the CPU,
+    each 'step' advancing a fake device clock by its own duration)."""
+    import sys
+    import types
+    import bench
+
+    clock = [0.0]
+
+    class Ev:
+        def __init__(self, enable_timing=False):
+            self.t = None
+
+        def record(self, stream=None):
+            self.t = clock[0]
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    fake = types.SimpleNamespace(cuda=types.SimpleNamespace(Event=Ev, synchronize=lambda: None))
+    monkeypatch.setitem(sys.modules, "torch", fake)
+    durations = [0.5 + 0.1 * (i % 10) for i in range(20)]
+
+    def run_one(i):
+        clock[0] += durations[i]
+
+    times = bench.per_call_ms(run_one, 20, stream=None)
+    assert times == [pytest.approx(d) for d in durations]
+    p = bench.percentiles_ms(times)
+    assert p["calls"] == 20 and p["p10"] <= p["p50"] <= p["p90"]
+    assert p["p50"] == pytest.approx(0.95)
