@@ -159,6 +159,12 @@ class LinearAttention:
             self.set_projection(W)
 
     def set_projection(self, W):
+        if W.dim() not in (2, 3):
+            raise ValueError(f"W: expected [H, D, F] or [D, F], got shape {tuple(W.shape)}")
+        if W.dtype != self.dtype:
+            raise ValueError(f"W: dtype {W.dtype}, the operator's is {self.dtype}")
+        if W.device.type != "cuda":
+            raise ValueError(f"W: on {W.device}, expected a CUDA tensor")
         if W.dim() == 2:
             H, (D, F), stride = 1, W.shape, 0
         else:
@@ -197,6 +203,8 @@ class LinearAttention:
         for name, t in ts:
             if t.device.type != "cuda" or t.device != q.device:
                 raise ValueError(f"{name}: on {t.device}, expected one CUDA device for all tensors")
+        if self.W is not None and self.W.device != q.device:
+            raise ValueError(f"W: on {self.W.device}, the inputs on {q.device}")
 
     def __call__(self, q, k, v, out=None, stream=None):
         if out is None:

@@ -205,3 +205,10 @@ def test_binding_checks_tensors_before_calling():
     with pytest.raises(ValueError, match="CUDA device"):
         op(x, x, x)
     op.close()
+    # the projection: its dtype must be the operator's, and it must be on a device
+    with pytest.raises(ValueError, match="W: dtype"):
+        la.LinearAttention(torch.bfloat16, W=torch.zeros(2, 128, 256))
+    with pytest.raises(ValueError, match="W: on cpu"):
+        la.LinearAttention(torch.bfloat16, W=torch.zeros(2, 128, 256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="W: expected"):
+        la.LinearAttention(torch.float32, W=torch.zeros(256))

@@ -50,7 +50,8 @@ def test_unfinished_wait_gives_up_and_reports(waitlib):
 def test_sync_status_reports_and_clears_a_recorded_timeout():
     import torch
     la_build.build()
-    w = torch.randn(1, 2, 256, 64, device="cuda:0").to(torch.bfloat16)
+    from linear_attention_diffusion_phi_b200.inputs import Workload, make_inputs
+    w = make_inputs(Workload("status", B=1, H=2, N=256, D=64, seed=31))[0].to("cuda:0")
     op = la.LinearAttention(torch.bfloat16, "elu", 1e-6)
     op(w, w, w)
     torch.cuda.synchronize()
