@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--soak-s", type=float, default=1.5, help="untimed load before timing (clock ramp)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step from the host")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads timed after the headline (1 GPU only)")
+    ap.add_argument("--no-parity", action="store_true", help="skip the oracle comparison of sampled heads")
     return ap.parse_args()
 
 
@@ -184,36 +187,72 @@ def per_call_ms(run_one, n, stream):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def cpu_baseline(w, budget_s=10.0):
-    """The float64 oracle, as it stands, on the host cores: whole-problem
-    forwards of the same workload until ~budget_s of CPU time has passed."""
-    from linear_attention_diffusion_phi_b200.inputs import as_float64, make_inputs
-    from oracle import la_oracle as ora
-    q, k, v, W = make_inputs(w)
-    q, k, v, W = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
-    heads = w.B * w.H
-    per_call = max(1, heads)
-    done_tokens = 0
-    t0 = time.perf_counter()
-    hs = 0
-    while True:
-        b, h = divmod(hs % heads, w.H)
-        sl = (slice(b, b + 1), slice(h, h + 1))
-        Wh = None if W is None else W[h:h + 1]
-        ora.forward(q[sl], k[sl], v[sl], w.fmap, w.eps, w.causal, Wh)
-        done_tokens += w.N
-        hs += 1
-        if time.perf_counter() - t0 >= budget_s and hs >= 1:
-            break
-    dt = time.perf_counter() - t0
+def _limit_blas_threads():
+    """Pool initializer: one BLAS thread per worker process, so that the
+    pool's size is the number of cores the oracle uses."""
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
     except Exception:
-        cores = 1
+        pass
+
+
+def _oracle_head(task):
+    """One head of the workload through the float64 oracle, as it stands."""
+    from oracle import la_oracle as ora
+    q, k, v, W, fmap, eps, causal = task
+    ora.forward(q[None, None], k[None, None], v[None, None], fmap, eps, causal, W)
+    return q.shape[0]
+
+
+def oracle_pool():
+    """A pool of host processes (spawn: safe after CUDA is initialised), one
+    per core this process may run on."""
+    import multiprocessing as mp
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    return mp.get_context("spawn").Pool(cores, initializer=_limit_blas_threads), cores
+
+
+def head_tasks(w, q, k, v, W):
+    """Per-head oracle tasks in (b, h) order, from the stored values (float32
+    holds bf16 values exactly; the oracle upcasts to float64)."""
+    from linear_attention_diffusion_phi_b200.inputs import as_float64
+    qf, kf, vf = (as_float64(x).astype(np.float32) for x in (q, k, v))
+    Wf = None if W is None else as_float64(W).astype(np.float32)
+    tasks = []
+    for b in range(w.B):
+        for h in range(w.H):
+            tasks.append((qf[b, h], kf[b, h], vf[b, h], None if Wf is None else Wf[h], w.fmap, w.eps, w.causal))
+    return tasks
+
+
+def cpu_baseline(w, budget_s=10.0, inputs=None):
+    """The float64 oracle, as it stands, on the host cores: whole heads of the
+    same workload, one head per worker process at a time, until ~budget_s of
+    wall time has passed."""
+    from linear_attention_diffusion_phi_b200.inputs import make_inputs
+    q, k, v, W = inputs if inputs is not None else make_inputs(w)
+    tasks = head_tasks(w, q, k, v, W)
+    pool, cores = oracle_pool()
+    try:
+        pool.map(_oracle_head, tasks[:cores])    # workers started and warm
+        done_tokens, heads = 0, 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            batch = [tasks[(heads + j) % len(tasks)] for j in range(cores)]
+            done_tokens += sum(pool.map(_oracle_head, batch, chunksize=1))
+            heads += len(batch)
+        dt = time.perf_counter() - t0
+    finally:
+        pool.close()
+        pool.join()
     return {"value": done_tokens / dt, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"{hs} heads of {w.name} (N={w.N}, D={w.D}, F={w.F}, causal={int(w.causal)}) "
-                      f"through oracle.forward in {dt:.1f} s", "per_call_heads": per_call}
+            "sample": f"{heads} heads of {w.name} (N={w.N}, D={w.D}, F={w.F}, causal={int(w.causal)}), "
+                      f"one head per process on {cores} processes with one BLAS thread each, {dt:.1f} s",
+            "cores_meaning": "host processes running the oracle at once, one BLAS thread each"}
 
 
 def dist_env():
@@ -245,50 +284,235 @@ def job_throughput(tokens_per_rank, world_size, steps, ms_total):
 
 
 def run_reference(args, w):
+    """The float64 oracle as the reference arm: each step is a bounded sample
+    of the workload, one whole head per host process (every core busy)."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    from linear_attention_diffusion_phi_b200.inputs import as_float64, make_inputs
-    from oracle import la_oracle as ora
-    q, k, v, W = make_inputs(w)
-    q, k, v, W = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
-    heads_per_step = 2   # bounded sample of the workload per step
-    def step(i):
-        for j in range(heads_per_step):
-            hs = (i * heads_per_step + j) % (w.B * w.H)
-            b, h = divmod(hs, w.H)
-            ora.forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], w.fmap, w.eps,
-                        w.causal, None if W is None else W[h:h + 1])
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i)
-    dt = time.perf_counter() - t0
-    tokens = args.steps * heads_per_step * w.N
-    value = tokens / dt
+    from linear_attention_diffusion_phi_b200.inputs import make_inputs
+    tasks = head_tasks(w, *make_inputs(w))
+    pool, cores = oracle_pool()
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
+        def step(i):
+            batch = [tasks[(i * cores + j) % len(tasks)] for j in range(cores)]
+            return sum(pool.map(_oracle_head, batch, chunksize=1))
+        for i in range(getattr(args, "warmup", 0)):
+            step(i)
+        t0 = time.perf_counter()
+        tokens = 0
+        for i in range(args.steps):
+            tokens += step(i)
+        dt = time.perf_counter() - t0
+    finally:
+        pool.close()
+        pool.join()
+    value = tokens / dt
+    sample = f"{cores} of {w.B * w.H} heads per step, one per host process, float64 oracle"
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "warmup": getattr(args, "warmup", 0), "ms_per_step": dt / max(args.steps, 1) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "F": w.F,
-                       "feature_map": w.fmap, "causal": w.causal,
-                       "sample": f"{heads_per_step} heads per step"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-                             "sample": f"{heads_per_step} of {w.B * w.H} heads per step, float64 oracle"},
+                       "feature_map": w.fmap, "causal": w.causal, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
+# bf16 bar (fp32 accumulation), with the self-imposed relative L2 bound; fp32 bar
+BF16_MAX_ABS, BF16_MEAN_ABS, BF16_REL_L2, F32_REL_INF = 2e-2, 2e-3, 1e-2, 1e-5
+
+
+def parity_samples(w):
+    """(b, h, rows) picked for the oracle comparison of a timed workload:
+    whole heads when the oracle's grouped form is cheap (non-causal), else
+    512-row slices (start, a middle stretch, the end) checked row by row
+    against the prefix-masked definition."""
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
+    heads = list(dict.fromkeys(heads))
+    if not w.causal:
+        return [(b, h, None) for b, h in heads]
+    n = w.N
+    sl = sorted(set(range(0, min(512, n))) | set(range(max(0, n // 4 - 256), min(n, n // 4 + 256))) |
+                set(range(max(0, n - 512), n)))
+    return [(b, h, sl) for b, h in heads[:2]]
+
+
+def parity_block(w, q, k, v, W, got):
+    """Error figures of the GPU output `got` against the float64 oracle on
+    the sampled heads / rows (CPU torch tensors of the stored values)."""
+    from linear_attention_diffusion_phi_b200.inputs import as_float64
+    from oracle import la_oracle as ora
+    qf, kf, vf, Wf = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
+    diffs, refs, n_rows = [], [], 0
+    for b, h, rows in parity_samples(w):
+        g = as_float64(got[b, h])
+        Wh = None if Wf is None else Wf[h:h + 1]
+        if rows is None:
+            ref = ora.forward(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1], w.fmap, w.eps,
+                              w.causal, Wh)[0, 0]
+        else:
+            ref = ora.rows(qf, kf, vf, b, h, rows, w.fmap, w.eps, w.causal, None if Wf is None else Wf)
+            g = g[rows]
+        diffs.append(np.abs(g - ref).ravel())
+        refs.append(ref.ravel())
+        n_rows += ref.shape[0]
+    d, r = np.concatenate(diffs), np.concatenate(refs)
+    out = {"max_abs": float(d.max()), "mean_abs": float(d.mean()),
+           "rel_l2": float(np.linalg.norm(d) / max(np.linalg.norm(r), 1e-300)),
+           "rel_inf": float(d.max() / max(np.abs(r).max(), 1e-300)),
+           "ref_rms": float(np.sqrt(np.mean(r * r))),
+           "heads_checked": len(parity_samples(w)), "rows_checked": n_rows}
+    if w.dtype == "bf16":
+        out["bar"] = {"max_abs": BF16_MAX_ABS, "mean_abs": BF16_MEAN_ABS, "rel_l2": BF16_REL_L2}
+        out["pass"] = bool(out["max_abs"] <= BF16_MAX_ABS and out["mean_abs"] <= BF16_MEAN_ABS and
+                           out["rel_l2"] <= BF16_REL_L2)
+        out["margin"] = float(min(BF16_MAX_ABS / max(out["max_abs"], 1e-300),
+                                  BF16_MEAN_ABS / max(out["mean_abs"], 1e-300),
+                                  BF16_REL_L2 / max(out["rel_l2"], 1e-300)))
+    else:
+        out["bar"] = {"rel_inf": F32_REL_INF}
+        out["pass"] = bool(out["rel_inf"] <= F32_REL_INF)
+        out["margin"] = float(F32_REL_INF / max(out["rel_inf"], 1e-300))
+    return out
+
+
+class Timed:
+    """One workload resident on the device: rotating input sets whose total
+    exceeds 3x L2 (set 0 holds the seeded inputs; the others are copies of it
+    shifted along the sequence, so every step reads memory the previous steps
+    did not touch), the operator, and CUDA graphs of its steps."""
+
+    def __init__(self, w, dev, rank, graphs=True):
+        import torch
+        import linear_attention_diffusion_phi_b200 as la
+        from linear_attention_diffusion_phi_b200.inputs import make_inputs
+        self.w = w
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.set_bytes = 4 * w.B * w.H * w.N * w.D * (2 if w.dtype == "bf16" else 4)
+        self.nsets = max(2, -(-3 * L2_BYTES // self.set_bytes))
+        self.host = make_inputs(w, seed=input_seed(w, 0, rank))
+        q, k, v, W = self.host
+        base = (q.to(dev), k.to(dev), v.to(dev))
+        self.sets = [base + (torch.empty_like(base[0]),)]
+        for i in range(1, self.nsets):
+            sh = (97 * i) % max(w.N, 1)
+            self.sets.append(tuple(torch.roll(x, shifts=sh, dims=2) for x in base) + (torch.empty_like(base[0]),))
+        self.op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, None if W is None else W.to(dev))
+        self.graphs = graphs
+        self.g_all = None
+        self.g_one = []
+
+    def step(self, i):
+        q, k, v, o = self.sets[i % self.nsets]
+        self.op(q, k, v, out=o)
+
+    def capture(self):
+        import torch
+        if not self.graphs:
+            return
+        self.g_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_all):
+            for j in range(self.nsets):
+                self.step(j)
+        for j in range(self.nsets):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.step(j)
+            self.g_one.append(g)
+        self.g_all.replay()
+        torch.cuda.synchronize()
+
+    def run_steps(self, k):
+        if not self.graphs:
+            for i in range(k):
+                self.step(i)
+            return
+        i = 0
+        while i + self.nsets <= k:
+            self.g_all.replay()
+            i += self.nsets
+        while i < k:
+            self.g_one[i % self.nsets].replay()
+            i += 1
+
+    def run_one(self, i):
+        if self.graphs:
+            self.g_one[i % self.nsets].replay()
+        else:
+            self.step(i)
+
+    def warm(self, warmup, soak_s):
+        import torch
+        for i in range(max(3, warmup)):
+            self.step(i)
+        torch.cuda.synchronize()
+        t_end = time.perf_counter() + soak_s
+        i = 0
+        while time.perf_counter() < t_end:   # untimed load so clocks settle
+            for _ in range(50):
+                self.step(i)
+                i += 1
+            torch.cuda.synchronize()
+        self.capture()
+
+    def timed_ms(self, steps, stream, ws):
+        """Device time (ms) of `steps` steps between CUDA events on the
+        launching stream, bracketed by a barrier and a synchronize."""
+        import torch
+        import torch.distributed as dist
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        self.run_steps(steps)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        return ev0.elapsed_time(ev1)
+
+    def output0(self):
+        """The output of input set 0 (the seeded inputs), on the host."""
+        import torch
+        self.step(0)
+        torch.cuda.synchronize()
+        return self.sets[0][3].cpu()
+
+    def close(self):
+        self.g_all = None
+        self.g_one = []
+        self.sets = []
+        self.op.close()
+
+
+def roofline(w, per_step_s, hbm, tflops, src, sms):
+    abytes = algorithmic_bytes(w)
+    achieved = abytes / per_step_s / 1e9
+    kdesc, launches = kernels_per_step(w, sms)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": captured_traffic(w), "peak_source": f"{src} hbm_gbs", "frac_of": src, "kernel": kdesc,
+            "algorithmic_bytes_per_step": abytes}
+    if w.F:
+        # the projected workload is reported against the tensor roofline (dense
+        # bf16, the burst figure: a step lasts tens of microseconds); its HBM
+        # fraction is kept alongside
+        af = algorithmic_flops(w)
+        hbm_part = {k: roof[k] for k in ("achieved", "peak", "unit", "frac")}
+        roof.update({"bound": "tensor", "achieved": af / per_step_s / 1e12, "peak": tflops, "unit": "TFLOP/s",
+                     "frac": af / per_step_s / 1e12 / tflops, "peak_source": f"{src} bf16_tflops",
+                     "algorithmic_flops_per_step": af, "hbm": hbm_part})
+    return roof, launches
+
+
+EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k")
+
+
 def main():
     args = parse()
-    from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, make_inputs
+    from linear_attention_diffusion_phi_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
@@ -309,108 +533,45 @@ def main():
             la_build.build()
         if ws > 1:
             dist.barrier()
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-
-    # input sets rotated step to step so that consecutive steps never find
-    # their inputs in L2 (total > 3x L2)
-    set_bytes = 4 * w.B * w.H * w.N * w.D * (2 if w.dtype == "bf16" else 4)
-    nsets = max(2, -(-3 * L2_BYTES // set_bytes))
-    sets = []
-    for i in range(nsets):
-        q, k, v, W = make_inputs(w, seed=input_seed(w, i, rank))
-        sets.append((q.to(dev), k.to(dev), v.to(dev), torch.empty_like(q, device=dev)))
-    Wd = None if W is None else W.to(dev)
-    op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, Wd)
     stream = torch.cuda.current_stream(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    hbm, tflops, src = peaks()
 
-    def step(i):
-        q, k, v, o = sets[i % nsets]
-        op(q, k, v, out=o)
-
+    tw = Timed(w, dev, rank, graphs=not args.no_graph)
     sampler = ClockSampler(local)
     sampler.start()
-    for i in range(max(3, args.warmup)):
-        step(i)
-    torch.cuda.synchronize()
-    t_end = time.perf_counter() + args.soak_s
-    i = 0
-    while time.perf_counter() < t_end:   # untimed load so clocks settle
-        for _ in range(200):
-            step(i)
-            i += 1
-        torch.cuda.synchronize()
-
-    # CUDA graphs remove host launch overhead: one graph runs one step over
-    # every input set in turn, single-step graphs cover a remainder.
-
-    if not args.no_graph:
-        g_all = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_all):
-            for j in range(nsets):
-                step(j)
-        g_one = []
-        for j in range(nsets):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step(j)
-            g_one.append(g)
-        g_all.replay()
-        torch.cuda.synchronize()
-
-    def run_steps(k):
-        if args.no_graph:
-            for i in range(k):
-                step(i)
-            return
-        i = 0
-        while i + nsets <= k:
-            g_all.replay()
-            i += nsets
-        while i < k:
-            g_one[i % nsets].replay()
-            i += 1
-
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    run_steps(args.steps)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    ms = ev0.elapsed_time(ev1)
+    tw.warm(args.warmup, args.soak_s)
+    ms = tw.timed_ms(args.steps, stream, ws)
     clocks = sampler.stop()
-    assert op.sync_status() == la.LA_OK, "device-side error during the timed region"
+    assert tw.op.sync_status() == la.LA_OK, "device-side error during the timed region"
 
     # distribution of single calls (this rank's), informational: the value
     # above is the mean over the bracketed steps
     try:
-        one = (lambda i: step(i)) if args.no_graph else (lambda i: g_one[i % nsets].replay())
-        per_call = percentiles_ms(per_call_ms(one, max(10, min(args.steps, 100)), stream))
+        per_call = percentiles_ms(per_call_ms(tw.run_one, max(10, min(args.steps, 100)), stream))
     except Exception as e:   # never let the extra figure cost the bench line
         per_call = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     # end to end through the host-buffer entry point: pinned host inputs,
     # H2D copies, forward, D2H copy of the result, every step
-    qh = [s[0].cpu().pin_memory() for s in sets[:2]]
-    kh = [s[1].cpu().pin_memory() for s in sets[:2]]
-    vh = [s[2].cpu().pin_memory() for s in sets[:2]]
+    qh = [s[0].cpu().pin_memory() for s in tw.sets[:2]]
+    kh = [s[1].cpu().pin_memory() for s in tw.sets[:2]]
+    vh = [s[2].cpu().pin_memory() for s in tw.sets[:2]]
     oh = [torch.empty_like(x).pin_memory() for x in qh]
-    dq, dk, dv, do = (torch.empty_like(sets[0][0]) for _ in range(4))
+    dq, dk, dv, do = (torch.empty_like(tw.sets[0][0]) for _ in range(4))
     e2e_steps = max(3, min(args.steps, 50))
     s_ptr = stream.cuda_stream
 
     def e2e_step(i):
         j = i % 2
-        st = la.la_forward_host(op.handle, qh[j].data_ptr(), kh[j].data_ptr(), vh[j].data_ptr(),
+        st = la.la_forward_host(tw.op.handle, qh[j].data_ptr(), kh[j].data_ptr(), vh[j].data_ptr(),
                                 oh[j].data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), do.data_ptr(),
                                 w.B, w.H, w.N, w.D, w.F, la.FEATURE_MAPS[w.fmap], w.eps, int(w.causal), s_ptr)
         la.check(st, "la_forward_host")
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:
         dist.barrier()
     ev0.record(stream)
@@ -419,8 +580,42 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ev0.elapsed_time(ev1)
+    del qh, kh, vh, oh, dq, dk, dv, do
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
+    got0 = tw.output0() if (rank == 0 and not args.no_parity) else None
+    tw.close()
+
+    # the other workloads, timed the same way after the headline (one GPU:
+    # their figures are reported beside it, the headline value is unchanged)
+    extras = []
+    if ws == 1 and not args.no_extra and w.name == "flux1024":
+        for name in EXTRA_WORKLOADS:
+            x = WORKLOADS[name]
+            try:
+                tx = Timed(x, dev, rank, graphs=not args.no_graph)
+                smp = ClockSampler(local)
+                smp.start()
+                tx.warm(args.warmup, 0.3)
+                xsteps = max(args.steps, 100)
+                xms = tx.timed_ms(xsteps, stream, ws)
+                xclk = smp.stop()
+                assert tx.op.sync_status() == la.LA_OK, "device-side error during the timed region"
+                xroof, xl = roofline(x, xms / 1e3 / xsteps, hbm, tflops, src, sms)
+                ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
+                       "causal": x.causal, "dtype": x.dtype, "steps": xsteps, "ms_per_step": xms / xsteps,
+                       "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
+                       "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
+                       "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
+                if not args.no_parity:
+                    ent["parity"] = parity_block(x, *tx.host, tx.output0())
+                tx.close()
+                del tx
+            except Exception as e:   # an extra figure never costs the headline line
+                ent = {"workload": name, "error": f"{type(e).__name__}: {e}"[:300]}
+            extras.append(ent)
+            torch.cuda.empty_cache()
+
     if ws > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -429,22 +624,7 @@ def main():
     tokens = w.tokens * ws
     per_step_s = ms / 1e3 / args.steps
     value = job_throughput(w.tokens, ws, args.steps, ms)
-    hbm, tflops, src = peaks()
-    abytes = algorithmic_bytes(w)
-    achieved = abytes / per_step_s / 1e9
-    kdesc, launches = kernels_per_step(w, torch.cuda.get_device_properties(dev).multi_processor_count)
-    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": captured_traffic(w), "peak_source": f"{src} hbm_gbs", "frac_of": src, "kernel": kdesc,
-            "algorithmic_bytes_per_step": abytes}
-    if w.F:
-        # the projected workload is reported against the tensor roofline (dense
-        # bf16, the burst figure: a step lasts tens of microseconds); its HBM
-        # fraction is kept alongside
-        af = algorithmic_flops(w)
-        hbm_part = {k: roof[k] for k in ("achieved", "peak", "unit", "frac")}
-        roof.update({"bound": "tensor", "achieved": af / per_step_s / 1e12, "peak": tflops, "unit": "TFLOP/s",
-                     "frac": af / per_step_s / 1e12 / tflops, "peak_source": f"{src} bf16_tflops",
-                     "algorithmic_flops_per_step": af, "hbm": hbm_part})
+    roof, launches = roofline(w, per_step_s, hbm, tflops, src, sms)
     elem = 2 if w.dtype == "bf16" else 4
     io = w.B * w.H * w.N * w.D * elem
     e2e = {"value": tokens / (e2e_ms / 1e3 / e2e_steps), "unit": UNIT, "h2d_bytes_per_step": 3 * io,
@@ -455,11 +635,17 @@ def main():
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "F": w.F,
                        "feature_map": w.fmap, "eps": w.eps, "causal": w.causal,
                        "global_batch": w.B * ws, "seq_len": w.N, "parallelism": f"replicas{ws}",
-                       "l2": f"{nsets} rotating input sets, {nsets * set_bytes / 2**20:.0f} MiB > 3x L2"},
-            "hbm_gbs": achieved, "roofline": roof, "clocks": clocks, "e2e": e2e, "per_call_ms": per_call,
-            "gpu_launches": None if launches is None else launches * args.steps, "launch": "cuda-graph" if not args.no_graph else "host"}
+                       "l2": f"{tw.nsets} rotating input sets, {tw.nsets * tw.set_bytes / 2**20:.0f} MiB > 3x L2"},
+            "hbm_gbs": roof["achieved"] if roof["bound"] == "hbm" else roof["hbm"]["achieved"],
+            "roofline": roof, "clocks": clocks, "e2e": e2e, "per_call_ms": per_call,
+            "gpu_launches": None if launches is None else launches * args.steps,
+            "launch": "cuda-graph" if not args.no_graph else "host"}
+    if got0 is not None:
+        line["parity"] = parity_block(w, *tw.host, got0)
+    if extras:
+        line["extra_configs"] = extras
     if not args.no_cpu_baseline and ws == 1:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, inputs=tw.host)
     print(json.dumps(line), flush=True)
     return 0
 

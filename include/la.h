@@ -39,9 +39,14 @@
  * out.  Ordinary launches are ordered as usual.
  *
  * Errors.  Argument errors are detected on the host before anything is
- * enqueued; out is then untouched.  Launch failures return LA_ERR_CUDA.
- * Errors detected on the device (a bounded wait that ran out) are recorded in a
- * status word inside the workspace and reported by la_sync_status().
+ * enqueued; out is then untouched.  A pointer that is not device memory of
+ * the current device is such an error (LA_ERR_INVALID_ARG).  Launch failures
+ * return LA_ERR_CUDA.  Errors detected on the device (a bounded wait that ran
+ * out) are recorded in a status word inside the workspace and reported by
+ * la_sync_status() only: la_forward enqueues and returns, and reading the
+ * word there would need a synchronisation with the stream, so it never looks
+ * at it.  The word of a newly bound workspace is cleared by the first
+ * la_forward (or la_sync_status) that uses it, on that call's stream.
  *
  * Threading.  A handle may be used by one host thread at a time.  Calls that
  * share a workspace must be ordered on the device (same stream, or events).
@@ -101,7 +106,9 @@ la_status_t la_set_projection(la_handle_t handle, const void* W, int H, int D, i
 size_t la_workspace_bytes(la_handle_t handle, int B, int H, int N, int D, int F, int causal);
 
 /* Bind a caller-owned device workspace (256-byte aligned).  The library writes
- * partial states and its status word there.  Bytes = 0 or ptr = NULL unbinds. */
+ * partial states and its status word there.  Bytes = 0 or ptr = NULL unbinds.
+ * Nothing is enqueued and nothing waits: the status word is cleared by the
+ * next la_forward or la_sync_status, on that call's stream. */
 la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
 
 /* Enqueue out = phi-attention(q, k, v) on `stream` (see the top of this file).
@@ -127,9 +134,11 @@ la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* 
                             void* dout, int B, int H, int N, int D, int F, int feature_map,
                             float eps, int causal, void* stream);
 
-/* Wait for `stream`, then read and clear the device status word of the bound
- * workspace.  Returns LA_OK, LA_ERR_TIMEOUT (a kernel abandoned a bounded
- * wait; its output is undefined) or LA_ERR_CUDA. */
+/* Read the device status word of the bound workspace after the work queued
+ * on `stream` (a copy on that stream, then a wait for the stream only), and
+ * clear it on the same stream if it was set.  Returns LA_OK, LA_ERR_TIMEOUT
+ * (a kernel abandoned a bounded wait; its output is undefined) or
+ * LA_ERR_CUDA. */
 la_status_t la_sync_status(la_handle_t handle, void* stream);
 
 /* Size of the static scratch array behind la_forward_noalloc (2 MiB).  A
@@ -149,10 +158,14 @@ la_status_t la_sync_status(la_handle_t handle, void* stream);
  * that needed more than the array would return LA_ERR_WORKSPACE before
  * anything is enqueued.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Every call on a device shares the one
- * array and it keeps the last call's contents: calls that overlap on the GPU
- * (different streams without ordering between them) race and give undefined
- * results.  Device-side timeouts of this entry point are not reported. */
+ * call before any stream capture.  The address is cached for the life of the
+ * process, so this entry point must not be used on a device after
+ * cudaDeviceReset.  Every call on a device shares the one array and it keeps
+ * the last call's contents: calls that overlap on the GPU (different streams
+ * without ordering between them) race and give undefined results.  The
+ * kernel only writes the array's status word (on a device-side timeout) and
+ * nothing reads it: timeouts of this entry point are not reported, and no
+ * clearing operation is enqueued between calls. */
 la_status_t la_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
                                int D, int feature_map, float eps, void* stream);
 

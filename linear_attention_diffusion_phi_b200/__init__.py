@@ -211,15 +211,20 @@ class LinearAttention:
             out = self.torch.empty_like(q)
         self._check_tensors(q, k, v, out)
         B, H, N, D = q.shape
-        self._bind_workspace(B, H, N, D, q.device)
-        s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
-        check(la_forward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                         B, H, N, D, self.F, self.fmap, self.eps, self.causal, s), "la_forward")
+        # the library launches on the current device and expects every
+        # pointer to belong to it: make the tensors' device current
+        with self.torch.cuda.device(q.device):
+            self._bind_workspace(B, H, N, D, q.device)
+            s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
+            check(la_forward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             B, H, N, D, self.F, self.fmap, self.eps, self.causal, s), "la_forward")
         return out
 
     def sync_status(self, stream=None):
-        s = stream if stream is not None else self.torch.cuda.current_stream().cuda_stream
-        return la_sync_status(self.handle, s)
+        dev = self._ws.device if self._ws is not None else self.torch.cuda.current_device()
+        with self.torch.cuda.device(dev):
+            s = stream if stream is not None else self.torch.cuda.current_stream(dev).cuda_stream
+            return la_sync_status(self.handle, s)
 
     def close(self):
         if self.handle:

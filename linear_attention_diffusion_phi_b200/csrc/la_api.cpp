@@ -20,6 +20,9 @@ struct la_handle_s {
   long long w_head_stride;
   void* ws;
   size_t ws_bytes;
+  // The status word of a newly bound workspace is cleared by the next call
+  // that uses it, on that call's stream (no device-wide synchronisation).
+  bool ws_clear_pending;
 };
 
 namespace {
@@ -190,6 +193,29 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 namespace la {
 
+// Whether `p` is device (or managed) memory of the current device.  A
+// pointer the runtime does not know (plain host memory) or one of another
+// device is refused before anything is launched: a kernel given it would
+// fault or read the wrong memory.
+bool on_current_device(const void* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (attr.type == cudaMemoryTypeManaged) return true;
+  return attr.type == cudaMemoryTypeDevice && attr.device == dev;
+}
+
+}  // namespace la
+
+namespace la {
+
 // Plan of the fused cluster kernel (la_forward_noalloc): the combine runs
 // through distributed shared memory, so the workspace is only the status word.
 void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p) {
@@ -302,14 +328,12 @@ la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
   }
   if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return LA_ERR_MISALIGNED;
   if (bytes < la::kHeaderBytes) return LA_ERR_WORKSPACE;
-  // Clear the status word once: later reads see only errors of calls made
-  // with this workspace.
-  if (cudaMemset(ptr, 0, la::kHeaderBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
-    cudaGetLastError();
-    return LA_ERR_CUDA;
-  }
+  // The status word is cleared by the next la_forward (or la_sync_status)
+  // on its own stream, so later reads see only errors of calls made with
+  // this workspace; nothing is enqueued here.
   h->ws = ptr;
   h->ws_bytes = bytes;
+  h->ws_clear_pending = true;
   return LA_OK;
 }
 
@@ -349,6 +373,17 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
   Plan p;
   make_plan(h, B, H, N, D, F, fmap, eps, causal, di.sms, &p);
   if (!h->ws || h->ws_bytes < p.bytes) return LA_ERR_WORKSPACE;
+  if (!la::on_current_device(q) || !la::on_current_device(k) || !la::on_current_device(v) ||
+      !la::on_current_device(out) || !la::on_current_device(h->ws) || (F > 0 && !la::on_current_device(h->W)))
+    return LA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (h->ws_clear_pending) {
+    if (cudaMemsetAsync(h->ws, 0, la::kHeaderBytes, cs) != cudaSuccess) {
+      cudaGetLastError();
+      return LA_ERR_CUDA;
+    }
+    h->ws_clear_pending = false;
+  }
 
   la::LaunchArgs a = {};
   a.p = &p;
@@ -356,7 +391,7 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
   a.W = F ? h->W : nullptr;
   a.w_head_stride = h->w_head_stride;
   a.ws = static_cast<char*>(h->ws);
-  a.stream = static_cast<cudaStream_t>(stream);
+  a.stream = cs;
 
   cudaError_t err;
   if (h->dtype == LA_F32) {
@@ -400,6 +435,8 @@ la_status_t la_forward_host(la_handle_t h, const void* q_host, const void* k_hos
   for (int i = 0; i < 4; ++i)
     for (int j = i + 1; j < 4; ++j)
       if (la::overlap(dev[i], n, dev[j], n)) return LA_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (!la::on_current_device(dev[i])) return LA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
@@ -420,15 +457,24 @@ la_status_t la_sync_status(la_handle_t h, void* stream) {
   if (!h) return LA_ERR_INVALID_ARG;
   if (!h->ws) return LA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (h->ws_clear_pending) {   // no call has used this workspace yet
+    if (cudaMemsetAsync(h->ws, 0, la::kHeaderBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return LA_ERR_CUDA;
+    }
+    h->ws_clear_pending = false;
+    return LA_OK;
+  }
   int word = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess ||
-      cudaMemcpy(&word, h->ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+  if (cudaMemcpyAsync(&word, h->ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }
   if (word == 0) return LA_OK;
-  // An abandoned wait can leave barrier counts mid-way: clear the header.
-  if (cudaMemset(h->ws, 0, la::kHeaderBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+  // An abandoned wait can leave barrier counts mid-way: clear the header,
+  // ordered on the same stream.
+  if (cudaMemsetAsync(h->ws, 0, la::kHeaderBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }

@@ -63,6 +63,8 @@ bool encode_tile_map_bf16(CUtensorMap* m, const void* base, long long outer, lon
                           long long outer_stride_elems);
 // SM count of the current device; false unless it is an sm_100 device.
 bool current_sm100(int* num_sms);
+// `p` is device (or managed) memory of the current device.
+bool on_current_device(const void* p);
 // The byte ranges [a, a + an) and [b, b + bn) share at least one byte.
 bool overlap(const void* a, size_t an, const void* b, size_t bn);
 

@@ -19,14 +19,17 @@ namespace {
 
 constexpr size_t kScratchBytes = LA_NOALLOC_SCRATCH_BYTES;
 
-// Scratch for la_forward_noalloc: the status word of its kernel.  In host code this name is only a handle for
+// Scratch for la_forward_noalloc: the status word of its kernel (written on a
+// device-side timeout, read by nobody).  In host code this name is only a handle for
 // cudaGetSymbolAddress, never a device address.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 
 // Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached for the life of the
+// process: after a cudaDeviceReset the cached address would be stale, so
+// this entry point must not be used across a reset.
 bool scratch_address(void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
@@ -69,6 +72,9 @@ extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const vo
 
   int sms = 0;
   if (!la::current_sm100(&sms)) return LA_ERR_NO_DEVICE;
+  if (!la::on_current_device(q) || !la::on_current_device(k) || !la::on_current_device(v) ||
+      !la::on_current_device(out))
+    return LA_ERR_INVALID_ARG;
   la::Plan p;
   la::plan_bf16_noncausal(B, H, N, D, feature_map, eps, sms, &p);
   if (p.bytes > kScratchBytes) return LA_ERR_WORKSPACE;   // problem too large for the static scratch
@@ -76,13 +82,10 @@ extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const vo
   void* scratch = nullptr;
   if (!scratch_address(&scratch)) return LA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents; the status word must start
-  // at zero (the kernel reads nothing else from it).
-  if (cudaMemsetAsync(static_cast<char*>(scratch), 0, p.off_status + la::kStatusBytes, s) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return LA_ERR_CUDA;
-  }
+  // The array keeps the previous call's contents.  Nothing in it has to
+  // start at zero: the kernel only ever writes the status word (first error
+  // wins) and never reads it, and this entry point does not report it, so no
+  // clearing operation is put between consecutive forwards on the stream.
 
   CUtensorMap tq, tk, tv, to;
   const long long BH = p.BH, hs = static_cast<long long>(N) * D;

@@ -56,8 +56,13 @@ def errors(got, ref):
     }
 
 
-def assert_parity(got, ref, dtype):
+def assert_parity(got, ref, dtype, label=None):
     e = errors(got, ref)
+    if label is not None:
+        import conftest
+        bar = {"rel_inf": F32_REL} if dtype == "f32" else {"max_abs": BF16_MAX, "mean_abs": BF16_MEAN,
+                                                          "rel_l2": BF16_RL2}
+        conftest.PARITY_RECORDS.append((label, e, bar))
     assert np.all(np.isfinite(as_float64(got) if not isinstance(got, np.ndarray) else got))
     if dtype == "f32":
         assert e["rel_inf"] <= F32_REL, e
@@ -70,10 +75,10 @@ def oracle_full(w, q, k, v, W):
     return ora.forward(as_float64(q), as_float64(k), as_float64(v), w.fmap, w.eps, w.causal, as_float64(W))
 
 
-def check_workload(w, seed=None):
+def check_workload(w, seed=None, label=None):
     q, k, v, W = make_inputs(w, seed)
     got = run_gpu(w, q, k, v, W)
-    return assert_parity(got, oracle_full(w, q, k, v, W), w.dtype)
+    return assert_parity(got, oracle_full(w, q, k, v, W), w.dtype, label)
 
 
 # ------------------------------------------------------------------ fp32 path
@@ -85,7 +90,7 @@ def test_tiny_f32_against_definition():
     q, k, v, _ = make_inputs(w)
     got = run_gpu(w, q, k, v)
     ref = ora.brute_force(as_float64(q), as_float64(k), as_float64(v), w.fmap, w.eps, False)
-    assert_parity(got, ref, "f32")
+    assert_parity(got, ref, "f32", "tiny_f32 (all elements)")
 
 
 F32_CASES = [
@@ -136,12 +141,12 @@ def test_bf16_noncausal_shapes(case):
 def test_flux1024_full():
     """Flux-1024 shape (B=1, H=24, N=4608, D=128, elu+1, unit-norm x sqrt(D)
     queries and keys), every output element against the oracle."""
-    check_workload(WORKLOADS["flux1024"])
+    check_workload(WORKLOADS["flux1024"], label="flux1024 (all elements)")
 
 
 def test_flux2048_cfg_full():
     """Flux-2048 CFG pair (B=2, H=24, N=16896, D=128, relu), every element."""
-    check_workload(WORKLOADS["flux2048_cfg"])
+    check_workload(WORKLOADS["flux2048_cfg"], label="flux2048_cfg (all elements)")
 
 
 def test_bf16_deterministic_and_guard_bands():
@@ -210,7 +215,7 @@ def test_bf16_projected_shapes(case):
 def test_proj256_full():
     """The projected-feature workload (B=1, H=24, N=4608, D=128, F=256,
     elu(xW)+1), every output element."""
-    check_workload(WORKLOADS["proj256"])
+    check_workload(WORKLOADS["proj256"], label="proj256 (all elements)")
 
 
 def test_bf16_projected_shared_matrix():
@@ -261,11 +266,16 @@ def test_causal32k_sampled_rows():
     assert torch_isfinite(got)
     qf, kf, vf = as_float64(q), as_float64(k), as_float64(v)
     slices = [range(0, 512), range(8192 - 256, 8192 + 256), range(w.N - 512, w.N)]
+    rows_g, rows_r = [], []
     for b, h in ((0, 0), (3, 7)):
         for sl in slices:
             idx = list(sl)
             ref = ora.rows(qf, kf, vf, b, h, idx, w.fmap, w.eps, True)
             assert_parity(as_float64(got[b, h])[idx], ref, "bf16")
+            rows_g.append(as_float64(got[b, h])[idx])
+            rows_r.append(ref)
+    # all sampled rows together, for the record
+    assert_parity(np.concatenate(rows_g), np.concatenate(rows_r), "bf16", "causal32k (6 x 512 sampled rows)")
     rng = np.random.default_rng(7)
     for b, h in ((1, 5), (2, 2)):
         idx = sorted(set(rng.integers(0, w.N, 96).tolist()) | {127, 128, 16383, 16384, 24575, 24576})
@@ -445,3 +455,33 @@ def test_overlapping_output_is_refused_before_launch():
     assert torch.equal(op(qd, kd, vd), ref)
     op.close()
     op2.close()
+
+
+def test_pointer_not_on_current_device_is_refused():
+    """A host pointer (pinned or not) where a device buffer belongs is refused
+    on the host with LA_ERR_INVALID_ARG before anything is enqueued, by
+    la_forward, la_forward_host and la_forward_noalloc alike."""
+    import torch
+    w = Workload("hostptr", B=1, H=2, N=300, D=128, seed=14)
+    q, k, v, _ = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, "elu", w.eps)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    ref = op(qd, kd, vd).clone()
+    out = torch.zeros_like(qd)
+    s = torch.cuda.current_stream().cuda_stream
+    args = (1, 2, 300, 128, 0, la.LA_PHI_ELU1, w.eps, 0, s)
+    qp = q.pin_memory()
+    for host in (qp.data_ptr(), q.data_ptr()):
+        assert la.la_forward(op.handle, host, kd.data_ptr(), vd.data_ptr(), out.data_ptr(), *args) == \
+            la.LA_ERR_INVALID_ARG
+        assert la.la_forward_noalloc(host, kd.data_ptr(), vd.data_ptr(), out.data_ptr(), 1, 2, 300, 128,
+                                     la.LA_PHI_ELU1, w.eps, s) == la.LA_ERR_INVALID_ARG
+    oh = torch.empty_like(qp).pin_memory()
+    assert la.la_forward_host(op.handle, qp.data_ptr(), qp.data_ptr(), qp.data_ptr(), oh.data_ptr(),
+                              qp.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), *args) == \
+        la.LA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    assert torch.equal(op(qd, kd, vd), ref)
+    op.close()
