@@ -8,7 +8,8 @@
 // One kernel.  Each head is served by a thread-block cluster of S CTAs (one
 // per SM); CTA r owns the r-th run of 128-token tiles of the head.
 //   phase 1  TMA streams the CTA's K and V tiles into a ring of shared-memory
-//            slots; eight warps apply phi to K in place; one thread issues
+//            slots; eight warps apply phi to K in place (V tiles need no work
+//            and go straight to the tensor core); one thread issues
 //            tcgen05.mma  kv^T += V^T phi(K)  and  ksum^T += 1^T phi(K)  into
 //            tensor memory (fp32).
 //   combine  four warps copy the CTA's partial (kv | ksum)^T from tensor
@@ -67,10 +68,19 @@ struct Cfg {
   static constexpr int kChunksPerRow = D / 8;                      // 16-byte chunks per token row
   static constexpr int kThreadsPerChunk = kPhiThreads / kChunksPerRow;
   static constexpr int kRowsPerThread = 128 / kThreadsPerChunk;
-  static constexpr int kCombWarp0 = 2 + kPhiWarps;                 // 4 warps: partial, combine
-  static constexpr int kEpiWarp0 = kCombWarp0 + 4;                 // 4 warps: outputs
-  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+  static constexpr int kCombWarp0 = 2 + kPhiWarps;                 // 8 warps: combine, then outputs
+  static constexpr int kThreads = 32 * (kCombWarp0 + 8);
 };
+
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 template <int D, int FMAP>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
@@ -79,7 +89,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                  int* status, int N, int tiles, float eps) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[C::kRing1], ready[C::kRing1], empty[C::kRing1];
+  // full / ready: arrival of a K or Q tile / phi done on it (the phi warps
+  // wait on every phase of full[] in order); vfull: arrival of a V tile
+  // (waited on by the MMA issuer only); empty: every use of a slot.
+  __shared__ __align__(8) uint64_t full[C::kRing1], ready[C::kRing1], vfull[C::kRing1], empty[C::kRing1];
   // Tensor-memory accumulators a = 0, 1: phase 1 uses accumulator 0 once
   // (p1full / p1empty, consumed by the combine warps); phase-2 tile u uses
   // accumulator u & 1 (accfull / accempty, consumed by the output warps).
@@ -114,18 +127,26 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   auto ring2 = [&](int j) { return j < C::kSlots ? j : C::kSlots + 1; };
   auto q_slot = [&](int u) { return ring2(u % C::kRing2); };
   auto q_round = [&](int u) { return uses1(ring2(u % C::kRing2)) + u / C::kRing2; };
+  // Phases of full[] / ready[] before Q tile u: the phase-1 K uses of its
+  // slot (K tiles land in even slots, V tiles in odd ones) and the earlier Q
+  // uses.
+  auto q_kround = [&](int u) {
+    const int s = ring2(u % C::kRing2);
+    return ((s & 1) == 0 ? uses1(s) : 0) + u / C::kRing2;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kRing1; ++i) {
       mbar_init(&full[i], 1);
+      mbar_init(&vfull[i], 1);
       mbar_init(&ready[i], C::kPhiWarps);
       mbar_init(&empty[i], 1);
     }
     mbar_init(&p1full, 1);
-    mbar_init(&p1empty, 4);
+    mbar_init(&p1empty, 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
+      mbar_init(&accempty[i], 8);
     }
     mbar_init(&stage_ready, S);
     mbar_init(&blob_ready, S);
@@ -179,13 +200,15 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         if (!mbar_wait_cluster(&blob_ready, 0, status)) return;
         staging_free = true;
       }
-      const CUtensorMap* m = p1 ? ((seq & 1) ? &tm_v : &tm_k) : &tm_q;
+      const bool is_v = p1 && (seq & 1);
+      const CUtensorMap* m = p1 ? (is_v ? &tm_v : &tm_k) : &tm_q;
       const int tile = p1 ? seq / 2 : seq - 2 * T;
+      uint64_t* bar = is_v ? &vfull[s] : &full[s];
       uint8_t* dst = slot_ptr(s);
-      mbar_arrive_expect_tx(&full[s], C::kSlotBytes);
+      mbar_arrive_expect_tx(bar, C::kSlotBytes);
 #pragma unroll
       for (int b = 0; b < C::kBoxes; ++b)
-        tma_load_3d(dst + b * kBoxBytes, m, &full[s], 64 * b, (tile0 + tile) * kTileTokens, bh);
+        tma_load_3d(dst + b * kBoxBytes, m, bar, 64 * b, (tile0 + tile) * kTileTokens, bh);
       ++seq;
     }
   };
@@ -214,8 +237,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       for (int t = 0; t < T; ++t) {
         const int qk = 2 * t, qv = 2 * t + 1;
         const int sk = qk % C::kRing1, sv = qv % C::kRing1;
+        // phi(K) done; V as it arrived
         if (!mbar_wait(&ready[sk], (qk / C::kRing1) & 1, status) ||
-            !mbar_wait(&ready[sv], (qv / C::kRing1) & 1, status)) {
+            !mbar_wait(&vfull[sv], (qv / C::kRing1) & 1, status)) {
           ok = false;
           break;
         }
@@ -249,7 +273,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         for (int u = 0; u < T; ++u) {
           const int s = q_slot(u);
           const int a = u & 1, ar = u >> 1;
-          bool got = mbar_wait(&ready[s], q_round(u) & 1, status);
+          bool got = mbar_wait(&ready[s], q_kround(u) & 1, status);
           if (got && ar == 0 && a == 0) got = mbar_wait(&p1empty, 0, status);   // freed by the combine warps
           if (got && ar > 0) got = mbar_wait(&accempty[a], (ar - 1) & 1, status);
           if (!got) break;
@@ -269,105 +293,105 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       }
     }
   } else if (warp < C::kCombWarp0) {
-    // ------------------------------------- phi on K and Q; V passes through
-    // Every slot use, whatever it holds, completes one phase of full[] and one
-    // of ready[], so the phase parity of both follows the slot's round.
+    // ----------------- phi on the K tiles, then on the Q tiles, in place
+    // Every K or Q use of a slot completes one phase of full[] and one of
+    // ready[]; V tiles are not touched here.
     const int pt = threadIdx.x - 64;
     const int cc = pt / C::kThreadsPerChunk;
     const int r0 = pt % C::kThreadsPerChunk;
-    for (int seq = 0; seq < 3 * T; ++seq) {
-      const bool in_kv = seq < 2 * T;
-      const bool is_v = in_kv && (seq & 1);
-      const int s = in_kv ? seq % C::kRing1 : q_slot(seq - 2 * T);
-      const int round = in_kv ? seq / C::kRing1 : q_round(seq - 2 * T);
+    for (int v = 0; v < 2 * T; ++v) {
+      const bool is_k = v < T;
+      const int u = v - T;
+      const int s = is_k ? (2 * v) % C::kRing1 : q_slot(u);
+      const int round = is_k ? (2 * v) / C::kRing1 : q_kround(u);
       if (!warp_wait(&full[s], round & 1, status)) break;
-      if (!is_v) {
-        uint8_t* tile = slot_ptr(s);
-        // key rows past the sequence end must not reach ksum
-        const int valid = in_kv ? min(kTileTokens, N - (tile0 + seq / 2) * kTileTokens) : kTileTokens;
-        phi_rows<FMAP, C::kRowsPerThread, C::kThreadsPerChunk>(tile, cc, r0, valid);
-        fence_proxy_async_smem();
-      }
+      // key rows past the sequence end must not reach kv or ksum
+      const int valid = is_k ? min(kTileTokens, N - (tile0 + v) * kTileTokens) : kTileTokens;
+      phi_rows<FMAP, C::kRowsPerThread, C::kThreadsPerChunk>(slot_ptr(s), cc, r0, valid);
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ready[s]);
     }
   } else {
-    // ------------------------------------------- combine and output warps
-    // Warps kCombWarp0.. (4) copy the partial to shared memory; then they and
-    // the four output warps sum the cluster's partials; then the output warps
-    // write the phase-2 results.
+    // --------------------------------------- combine, then the outputs
+    // Eight warps, two per tensor-memory lane quarter, each taking one half
+    // of the columns: (1) copy the partial (kv | ksum)^T into the CTA's own
+    // shared memory; (2) sum their share of the cluster's partials; (3) write
+    // the phase-2 outputs.
     const int ct = threadIdx.x - 32 * C::kCombWarp0;   // 0..255
-    const bool comb = warp < C::kEpiWarp0;
+    const int half = ct >> 7;
     const bool leader = ct == 0;
     const int q = warp & 3;                             // TMEM lane quarter
-    if (comb) {
-      // (1) partial (kv | ksum)^T -> own shared memory, bf16, image layout
-      bool ok = true;
-      if (leader && !mbar_wait(&p1full, 0, status)) comb_flag = 1;
-      named_bar_sync(1, 128);
-      if (comb_flag) ok = false;
-      if (ok) {
-        tc_fence_after();
-        auto put_row = [&](int n, const float* v, int c0) {   // 32 values of row n from column c0
+    const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
+    bool got = true;
+    auto sync_ok = [&](bool mine) {   // every warp takes the leader's verdict
+      if (leader && !mine) comb_flag = 1;
+      named_bar_sync(3, 256);
+      return comb_flag == 0;
+    };
+    if (leader) got = mbar_wait(&p1full, 0, status);
+    bool ok = sync_ok(got);
+    if (ok) {
+      // (1) partial -> own shared memory, bf16, image layout
+      tc_fence_after();
+      auto put_row = [&](int n, const float* v, int c0) {   // 32 values of row n from column c0
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t w[4];
+        for (int j = 0; j < 4; ++j) {
+          const int c = c0 / 8 + j;
+          *reinterpret_cast<uint4*>(stage + (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4)) =
+              pack8(v + 8 * j);
+        }
+      };
+      constexpr int kHalfCols = D / 2;
+      // kv^T: M = 128 -> row = lane; M = 64 -> rows 16q..16q+15 in lanes 32q..32q+15
+      const bool valid = (D == 128) || lane < 16;
+      const int n = (D == 128) ? 32 * q + lane : 16 * q + lane;
+      {
+        float v[kHalfCols];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-              w[e] = *reinterpret_cast<uint32_t*>(&b);
-            }
-            const int c = c0 / 8 + j;
-            *reinterpret_cast<uint4*>(stage + (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        };
-        const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
-        // kv^T: M = 128 -> row = lane; M = 64 -> rows 16q..16q+15 in lanes 32q..32q+15
-        const bool valid = (D == 128) || lane < 16;
-        const int n = (D == 128) ? 32 * q + lane : 16 * q + lane;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + tq + c0, v);
-          tmem_wait_ld();
-          if (valid) put_row(n, v, c0);
-        }
-        // ksum^T is row 0 of the M = 64 product: lane 0 of quarter 0
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + tq + D + c0, v);
-          tmem_wait_ld();
-          if (q == 0 && lane == 0) put_row(D, v, c0);
-        }
-        if (C::kExtra) {   // the image region held K/V tiles: restore its zero padding rows
-          for (int i = ct; i < (D / 64) * (C::kNB - D - 1) * 8; i += 128) {
-            const int a = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
-            *reinterpret_cast<uint4*>(blob + a * C::kBlobAtomBytes + (D + 1 + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p1empty);
-        // The CTA barrier orders every thread's staging stores before the
-        // leader's release-arrive at cluster scope (release is cumulative).
-        named_bar_sync(1, 128);
-        if (leader) {
-          for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stage_ready), p));
-          if (!mbar_wait_cluster(&stage_ready, 0, status)) comb_flag = 1;
-        }
+        for (int c0 = 0; c0 < kHalfCols; c0 += 32) tmem_ld32(tmem + tq + half * kHalfCols + c0, *reinterpret_cast<float(*)[32]>(v + c0));
+        tmem_wait_ld();
+        if (valid)
+#pragma unroll
+          for (int c0 = 0; c0 < kHalfCols; c0 += 32) put_row(n, v + c0, half * kHalfCols + c0);
       }
+      // ksum^T is row 0 of the M = 64 product: lane 0 of quarter 0
+      if (q == 0) {
+        float v[kHalfCols];
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfCols; c0 += 32) tmem_ld32(tmem + D + half * kHalfCols + c0, *reinterpret_cast<float(*)[32]>(v + c0));
+        tmem_wait_ld();
+        if (lane == 0)
+#pragma unroll
+          for (int c0 = 0; c0 < kHalfCols; c0 += 32) put_row(D, v + c0, half * kHalfCols + c0);
+      }
+      if (C::kExtra) {   // the image region held K/V tiles: restore its zero padding rows
+        for (int i = ct; i < (D / 64) * (C::kNB - D - 1) * 8; i += 256) {
+          const int at = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
+          *reinterpret_cast<uint4*>(blob + at * C::kBlobAtomBytes + (D + 1 + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p1empty);
+      // The CTA barrier orders every thread's staging stores before the
+      // leader's release-arrive at cluster scope (release is cumulative).
+      named_bar_sync(3, 256);
+      if (leader) {
+        for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stage_ready), p));
+        got = mbar_wait_cluster(&stage_ready, 0, status);
+      }
+      ok = sync_ok(got);
     }
-    // (2) chunks [i0, i1) of rows 0..D of the image: the sum over the
-    // cluster's staged partials, in ascending CTA order, stored into every
-    // CTA's image.  Two chunks per thread and pass, all loads in flight.
-    named_bar_sync(3, 256);
-    const bool ok2 = comb_flag == 0;
-    if (ok2) {
+    if (ok) {
+      // (2) chunks [i0, i1) of rows 0..D of the image: the sum over the
+      // cluster's staged partials, in ascending CTA order, stored into every
+      // CTA's image.  Two chunks per thread and pass; the loads of every
+      // peer are in flight together.
       constexpr int kChunks = (D + 1) * (D / 8);
+      constexpr int kMaxS = 8;
       const int i0 = rank * kChunks / S, i1 = (rank + 1) * kChunks / S;
       const uint32_t stage_base = smem_u32(stage), blob_base = smem_u32(blob);
       for (int i = i0 + ct; i < i1; i += 2 * 256) {
@@ -377,91 +401,74 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         for (int h = 0; h < 2; ++h) {
           const int ii = i + h * 256;
           has[h] = ii < i1;
-          const int n = ii / (D / 8), c = ii % (D / 8);
-          off[h] = (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4);
+          const int nn = ii / (D / 8), c = ii % (D / 8);
+          off[h] = (c >> 3) * C::kBlobAtomBytes + nn * 128 + (((c & 7) ^ (nn & 7)) << 4);
         }
-        float acc[2][8];
+        uint32_t w[2][kMaxS][4];
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-        for (int p0 = 0; p0 < S; p0 += 4) {
-          uint32_t w[2][4][4];
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (has[h] && p0 + j < S) ld_cluster_v4(mapa_shared(stage_base + off[h], p0 + j), w[h][j]);
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (has[h] && p0 + j < S) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[h][j][e]));
-                  acc[h][2 * e] += x.x;
-                  acc[h][2 * e + 1] += x.y;
-                }
-              }
-            }
-        }
+          for (int p = 0; p < kMaxS; ++p)
+            if (has[h] && p < S) ld_cluster_v4(mapa_shared(stage_base + off[h], p), w[h][p]);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (!has[h]) continue;
-          uint32_t o[4];
+          float acc[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 b = __floats2bfloat162_rn(acc[h][2 * e], acc[h][2 * e + 1]);
-            o[e] = *reinterpret_cast<uint32_t*>(&b);
+          for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+          for (int p = 0; p < kMaxS; ++p) {
+            if (p < S) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[h][p][e]));
+                acc[2 * e] += x.x;
+                acc[2 * e + 1] += x.y;
+              }
+            }
           }
-          const uint4 val = make_uint4(o[0], o[1], o[2], o[3]);
+          const uint4 val = pack8(acc);
           for (int p = 0; p < S; ++p) st_cluster_v4(mapa_shared(blob_base + off[h], p), val);
         }
       }
+      named_bar_sync(3, 256);
+      if (leader)
+        for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&blob_ready), p));
     }
-    named_bar_sync(3, 256);
-    if (leader && ok2)
-      for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&blob_ready), p));
-    if (!comb) {
-      // (3) outputs of the CTA's Q tiles
-      const bool eleader = threadIdx.x == 32 * C::kEpiWarp0;
+    if (ok) {
+      // (3) outputs of the CTA's Q tiles: each warp its rows' half of the
+      // value columns
+      constexpr int kHalfCols = D / 2;
       int prev_slot = -1;
       for (int u = 0; u < T; ++u) {
         const int s = q_slot(u);
         const int a = u & 1, ar = u >> 1;
-        if (eleader && !mbar_wait(&accfull[a], ar & 1, status)) ep_flag = 1;
-        named_bar_sync(2, 128);
+        got = true;
+        if (leader) got = mbar_wait(&accfull[a], ar & 1, status);
+        if (leader && !got) ep_flag = 1;
+        named_bar_sync(2, 256);
         if (ep_flag) break;
         tc_fence_after();
-        const uint32_t trow = tmem + a * C::kAccStride + (static_cast<uint32_t>(32 * q) << 16);
+        const uint32_t trow = tmem + a * C::kAccStride + tq;
         const int r = 32 * q + lane;   // token row within the tile
+        float v[kHalfCols];
         const float den = tmem_ld1(trow + D);
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfCols; c0 += 32) tmem_ld32(trow + half * kHalfCols + c0, *reinterpret_cast<float(*)[32]>(v + c0));
         tmem_wait_ld();
-        const float inv = 1.0f / (den + eps);
-        uint8_t* ob = slot_ptr(s);   // the MMA is done with this Q tile
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(trow + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * jj + 2 * e] * inv, v[8 * jj + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&b);
-            }
-            *reinterpret_cast<uint4*>(ob + swz_off(r, c0 / 8 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&accempty[a]);
+        if (lane == 0) mbar_arrive(&accempty[a]);   // the accumulator is free for tile u + 2
+        const float inv = 1.0f / (den + eps);
+#pragma unroll
+        for (int e = 0; e < kHalfCols; ++e) v[e] *= inv;
+        uint8_t* ob = slot_ptr(s);   // the MMA is done with this Q tile
+#pragma unroll
+        for (int jj = 0; jj < kHalfCols / 8; ++jj)
+          *reinterpret_cast<uint4*>(ob + swz_off(r, half * (kHalfCols / 8) + jj)) = pack8(v + 8 * jj);
         fence_proxy_async_smem();
-        named_bar_sync(2, 128);
-        if (eleader) {
+        named_bar_sync(2, 256);
+        if (leader) {
 #pragma unroll
           for (int b = 0; b < C::kBoxes; ++b)
             tma_store_3d(&tm_out, ob + b * kBoxBytes, 64 * b, (tile0 + u) * kTileTokens, bh);
@@ -473,7 +480,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         }
         prev_slot = s;
       }
-      if (eleader) bulk_wait_group<0>();
+      if (leader) bulk_wait_group<0>();
     }
   }
   tc_fence_before();
@@ -482,46 +489,50 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   cluster_sync_all();   // no CTA leaves while the cluster may still address its shared memory
 }
 
-// Largest cluster size S <= min(8, tiles) for which B*H clusters fit on the
-// device at once (one wave), per device and kernel; 1 when none does.
-template <typename K>
-int pick_cluster(K kern, uint32_t smem, int threads, long long BH, int tiles) {
+// Largest cluster size S <= min(8, tiles) for which B*H clusters of `kern`
+// fit on the device at once (one wave), per device and kernel; 1 when none
+// does.
+int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int tiles) {
   static std::mutex mu;
-  static int cache[64][9];
-  static bool have[64][9] = {};
+  static const void* key[16];
+  static int cache[64][16][9];
+  static bool have[64][16][9] = {};
+  static int nkeys = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return 1;
   }
+  std::lock_guard<std::mutex> lock(mu);
+  int k = 0;
+  while (k < nkeys && key[k] != kern) ++k;
+  if (k == nkeys) {
+    if (nkeys == 16) return 1;
+    key[nkeys++] = kern;
+  }
   const int smax = tiles < 8 ? tiles : 8;
   for (int s = smax; s >= 2; --s) {
-    int n;
-    {
-      std::lock_guard<std::mutex> lock(mu);
-      if (!have[dev][s]) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(s), 1);
-        cfg.blockDim = dim3(threads);
-        cfg.dynamicSmemBytes = smem;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(s);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int m = 0;
-        if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
-          cudaGetLastError();
-          m = 0;
-        }
-        cache[dev][s] = m;
-        have[dev][s] = true;
+    if (!have[dev][k][s]) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(s), 1);
+      cfg.blockDim = dim3(threads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int m = 0;
+      if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        m = 0;
       }
-      n = cache[dev][s];
+      cache[dev][k][s] = m;
+      have[dev][k][s] = true;
     }
-    if (n >= BH) return s;
+    if (cache[dev][k][s] >= BH) return s;
   }
   return 1;
 }
@@ -533,7 +544,7 @@ cudaError_t run(const LaunchArgs& a) {
   auto kern = fused_kernel<D, FMAP>;
   cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
-  const int S = pick_cluster(kern, C::kSmemBytes, C::kThreads, p.BH, p.tiles);
+  const int S = pick_cluster(reinterpret_cast<const void*>(kern), C::kSmemBytes, C::kThreads, p.BH, p.tiles);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(S);

@@ -83,6 +83,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // phase completes or the hint runs out), records LA_ERR_TIMEOUT and returns
 // false; the caller then winds down.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_test(bar, parity)) return true;   // already complete: no suspend/resume round trip
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
