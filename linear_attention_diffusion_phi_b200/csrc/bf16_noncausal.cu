@@ -12,14 +12,14 @@
 //            and go straight to the tensor core); one thread issues
 //            tcgen05.mma  kv^T += V^T phi(K)  and  ksum^T += 1^T phi(K)  into
 //            tensor memory (fp32).
-//   combine  four warps copy the CTA's partial (kv | ksum)^T from tensor
-//            memory into its own shared memory, rounded to bf16 and already in
-//            the layout of the apply MMA's B operand; after a cluster
-//            handshake eight warps of every CTA sum their share of that image
-//            over the cluster's CTAs in ascending order (no atomics, so bitwise
-//            reproducible), reading the peers' shared memory, and store the
-//            sums into the shared memory of every CTA of the cluster
-//            (distributed shared memory, no global round trip).
+//   combine  eight warps read the CTA's partial (kv | ksum)^T from tensor
+//            memory, round it to bf16 and send each 16-byte chunk to the
+//            cluster CTA that owns it (asynchronous distributed-shared-memory
+//            stores whose bytes complete on the owner's barrier; no global
+//            round trip).  Every CTA sums the partials of the chunks it owns
+//            in ascending CTA order (no atomics, so bitwise reproducible) and
+//            sends the sums into the image of every CTA of the cluster: the
+//            apply MMA's B operand, in its layout.
 //   phase 2  the CTA's Q tiles (prefetched during the combine) get phi in
 //            place, one MMA per tile computes [num | den] = phi(Q) [kv | ksum],
 //            and four warps write out = num / (den + eps) as bf16 into the Q
@@ -49,18 +49,21 @@ struct Cfg {
   // each row's D features are split in 64-feature k-atoms of kNB rows.
   static constexpr uint32_t kBlobAtomBytes = kNB * 128;
   static constexpr uint32_t kBlobBytes = (D / 64) * kBlobAtomBytes;
-  // This CTA's partial (kv | ksum)^T in bf16, same layout as the image (rows
-  // 0..D), read by the cluster's CTAs.
-  static constexpr uint32_t kStageBytes = kBlobBytes;
+  // 16-byte chunks of image rows 0..D, the unit of the cluster combine.
+  static constexpr int kChunks = (D + 1) * (D / 8);
+  // Receive buffer of the combine: S slices of at most ceil(kChunks / S)
+  // chunks, one per sending CTA; S * ceil(kChunks / S) <= kChunks + 7.
+  static constexpr uint32_t kRecvBytes = kBlobBytes;
+  static_assert((kChunks + 7) * 16 <= kRecvBytes, "receive buffer too small");
   static constexpr uint32_t kOnesBytes = 2048;                     // A of the ksum MMA (64 x 16)
   static constexpr int kSlots = D == 128 ? 4 : 8;                 // ring of tile slots
-  // During phase 1 the image and staging regions are idle; where a tile fits
+  // During phase 1 the image and receive regions are idle; where a tile fits
   // in them they serve as two more K/V slots.
   static constexpr int kExtra = (kBlobBytes >= kSlotBytes) ? 2 : 0;
   static constexpr int kRing1 = kSlots + kExtra;                   // phase-1 ring (K, V tiles)
-  // Phase 2 adds the staging region once the cluster has read it.
+  // Phase 2 adds the receive region once this CTA has summed its chunks.
   static constexpr int kRing2 = kSlots + kExtra / 2;
-  static constexpr uint32_t kSmemBytes = kBlobBytes + kStageBytes + kOnesBytes + kSlots * kSlotBytes + 1024;
+  static constexpr uint32_t kSmemBytes = kBlobBytes + kRecvBytes + kOnesBytes + kSlots * kSlotBytes + 1024;
   static constexpr uint32_t kAccStride = D == 128 ? 256 : 128;    // TMEM columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccStride;
   static constexpr int kPhiWarps = 8;
@@ -99,7 +102,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // Separate barriers keep each barrier's phases consumed in order by one
   // consumer, so parity waits cannot alias.
   __shared__ __align__(8) uint64_t p1full, p1empty, accfull[2], accempty[2];
-  __shared__ __align__(8) uint64_t stage_ready, blob_ready;   // arrivals from every CTA of the cluster
+  // Combine: peers_free gets one (relaxed) arrival from every CTA of the
+  // cluster once its image and receive regions are out of phase-1 use;
+  // recv_full completes when every CTA's share of this CTA's chunks has
+  // arrived, blob_full when the whole image has (transaction counts of the
+  // asynchronous stores); recv_drained once this CTA has summed its chunks.
+  __shared__ __align__(8) uint64_t peers_free, recv_full, blob_full, recv_drained;
   __shared__ uint32_t tmem_slot;
   __shared__ int comb_flag, ep_flag;
 
@@ -111,17 +119,17 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   const int T = (rank + 1) * tiles / S - tile0;   // >= 1 because S <= tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* blob = smem;
-  uint8_t* stage = blob + C::kBlobBytes;
-  uint8_t* ones = stage + C::kStageBytes;
+  uint8_t* recv = blob + C::kBlobBytes;
+  uint8_t* ones = recv + C::kRecvBytes;
   uint8_t* slots = ones + C::kOnesBytes;
   // Physical slots 0..kSlots-1 are the ring, kSlots and kSlots+1 the image
-  // and staging regions.  Phase-1 use i (K, V of tile i / 2) takes slot
+  // and receive regions.  Phase-1 use i (K, V of tile i / 2) takes slot
   // i % kRing1; phase-2 use u (Q tile u) takes ring2(u % kRing2), the ring
-  // plus the staging region.  Every use of a slot completes one phase of its
+  // plus the receive region.  Every use of a slot completes one phase of its
   // full / ready / empty barriers, so a use's phase parity is the number of
   // earlier uses of that slot.
   auto slot_ptr = [&](int phys) {
-    return phys < C::kSlots ? slots + phys * C::kSlotBytes : (phys == C::kSlots ? blob : stage);
+    return phys < C::kSlots ? slots + phys * C::kSlotBytes : (phys == C::kSlots ? blob : recv);
   };
   auto uses1 = [&](int phys) { return (2 * T + C::kRing1 - 1 - phys) / C::kRing1; };   // phase-1 uses
   auto ring2 = [&](int j) { return j < C::kSlots ? j : C::kSlots + 1; };
@@ -148,9 +156,16 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       mbar_init(&accfull[i], 1);
       mbar_init(&accempty[i], 8);
     }
-    mbar_init(&stage_ready, S);
-    mbar_init(&blob_ready, S);
+    mbar_init(&peers_free, S);
+    mbar_init(&recv_full, 1);
+    mbar_init(&blob_full, 1);
+    mbar_init(&recv_drained, 1);
     fence_mbarrier_init();
+    // every CTA sends this CTA its share of the chunks [i0, i1) it owns; the
+    // owners together send the whole image
+    const int i0 = rank * C::kChunks / S, i1 = (rank + 1) * C::kChunks / S;
+    mbar_arrive_expect_tx(&recv_full, static_cast<uint32_t>(S * (i1 - i0) * 16));
+    mbar_arrive_expect_tx(&blob_full, static_cast<uint32_t>(C::kChunks * 16));
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -168,7 +183,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     const uint32_t w = one ? 0x3F803F80u : 0u;
     *reinterpret_cast<uint4*>(ones + off) = make_uint4(w, w, w, w);
   }
-  // Rows D+1..kNB-1 of the operand image are the MMA's zero padding.
+  // Rows D+1..kNB-1 of the operand image (the MMA's N padding) only feed
+  // accumulator columns D+1.. that nobody reads; they start at zero, and
+  // where the image region serves as a phase-1 slot they keep whatever the
+  // last tile left there.
   for (int i = threadIdx.x; i < (D / 64) * (C::kNB - D - 1) * 8; i += blockDim.x) {
     const int a = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
     const int n = D + 1 + rem / 8, c = rem % 8;
@@ -188,17 +206,17 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // Slot sequence: K, V of each phase-1 tile, then the Q tiles.  The first
   // round of slots is issued before the cluster handshake.
   int seq = 0;
-  bool staging_free = false;
+  bool recv_free = false;
   auto issue = [&](int upto) {
     while (seq < upto) {
       const bool p1 = seq < 2 * T;
       const int s = p1 ? seq % C::kRing1 : q_slot(seq - 2 * T);
       const int round = p1 ? seq / C::kRing1 : q_round(seq - 2 * T);
       if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, status)) return;
-      if (!p1 && s == C::kSlots + 1 && !staging_free) {
-        // the staging region is read by the whole cluster until the image is complete
-        if (!mbar_wait_cluster(&blob_ready, 0, status)) return;
-        staging_free = true;
+      if (!p1 && s == C::kSlots + 1 && !recv_free) {
+        // the receive region holds the cluster's partials until this CTA has summed them
+        if (!mbar_wait(&recv_drained, 0, status)) return;
+        recv_free = true;
       }
       const bool is_v = p1 && (seq & 1);
       const CUtensorMap* m = p1 ? (is_v ? &tm_v : &tm_k) : &tm_q;
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         umma_commit(&empty[sv]);
       }
       umma_commit(&p1full);
-      if (ok && mbar_wait_cluster(&blob_ready, 0, status)) {
+      if (ok && mbar_wait_cluster(&blob_full, 0, status)) {
         fence_proxy_async_smem();   // the cluster's stores into `blob` feed the tensor core
         const uint32_t ba = smem_u32(blob);
         for (int u = 0; u < T; ++u) {
@@ -332,14 +350,30 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     if (leader) got = mbar_wait(&p1full, 0, status);
     bool ok = sync_ok(got);
     if (ok) {
-      // (1) partial -> own shared memory, bf16, image layout
+      // (1) this CTA's image and receive regions are out of phase-1 use (the
+      // MMAs that read them are complete): tell every CTA, then wait until
+      // every CTA has said the same.  A signal only, so a relaxed arrive.
+      if (ct < S) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&peers_free), ct));
+      if (leader) got = mbar_wait_cluster(&peers_free, 0, status);
+      ok = sync_ok(got);
+    }
+    // Chunk i (row i / (D/8), feature chunk i % (D/8)) of image rows 0..D is
+    // owned by CTA o with i0(o) <= i < i0(o + 1), i0(o) = o * kChunks / S;
+    // slice `r` of o's receive buffer holds CTA r's partial of those chunks.
+    const int slice = (C::kChunks + S - 1) / S;
+    if (ok) {
+      // (2) the partial (kv | ksum)^T, rounded to bf16, chunk by chunk to
+      // the owners
       tc_fence_after();
-      auto put_row = [&](int n, const float* v, int c0) {   // 32 values of row n from column c0
+      const uint32_t recv_base = smem_u32(recv), recv_bar = smem_u32(&recv_full);
+      auto push_row = [&](int n, const float* v, int c0) {   // 32 values of row n from column c0
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int c = c0 / 8 + j;
-          *reinterpret_cast<uint4*>(stage + (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4)) =
-              pack8(v + 8 * j);
+          const int i = n * (D / 8) + c0 / 8 + j;
+          const int o = ((i + 1) * S - 1) / C::kChunks;
+          const int js = i - o * C::kChunks / S;
+          st_async_v4(mapa_shared(recv_base + (rank * slice + js) * 16, o), pack8(v + 8 * j),
+                      mapa_shared(recv_bar, o));
         }
       };
       constexpr int kHalfCols = D / 2;
@@ -353,7 +387,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         tmem_wait_ld();
         if (valid)
 #pragma unroll
-          for (int c0 = 0; c0 < kHalfCols; c0 += 32) put_row(n, v + c0, half * kHalfCols + c0);
+          for (int c0 = 0; c0 < kHalfCols; c0 += 32) push_row(n, v + c0, half * kHalfCols + c0);
       }
       // ksum^T is row 0 of the M = 64 product: lane 0 of quarter 0
       if (q == 0) {
@@ -363,77 +397,40 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         tmem_wait_ld();
         if (lane == 0)
 #pragma unroll
-          for (int c0 = 0; c0 < kHalfCols; c0 += 32) put_row(D, v + c0, half * kHalfCols + c0);
-      }
-      if (C::kExtra) {   // the image region held K/V tiles: restore its zero padding rows
-        for (int i = ct; i < (D / 64) * (C::kNB - D - 1) * 8; i += 256) {
-          const int at = i / ((C::kNB - D - 1) * 8), rem = i % ((C::kNB - D - 1) * 8);
-          *reinterpret_cast<uint4*>(blob + at * C::kBlobAtomBytes + (D + 1 + rem / 8) * 128 + (rem % 8) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
+          for (int c0 = 0; c0 < kHalfCols; c0 += 32) push_row(D, v + c0, half * kHalfCols + c0);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p1empty);
-      // The CTA barrier orders every thread's staging stores before the
-      // leader's release-arrive at cluster scope (release is cumulative).
-      named_bar_sync(3, 256);
-      if (leader) {
-        for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stage_ready), p));
-        got = mbar_wait_cluster(&stage_ready, 0, status);
-      }
+      if (leader) got = mbar_wait_cluster(&recv_full, 0, status);
       ok = sync_ok(got);
     }
     if (ok) {
-      // (2) chunks [i0, i1) of rows 0..D of the image: the sum over the
-      // cluster's staged partials, in ascending CTA order, stored into every
-      // CTA's image.  Two chunks per thread and pass; the loads of every
-      // peer are in flight together.
-      constexpr int kChunks = (D + 1) * (D / 8);
-      constexpr int kMaxS = 8;
-      const int i0 = rank * kChunks / S, i1 = (rank + 1) * kChunks / S;
-      const uint32_t stage_base = smem_u32(stage), blob_base = smem_u32(blob);
-      for (int i = i0 + ct; i < i1; i += 2 * 256) {
-        uint32_t off[2];
-        bool has[2];
+      // (3) this CTA's chunks: the sum over the S partials in ascending CTA
+      // order, rounded to bf16, sent into the image of every CTA
+      const int i0 = rank * C::kChunks / S, i1 = (rank + 1) * C::kChunks / S;
+      const uint32_t blob_base = smem_u32(blob), blob_bar = smem_u32(&blob_full);
+      for (int js = ct; js < i1 - i0; js += 256) {
+        float acc[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ii = i + h * 256;
-          has[h] = ii < i1;
-          const int nn = ii / (D / 8), c = ii % (D / 8);
-          off[h] = (c >> 3) * C::kBlobAtomBytes + nn * 128 + (((c & 7) ^ (nn & 7)) << 4);
-        }
-        uint32_t w[2][kMaxS][4];
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int p = 0; p < S; ++p) {
+          const uint4 w = *reinterpret_cast<const uint4*>(recv + (p * slice + js) * 16);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int p = 0; p < kMaxS; ++p)
-            if (has[h] && p < S) ld_cluster_v4(mapa_shared(stage_base + off[h], p), w[h][p]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!has[h]) continue;
-          float acc[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-          for (int p = 0; p < kMaxS; ++p) {
-            if (p < S) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[h][p][e]));
-                acc[2 * e] += x.x;
-                acc[2 * e + 1] += x.y;
-              }
-            }
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            acc[2 * e] += x.x;
+            acc[2 * e + 1] += x.y;
           }
-          const uint4 val = pack8(acc);
-          for (int p = 0; p < S; ++p) st_cluster_v4(mapa_shared(blob_base + off[h], p), val);
         }
+        const uint4 val = pack8(acc);
+        const int i = i0 + js, nn = i / (D / 8), c = i % (D / 8);
+        const uint32_t off = (c >> 3) * C::kBlobAtomBytes + nn * 128 + (((c & 7) ^ (nn & 7)) << 4);
+        for (int p = 0; p < S; ++p) st_async_v4(mapa_shared(blob_base + off, p), val, mapa_shared(blob_bar, p));
       }
       named_bar_sync(3, 256);
-      if (leader)
-        for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&blob_ready), p));
+      if (leader) mbar_arrive(&recv_drained);   // the receive region may take a Q tile
     }
     if (ok) {
       // (3) outputs of the CTA's Q tiles: each warp its rows' half of the

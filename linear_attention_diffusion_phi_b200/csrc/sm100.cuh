@@ -356,6 +356,40 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// Arrive on a cluster CTA's mbarrier without ordering this thread's earlier
+// memory accesses: a pure signal that publishes no data.  (A release arrive
+// at cluster scope also waits for the CTA's in-flight bulk loads, which costs
+// microseconds while tiles are streaming in.)
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 16-byte asynchronous store into a cluster CTA's shared memory whose bytes
+// complete a transaction count on an mbarrier of that same CTA: the receiver
+// learns of the data by waiting on its own barrier, without a release fence
+// on the sending side.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint4 v, uint32_t cluster_mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(cluster_mbar)
+               : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory into a cluster CTA's shared memory (address
+// from mapa_shared); the bytes complete a transaction count on that CTA's
+// mbarrier.  The copy engine moves whole lines; per-thread remote stores of
+// 16 bytes each tie up the shared-memory pipes of both SMs one small
+// transaction at a time.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                                     uint32_t mbar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(smem_u32(src)), "r"(bytes), "r"(mbar_cluster)
+      : "memory");
+}
+
 // 16-byte store into a cluster CTA's shared memory.
 __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v) {
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
