@@ -5,27 +5,34 @@
 // sequence into kv = phi(K)^T V and ksum = sum_j phi(k_j), then
 // out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).
 //
-// One kernel.  Each head is served by a thread-block cluster of S CTAs (one
-// per SM); CTA r owns the r-th run of 128-token tiles of the head.
-//   phase 1  TMA streams the CTA's K and V tiles into a ring of shared-memory
-//            slots; eight warps apply phi to K in place (V tiles need no work
-//            and go straight to the tensor core); one thread issues
-//            tcgen05.mma  kv^T += V^T phi(K)  and  ksum^T += 1^T phi(K)  into
-//            tensor memory (fp32).
-//   combine  eight warps read the CTA's partial (kv | ksum)^T from tensor
-//            memory, round it to bf16 and send each 16-byte chunk to the
-//            cluster CTA that owns it (asynchronous distributed-shared-memory
-//            stores whose bytes complete on the owner's barrier; no global
-//            round trip).  Every CTA sums the partials of the chunks it owns
-//            in ascending CTA order (no atomics, so bitwise reproducible) and
-//            sends the sums into the image of every CTA of the cluster: the
-//            apply MMA's B operand, in its layout.
-//   phase 2  the CTA's Q tiles (prefetched during the combine) get phi in
-//            place, one MMA per tile computes [num | den] = phi(Q) [kv | ksum],
-//            and four warps write out = num / (den + eps) as bf16 into the Q
-//            tile's own slot, which TMA stores to global memory.
+// One kernel per forward.  Each head is served by a thread-block cluster of S
+// CTAs (one per SM); CTA r owns the r-th run of 128-token tiles of the head.
 // S is the largest cluster size (<= 8) whose clusters for all heads can be
-// resident at once on this device.
+// resident at once on this device.  Two kernels share that plan:
+//
+// fused_t_kernel (D = 128)
+//   phase 1  TMA streams the CTA's K and V tiles into a ring of shared-memory
+//            slots.  Eight warps read each K tile transposed (ldmatrix.trans),
+//            apply phi and write phi(K)^T into tensor memory (lane = feature);
+//            the K slot is free again at once.  One thread issues tcgen05.mma
+//            kv = phi(K)^T V  (B = the V tile as TMA left it) and
+//            ksum = phi(K)^T 1  into tensor memory (fp32).
+//   combine  eight warps write the CTA's partial [kv | ksum], rounded to bf16,
+//            into its own copy of the apply MMA's B operand (stmatrix.trans:
+//            row = value, features contiguous).  The image rows are split
+//            among the cluster's CTAs; bulk copies send every owner its rows
+//            from every CTA, the owner sums them in ascending CTA order (no
+//            atomics: bitwise reproducible) and bulk-copies the sums into the
+//            image of every CTA.  No global round trip.
+//   phase 2  the CTA's Q tiles (prefetched during the combine) get phi into
+//            tensor memory (lane = token), one MMA per tile computes
+//            [num | den] = phi(Q) [kv | ksum], and eight warps write
+//            out = num / (den + eps) as bf16 into a staging buffer that TMA
+//            stores to global memory.
+//
+// fused_kernel (D = 64): the same plan with phi(K) and phi(Q) applied in place
+// in shared memory, kv^T = V^T phi(K) and ksum^T = 1^T phi(K), and a combine
+// by 16-byte asynchronous remote stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -486,6 +493,480 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   cluster_sync_all();   // no CTA leaves while the cluster may still address its shared memory
 }
 
+// ---------------------------------------------------------------------------
+// D = 128: phi(K)^T and phi(Q) in tensor memory.
+//
+// The phi warps read each K tile with ldmatrix.trans (16 tokens x 16 features
+// per instruction, two tokens of one feature per register), apply phi and
+// store the result with tcgen05.st into tensor memory, lane = feature and
+// column = token pair: the A operand of  kv = phi(K)^T V  (M = 128 features,
+// N = 128 values, B = the V tile as TMA left it) and of  ksum = phi(K)^T 1
+// (N = 16, B = a block of ones).  The K slot is free as soon as it has been
+// read, and the tensor core reads only V from shared memory.  Q tiles go the
+// same way untransposed (lane = token), as the A operand of the apply MMA.
+// The partial state [kv | ksum] (lane = feature, column = value) is written
+// into the CTA's image with stmatrix.trans (row = value, features
+// contiguous), and the cluster exchanges image rows with bulk copies:
+// every CTA sends the rows that CTA o owns to o, o sums them in ascending
+// CTA order and sends the sum back into every CTA's image.
+
+struct CfgT {
+  static constexpr int D = 128;
+  static constexpr int kBoxes = 2;
+  static constexpr uint32_t kSlotBytes = 128u * D * 2u;
+  static constexpr int kNB = D + 16;                       // apply MMA N: values + den
+  static constexpr uint32_t kBlobAtomBytes = kNB * 128;    // image: 2 k-atoms of kNB rows x 128 B
+  static constexpr uint32_t kBlobBytes = 2 * kBlobAtomBytes;
+  static constexpr int kRows = D + 1;                      // exchanged image rows: kv rows, ksum row
+  static constexpr uint32_t kRecvBytes = kBlobBytes;       // >= 8 senders x 2 atoms x 17 rows x 128 B
+  static_assert(8u * 2u * ((kRows + 7) / 8) * 128u <= kRecvBytes, "receive buffer too small");
+  static constexpr uint32_t kOnesBytes = 2048;
+  static constexpr int kSlots = 4;
+  static constexpr int kRing1 = kSlots + 2;                // phase 1 also uses the image and receive regions
+  static constexpr int kRing2 = kSlots - 1;                // phase-2 Q ring; slot kSlots-1 stages outputs
+  static constexpr uint32_t kSmemBytes = kBlobBytes + kRecvBytes + kOnesBytes + kSlots * kSlotBytes + 1024;
+  // tensor memory: [kv | ksum] of phase 1 at column 0 (lane = feature; ksum
+  // in columns D..D+15); phase-2 accumulators at 0 and kNB (lane = token);
+  // three A buffers of 64 columns above them.
+  static constexpr uint32_t kAccStride = kNB;
+  static constexpr int kABufs = 3;
+  static constexpr uint32_t kABufCols = 64;
+  static constexpr uint32_t kABuf0 = 2 * kNB;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kABuf0 + kABufs * kABufCols <= kTmemCols, "tensor memory");
+  static constexpr int kPhiWarps = 8;
+  static constexpr int kCombWarp0 = 2 + kPhiWarps;
+  static constexpr int kThreads = 32 * (kCombWarp0 + 8);
+};
+
+template <int FMAP>
+__global__ void __launch_bounds__(CfgT::kThreads, 1)
+    fused_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                   int* status, int N, int tiles, float eps) {
+  using C = CfgT;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  // full: a K or Q tile has arrived (waited on by the phi warps, every phase
+  // in order); vfull: a V tile has arrived (MMA issuer); empty: a phase-1
+  // slot is free again (a K slot once the phi warps have read it, a V slot
+  // once its MMAs are done); qfree: a Q tile has been read by the phi warps.
+  __shared__ __align__(8) uint64_t full[C::kRing1], vfull[C::kRing1], empty[C::kRing1], qfree[C::kRing1];
+  // A buffers in tensor memory, used in turn by the T key tiles and then the
+  // T query tiles: written by the phi warps (aready), read by the MMAs (aempty).
+  __shared__ __align__(8) uint64_t aready[C::kABufs], aempty[C::kABufs];
+  __shared__ __align__(8) uint64_t p1full, p1empty, accfull[2], accempty[2];
+  // combine: peers_free (one relaxed arrival per cluster CTA: its receive
+  // region is out of phase-1 use); recv_full (the rows this CTA owns have
+  // arrived from every other CTA); blob_full (the summed rows of every other
+  // owner have arrived, and this CTA's own sum is written).
+  __shared__ __align__(8) uint64_t peers_free, recv_full, blob_full;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int comb_flag, ep_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = static_cast<int>(gridDim.x);
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int bh = blockIdx.y;
+  const int tile0 = rank * tiles / S;
+  const int T = (rank + 1) * tiles / S - tile0;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* blob = smem;
+  uint8_t* recv = blob + C::kBlobBytes;
+  uint8_t* ones = recv + C::kRecvBytes;
+  uint8_t* slots = ones + C::kOnesBytes;
+  auto slot_ptr = [&](int phys) {
+    return phys < C::kSlots ? slots + phys * C::kSlotBytes : (phys == C::kSlots ? blob : recv);
+  };
+  // Phase-1 use j (K, V of tile j / 2) takes slot j % kRing1: K tiles in even
+  // slots, V tiles in odd ones.  Q tile u takes ring slot u % kRing2.
+  auto uses1 = [&](int phys) { return (2 * T + C::kRing1 - 1 - phys) / C::kRing1; };
+  auto q_full_round = [&](int u) {   // phases of full[] before Q tile u
+    const int s = u % C::kRing2;
+    return ((s & 1) == 0 ? uses1(s) : 0) + u / C::kRing2;
+  };
+  // image rows [row0(o), row0(o + 1)) are owned by cluster CTA o
+  auto row0 = [&](int o) { return o * C::kRows / S; };
+  const int rmax = (C::kRows + S - 1) / S;
+  const uint32_t recv_slot = 2u * static_cast<uint32_t>(rmax) * 128u;   // receive bytes per sender
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kRing1; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&vfull[i], 1);
+      mbar_init(&empty[i], (i & 1) == 0 ? C::kPhiWarps : 1);
+      mbar_init(&qfree[i], C::kPhiWarps);
+    }
+    for (int i = 0; i < C::kABufs; ++i) {
+      mbar_init(&aready[i], C::kPhiWarps);
+      mbar_init(&aempty[i], 1);
+    }
+    mbar_init(&p1full, 1);
+    mbar_init(&p1empty, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 8);
+    }
+    mbar_init(&peers_free, S);
+    mbar_init(&recv_full, 1);
+    mbar_init(&blob_full, 2);
+    fence_mbarrier_init();
+    const uint32_t mine = static_cast<uint32_t>(row0(rank + 1) - row0(rank));
+    mbar_arrive_expect_tx(&recv_full, static_cast<uint32_t>(S - 1) * mine * 256u);
+    mbar_arrive_expect_tx(&blob_full, static_cast<uint32_t>(C::kRows - static_cast<int>(mine)) * 256u);
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_out);
+    comb_flag = 0;
+    ep_flag = 0;
+  }
+  // B operand of the ksum MMA: a block of bf16 ones (any layout reads 1.0)
+  for (int i = threadIdx.x; i < static_cast<int>(C::kOnesBytes / 16); i += blockDim.x)
+    *reinterpret_cast<uint4*>(ones + 16 * i) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  // ------------------------------------------------------------ producer
+  int seq = 0;
+  auto issue = [&](int upto) {
+    while (seq < upto) {
+      const bool p1 = seq < 2 * T;
+      const int u = seq - 2 * T;
+      const int s = p1 ? seq % C::kRing1 : u % C::kRing2;
+      if (p1) {
+        const int round = seq / C::kRing1;
+        if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, status)) return;
+      } else if (u >= C::kRing2) {
+        if (!mbar_wait(&qfree[s], ((u / C::kRing2) - 1) & 1, status)) return;
+      } else if (uses1(s) > 0) {
+        if (!mbar_wait(&empty[s], (uses1(s) - 1) & 1, status)) return;
+      }
+      const bool is_v = p1 && (seq & 1);
+      const CUtensorMap* m = p1 ? (is_v ? &tm_v : &tm_k) : &tm_q;
+      const int tile = p1 ? seq / 2 : u;
+      uint64_t* bar = is_v ? &vfull[s] : &full[s];
+      uint8_t* dst = slot_ptr(s);
+      mbar_arrive_expect_tx(bar, C::kSlotBytes);
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b)
+        tma_load_3d(dst + b * kBoxBytes, m, bar, 64 * b, (tile0 + tile) * kTileTokens, bh);
+      ++seq;
+    }
+  };
+  pdl_wait();
+  pdl_launch_dependents();
+  cluster_arrive_relaxed();
+  if (warp == 0 && lane == 0) issue(min(C::kRing1, 2 * T));
+  cluster_wait();
+
+  if (warp == 0) {
+    if (lane == 0) issue(3 * T);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);        // A = phi(K)^T (TMEM), B = V (MN-major)
+      constexpr uint32_t idesc_ks = idesc_bf16_f32(128, 16, 0, 0);       // B = ones (K-major)
+      constexpr uint32_t idesc_ap = idesc_bf16_f32(128, C::kNB, 0, 0);   // A = phi(Q) (TMEM), B = image
+      const uint64_t ones_desc = smem_desc_noswz(smem_u32(ones), 128, 256);
+      bool ok = true;
+      for (int t = 0; t < T; ++t) {
+        const int sv = (2 * t + 1) % C::kRing1, b = t % C::kABufs;
+        if (!mbar_wait(&aready[b], (t / C::kABufs) & 1, status) ||
+            !mbar_wait(&vfull[sv], ((2 * t + 1) / C::kRing1) & 1, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t atm = tmem + C::kABuf0 + b * C::kABufCols;
+        const uint64_t vdesc = smem_desc_sw128(smem_u32(slot_ptr(sv)), kBoxBytes, 1024);
+        // 16 tokens per MMA: 8 A columns, 2048 bytes of V
+        if (t == 0) {
+          umma_ts<0>(tmem, atm, vdesc, idesc_kv);
+          umma_ts<0>(tmem + D, atm, ones_desc, idesc_ks);
+        } else {
+          umma_ts<1>(tmem, atm, vdesc, idesc_kv);
+          umma_ts<1>(tmem + D, atm, ones_desc, idesc_ks);
+        }
+#pragma unroll
+        for (int k = 1; k < kTileTokens / 16; ++k) {
+          umma_ts<1>(tmem, atm + 8 * k, desc_add(vdesc, 2048 * k), idesc_kv);
+          umma_ts<1>(tmem + D, atm + 8 * k, ones_desc, idesc_ks);
+        }
+        umma_commit(&empty[sv]);
+        umma_commit(&aempty[b]);
+      }
+      umma_commit(&p1full);
+      if (ok && mbar_wait_cluster(&blob_full, 0, status)) {
+        fence_proxy_async_smem();   // the cluster's copies into `blob` feed the tensor core
+        const uint64_t bdesc = smem_desc_sw128(smem_u32(blob), 16, 1024);
+        for (int u = 0; u < T; ++u) {
+          const int j = T + u, b = j % C::kABufs;
+          const int a = u & 1, ar = u >> 1;
+          bool got = mbar_wait(&aready[b], (j / C::kABufs) & 1, status);
+          if (got) got = ar == 0 ? mbar_wait(&p1empty, 0, status) : mbar_wait(&accempty[a], (ar - 1) & 1, status);
+          if (!got) break;
+          tc_fence_after();
+          const uint32_t atm = tmem + C::kABuf0 + b * C::kABufCols;
+          const uint32_t d = tmem + a * C::kAccStride;
+          umma_ts<0>(d, atm, bdesc, idesc_ap);
+#pragma unroll
+          for (int k = 1; k < D / 16; ++k)
+            umma_ts<1>(d, atm + 8 * k, desc_add(bdesc, (k >> 2) * C::kBlobAtomBytes + (k & 3) * 32), idesc_ap);
+          umma_commit(&aempty[b]);
+          umma_commit(&accfull[a]);
+        }
+      }
+    }
+  } else if (warp < C::kCombWarp0) {
+    // ------------------------------------------------------- phi warps
+    // Tensor-memory lane quarter qd (the warp's accessible lanes); half hf.
+    const int qd = warp & 3, hf = (warp - 2) >> 2;
+    bool ok = true;
+    // K tiles: features 32 qd .. 32 qd + 31 (two 16-lane halves), tokens
+    // 64 hf .. 64 hf + 63 (four 16-token blocks)
+    const int lm = lane >> 3, lr = lane & 7;
+    for (int t = 0; t < T && ok; ++t) {
+      const int s = (2 * t) % C::kRing1, b = t % C::kABufs;
+      if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) {
+        ok = false;
+        break;
+      }
+      const uint32_t base = smem_u32(slot_ptr(s));
+      uint32_t x[2][4][4];
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < 4; ++tb) {
+          // matrix lm: tokens +8 (lm >> 1), features +8 (lm & 1); row lr
+          const int tok = 64 * hf + 16 * tb + 8 * (lm >> 1) + lr;
+          const int cc = 4 * qd + 2 * fh + (lm & 1);
+          ldsm_x4_trans(base + swz_off(tok, cc), x[fh][tb]);
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);   // the K tile is in registers
+      // key rows past the sequence end must not reach kv or ksum
+      const int valid = min(kTileTokens, N - (tile0 + t) * kTileTokens);
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < 4; ++tb)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            uint32_t w = phi_pair<FMAP>(x[fh][tb][r]);
+            if (valid < kTileTokens) {
+              const int tok = 64 * hf + 16 * tb + 8 * (r >> 1) + 2 * (lane & 3);
+              w &= (tok < valid ? 0x0000FFFFu : 0u) | (tok + 1 < valid ? 0xFFFF0000u : 0u);
+            }
+            x[fh][tb][r] = w;
+          }
+      if (t >= C::kABufs && !warp_wait(&aempty[b], ((t / C::kABufs) - 1) & 1, status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < 4; ++tb)
+          tmem_st_16x128b_x2(tmem + (static_cast<uint32_t>(32 * qd + 16 * fh) << 16) + C::kABuf0 +
+                                 b * C::kABufCols + 32 * hf + 8 * tb,
+                             x[fh][tb]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[b]);
+    }
+    // Q tiles: token row 32 qd + lane, features 64 hf .. 64 hf + 63
+    const int i = 32 * qd + lane;
+    const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
+    for (int u = 0; u < T && ok; ++u) {
+      const int s = u % C::kRing2, j = T + u, b = j % C::kABufs;
+      if (!warp_wait(&full[s], q_full_round(u) & 1, status)) break;
+      const uint8_t* src = slot_ptr(s);
+      uint4 x[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
+      uint32_t w[32];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const uint4 y = phi_chunk<FMAP>(x[m]);
+        w[4 * m] = y.x;
+        w[4 * m + 1] = y.y;
+        w[4 * m + 2] = y.z;
+        w[4 * m + 3] = y.w;
+      }
+      if (j >= C::kABufs && !warp_wait(&aempty[b], ((j / C::kABufs) - 1) & 1, status)) break;
+      tc_fence_after();
+      tmem_st32(tmem + C::kABuf0 + b * C::kABufCols + 32 * hf + lanes, w);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[b]);
+    }
+  } else {
+    // ----------------------------------------- combine, then the outputs
+    const int ct = threadIdx.x - 32 * C::kCombWarp0;   // 0..255
+    const int half = ct >> 7;
+    const bool leader = ct == 0;
+    const int q = warp & 3;
+    const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
+    bool got = true;
+    auto sync_ok = [&](bool mine) {
+      if (leader && !mine) comb_flag = 1;
+      named_bar_sync(3, 256);
+      return comb_flag == 0;
+    };
+    if (leader) got = mbar_wait(&p1full, 0, status);
+    bool ok = sync_ok(got);
+    if (ok) {
+      // (1) the partial [kv | ksum] (lane = feature, column = value) into
+      // this CTA's image, bf16, row = value with the features contiguous:
+      // 16 features x 16 columns per tcgen05.ld / stmatrix.trans pair.
+      // Columns D..D+15 all hold ksum: they fill rows D..D+15, whose copies
+      // above row D only feed accumulator columns nobody reads.
+      tc_fence_after();
+      const uint32_t blob_base = smem_u32(blob);
+      auto put = [&](int fh, int n0) {
+        uint32_t r[8];
+        tmem_ld_16x256b_x2(tmem + tq + (static_cast<uint32_t>(16 * fh) << 16) + n0, r);
+        tmem_wait_ld();
+        // matrix m: features +8 (m & 1), values +8 (m >> 1); row = value
+        const int m = lane >> 3;
+        const int n = n0 + 8 * (m >> 1) + (lane & 7);
+        const int c = 4 * q + 2 * fh + (m & 1);   // 16-byte feature chunk
+        const uint32_t addr =
+            blob_base + (c >> 3) * C::kBlobAtomBytes + n * 128 + (((c & 7) ^ (n & 7)) << 4);
+        stsm_x4_trans(addr, pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                      pack_bf16x2(r[6], r[7]));
+      };
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int nb = 0; nb < 4; ++nb) put(fh, 64 * half + 16 * nb);
+      if (half == 1) {
+        put(0, D);
+        put(1, D);
+      }
+      fence_proxy_async_smem();   // read by the bulk copies and the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p1empty);
+      // (2) every CTA's receive region is out of phase-1 use: send each owner
+      // its rows, one bulk copy per owner and k-atom
+      named_bar_sync(3, 256);
+      if (ct < S) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&peers_free), ct));
+      if (ct < 32) {
+        int g = 1;
+        if (lane == 0) g = mbar_wait_cluster(&peers_free, 0, status) ? 1 : 0;
+        g = __shfl_sync(0xffffffffu, g, 0);
+        if (g && lane < 2 * (S - 1)) {
+          const int o = (rank + 1 + (lane >> 1)) % S, a = lane & 1;
+          const int n0 = row0(o), n1 = row0(o + 1);
+          bulk_copy_to_cluster(mapa_shared(smem_u32(recv) + rank * recv_slot + a * rmax * 128, o),
+                               blob + a * C::kBlobAtomBytes + n0 * 128, static_cast<uint32_t>(n1 - n0) * 128u,
+                               mapa_shared(smem_u32(&recv_full), o));
+        }
+        if (leader) got = g != 0;
+      }
+      if (leader && got) got = mbar_wait_cluster(&recv_full, 0, status);
+      ok = sync_ok(got);
+    }
+    if (ok) {
+      // (3) this CTA's rows: the sum over the S partials in ascending CTA
+      // order, rounded to bf16, into its own image, then into every other
+      // CTA's image.  Positions within a row are the same in every copy.
+      const int n0 = row0(rank), rows = row0(rank + 1) - n0;
+      for (int js = ct; js < 2 * rows * 8; js += 256) {
+        const int a = js / (rows * 8), rem = js % (rows * 8);
+        const uint32_t off_img = a * C::kBlobAtomBytes + (n0 + rem / 8) * 128 + (rem % 8) * 16;
+        const uint32_t off_rcv = a * rmax * 128 + rem * 16;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int p = 0; p < S; ++p) {
+          const uint8_t* src = p == rank ? blob + off_img : recv + p * recv_slot + off_rcv;
+          const uint4 w = *reinterpret_cast<const uint4*>(src);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            acc[2 * e] += x.x;
+            acc[2 * e + 1] += x.y;
+          }
+        }
+        *reinterpret_cast<uint4*>(blob + off_img) = pack8(acc);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(3, 256);
+      if (ct < 2 * (S - 1)) {
+        const int o = (rank + 1 + (ct >> 1)) % S, a = ct & 1;
+        const uint32_t off = a * C::kBlobAtomBytes + n0 * 128;
+        bulk_copy_to_cluster(mapa_shared(smem_u32(blob) + off, o), blob + off, static_cast<uint32_t>(rows) * 128u,
+                             mapa_shared(smem_u32(&blob_full), o));
+      }
+      if (leader) mbar_arrive(&blob_full);   // this CTA's own rows are in place
+    }
+    if (ok) {
+      // (4) outputs: each warp its rows' half of the value columns, staged
+      // in buffer u & 1 (the receive region, then the last ring slot), one
+      // TMA store per tile
+      constexpr int kHalfCols = D / 2;
+      for (int u = 0; u < T; ++u) {
+        const int a = u & 1, ar = u >> 1;
+        got = true;
+        if (leader) {
+          got = mbar_wait(&accfull[a], ar & 1, status);
+          if (u >= 2) bulk_wait_group_read<1>();
+        }
+        if (leader && !got) ep_flag = 1;
+        named_bar_sync(2, 256);
+        if (ep_flag) break;
+        tc_fence_after();
+        const uint32_t trow = tmem + a * C::kAccStride + tq;
+        const int r = 32 * q + lane;
+        float v[kHalfCols];
+        const float den = tmem_ld1(trow + D);
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfCols; c0 += 32) tmem_ld32(trow + half * kHalfCols + c0, *reinterpret_cast<float(*)[32]>(v + c0));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[a]);
+        const float inv = 1.0f / (den + eps);
+#pragma unroll
+        for (int e = 0; e < kHalfCols; ++e) v[e] *= inv;
+        uint8_t* ob = a == 0 ? recv : slots + (C::kSlots - 1) * C::kSlotBytes;
+#pragma unroll
+        for (int jj = 0; jj < kHalfCols / 8; ++jj)
+          *reinterpret_cast<uint4*>(ob + swz_off(r, half * (kHalfCols / 8) + jj)) = pack8(v + 8 * jj);
+        fence_proxy_async_smem();
+        named_bar_sync(2, 256);
+        if (leader) {
+#pragma unroll
+          for (int bb = 0; bb < C::kBoxes; ++bb)
+            tma_store_3d(&tm_out, ob + bb * kBoxBytes, 64 * bb, (tile0 + u) * kTileTokens, bh);
+          bulk_commit_group();
+        }
+      }
+      if (leader) bulk_wait_group<0>();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  cluster_sync_all();
+}
+
 // Largest cluster size S <= min(8, tiles) for which B*H clusters of `kern`
 // fit on the device at once (one wave), per device and kernel; 1 when none
 // does.
@@ -534,11 +1015,9 @@ int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int
   return 1;
 }
 
-template <int D, int FMAP>
-cudaError_t run(const LaunchArgs& a) {
-  using C = Cfg<D>;
+template <class C, class Kern>
+cudaError_t launch_fused(const LaunchArgs& a, Kern kern) {
   const Plan& p = *a.p;
-  auto kern = fused_kernel<D, FMAP>;
   cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
   const int S = pick_cluster(reinterpret_cast<const void*>(kern), C::kSmemBytes, C::kThreads, p.BH, p.tiles);
@@ -565,8 +1044,9 @@ cudaError_t run(const LaunchArgs& a) {
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
   const Plan& p = *a.p;
   if (p.F != 0) return cudaErrorNotSupported;
-  if (p.D == 128) return p.fmap == 0 ? run<128, 0>(a) : run<128, 1>(a);
-  if (p.D == 64) return p.fmap == 0 ? run<64, 0>(a) : run<64, 1>(a);
+  if (p.D == 128) return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0>) : launch_fused<CfgT>(a, fused_t_kernel<1>);
+  if (p.D == 64)
+    return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>) : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>);
   return cudaErrorNotSupported;
 }
 

@@ -252,6 +252,49 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// Four 8 x 8 b16 matrices, transposed: thread i gives the address of row
+// i % 8 of matrix i / 8 (16 contiguous bytes); register m of thread t holds
+// rows 2 (t % 4) and 2 (t % 4) + 1 of column t / 4 of matrix m (the lower
+// row in the low half).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// The inverse: register m of thread t holds elements (t / 4, 2 (t % 4)) and
+// (t / 4, 2 (t % 4) + 1) of matrix m; column c of matrix m is stored as 16
+// contiguous bytes at the address given by thread 8 m + c.
+__device__ __forceinline__ void stsm_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0),
+               "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
+// 16 lanes x 8 columns: r0 -> (lane t/4, col t%4), r1 -> (lane 8 + t/4, col
+// t%4), r2, r3 the same at col 4 + t%4 (t = thread of the warp).
+__device__ __forceinline__ void tmem_st_16x128b_x2(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+
+// 16 lanes x 16 columns: r0, r1 -> (lane t/4, cols 2(t%4), 2(t%4)+1), r2, r3
+// -> lane 8 + t/4, the same columns; r4..r7 the same at columns + 8.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+
+// Two fp32 values (as bits) rounded to a bf16 pair, `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------- descriptors (sm_100 UMMA)
