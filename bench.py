@@ -402,7 +402,12 @@ class Timed:
         self.op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, None if W is None else W.to(dev))
         self.graphs = graphs
         self.g_all = None
+        self.g_all_steps = 0
         self.g_one = []
+        # steps the timed region will run: the big graph holds as many whole
+        # rounds of the input sets as fit in it (at most 64 steps), so a timed
+        # region of K steps pays few graph launches
+        self.steps_hint = 64
 
     def step(self, i):
         q, k, v, o = self.sets[i % self.nsets]
@@ -412,9 +417,11 @@ class Timed:
         import torch
         if not self.graphs:
             return
+        rounds = max(1, min(self.steps_hint, 64) // self.nsets)
+        self.g_all_steps = rounds * self.nsets
         self.g_all = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.g_all):
-            for j in range(self.nsets):
+            for j in range(self.g_all_steps):
                 self.step(j)
         for j in range(self.nsets):
             g = torch.cuda.CUDAGraph()
@@ -430,9 +437,9 @@ class Timed:
                 self.step(i)
             return
         i = 0
-        while i + self.nsets <= k:
+        while i + self.g_all_steps <= k:
             self.g_all.replay()
-            i += self.nsets
+            i += self.g_all_steps
         while i < k:
             self.g_one[i % self.nsets].replay()
             i += 1
@@ -538,6 +545,7 @@ def main():
     hbm, tflops, src = peaks()
 
     tw = Timed(w, dev, rank, graphs=not args.no_graph)
+    tw.steps_hint = args.steps
     sampler = ClockSampler(local)
     sampler.start()
     tw.warm(args.warmup, args.soak_s)
@@ -594,10 +602,11 @@ def main():
             x = WORKLOADS[name]
             try:
                 tx = Timed(x, dev, rank, graphs=not args.no_graph)
+                xsteps = max(args.steps, 100)
+                tx.steps_hint = xsteps
                 smp = ClockSampler(local)
                 smp.start()
                 tx.warm(args.warmup, 0.3)
-                xsteps = max(args.steps, 100)
                 xms = tx.timed_ms(xsteps, stream, ws)
                 xclk = smp.stop()
                 assert tx.op.sync_status() == la.LA_OK, "device-side error during the timed region"

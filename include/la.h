@@ -97,12 +97,17 @@ la_status_t la_set_projection(la_handle_t handle, const void* W, int H, int D, i
 
 /* Workspace bytes la_forward needs for this problem (0 if the arguments are
  * invalid for the handle).  The size depends only on the arguments and the
- * device's SM count.  It is 256 bytes (the status word) for bf16 non-causal
- * problems with F = 0 and for bf16 causal problems with at least as many
- * heads (B*H) as SMs; otherwise it holds fp32 partial states and grows with
- * B*H and the number of splits per head: on 148 SMs about 2 MB for causal
- * [4, 8, 32768, 64], 11 MB for [1, 24, 4608, 128] with F = 256, and 13.5 GB
- * for B*H = 65535 with F = 256. */
+ * device (its SM count and how many thread-block clusters of the kernels fit
+ * on it at once).  Every workspace starts with a 4352-byte header (the status
+ * word and the synchronisation words of the exchange below).  bf16 non-causal
+ * problems with F = 0 need the header only, plus, when a head is spread over
+ * several clusters (D = 128 with fewer heads than SMs), an exchange area of
+ * 36 KB per head and cluster: 2.6 MB for [1, 24, 4608, 128] on 148 SMs, never
+ * more than 36 KB per SM.  bf16 causal problems with at least as many heads
+ * (B*H) as SMs need the header only.  Otherwise the workspace holds fp32
+ * partial states and grows with B*H and the number of splits per head: on
+ * 148 SMs about 2 MB for causal [4, 8, 32768, 64], 11 MB for
+ * [1, 24, 4608, 128] with F = 256, and 13.5 GB for B*H = 65535 with F = 256. */
 size_t la_workspace_bytes(la_handle_t handle, int B, int H, int N, int D, int F, int causal);
 
 /* Bind a caller-owned device workspace (256-byte aligned).  The library writes
@@ -141,10 +146,10 @@ la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* 
  * LA_ERR_CUDA. */
 la_status_t la_sync_status(la_handle_t handle, void* stream);
 
-/* Size of the static scratch array behind la_forward_noalloc (2 MiB).  A
+/* Size of the static scratch array behind la_forward_noalloc (8 MiB).  A
  * device holds it from the moment the library's code is loaded on it (at the
  * latest, the first la_forward_noalloc call there) until the process exits. */
-#define LA_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+#define LA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
 /* For callers that cannot allocate device memory (no cudaMalloc, no pool of
  * their own, nothing to bind with la_set_workspace): the bf16, non-causal,
@@ -153,19 +158,22 @@ la_status_t la_sync_status(la_handle_t handle, void* stream);
  * pages have no counterpart; this entry point exists only for such callers.
  * q, k, v, out: device pointers, bf16 [B, H, N, D] as for la_forward (out
  * overlapping q, k or v gives LA_ERR_INVALID_ARG); D is 64 or 128.  No handle is used and nothing is allocated, on host or device.
- * The scratch this path needs (its status word, 256 bytes) does not grow
- * with the problem, so every supported shape fits; a plan
- * that needed more than the array would return LA_ERR_WORKSPACE before
- * anything is enqueued.  The first call on a device looks up the array's device
+ * The scratch this path needs (the la_forward workspace of the same problem:
+ * the header, plus at most 36 KB per SM of exchange area) fits the array on
+ * devices of up to 220 SMs; a plan that needed more than the array would
+ * return LA_ERR_WORKSPACE before anything is enqueued.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
  * call before any stream capture.  The address is cached for the life of the
  * process, so this entry point must not be used on a device after
  * cudaDeviceReset.  Every call on a device shares the one array and it keeps
  * the last call's contents: calls that overlap on the GPU (different streams
  * without ordering between them) race and give undefined results.  The
- * kernel only writes the array's status word (on a device-side timeout) and
- * nothing reads it: timeouts of this entry point are not reported, and no
- * clearing operation is enqueued between calls. */
+ * kernel writes the array's status word (on a device-side timeout), which
+ * nothing reads: timeouts of this entry point are not reported.  Its
+ * synchronisation words (a launch count and one flag per CTA, zero when the
+ * array is loaded) carry over from call to call, and every launch leaves them
+ * consistent for the next, so no clearing operation is enqueued between
+ * calls. */
 la_status_t la_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
                                int D, int feature_map, float eps, void* stream);
 

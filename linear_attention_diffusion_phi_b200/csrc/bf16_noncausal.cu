@@ -37,7 +37,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "bf16_common.cuh"
 #include "la_internal.h"
@@ -537,13 +539,45 @@ struct CfgT {
   static constexpr int kPhiWarps = 8;
   static constexpr int kCombWarp0 = 2 + kPhiWarps;
   static constexpr int kThreads = 32 * (kCombWarp0 + 8);
+  static constexpr int kMaxClusters = 4;                   // clusters per head
 };
 
-template <int FMAP>
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// 16 bytes from global memory, cached in L2 only (written by another SM in
+// this launch).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// XC: a head may span several clusters (the exchange through L2 is compiled
+// in only then).
+template <int FMAP, bool XC>
 __global__ void __launch_bounds__(CfgT::kThreads, 1)
     fused_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                   int* status, int N, int tiles, float eps) {
+                   int* status, uint32_t* sync, uint8_t* xchg, int N, int tiles, float eps) {
   using C = CfgT;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -564,12 +598,16 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ int comb_flag, ep_flag;
 
+  // A head is served by P CTAs (blockIdx.x), NC clusters of S CTAs.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = static_cast<int>(gridDim.x);
+  const int P = static_cast<int>(gridDim.x);
+  const int S = static_cast<int>(cluster_nctarank());
+  const int NC = XC ? P / S : 1;
   const int rank = static_cast<int>(cluster_ctarank());
+  const int cl = static_cast<int>(blockIdx.x) / S;   // this CTA's cluster within the head
   const int bh = blockIdx.y;
-  const int tile0 = rank * tiles / S;
-  const int T = (rank + 1) * tiles / S - tile0;
+  const int tile0 = static_cast<int>(blockIdx.x) * tiles / P;
+  const int T = (static_cast<int>(blockIdx.x) + 1) * tiles / P - tile0;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* blob = smem;
   uint8_t* recv = blob + C::kBlobBytes;
@@ -663,6 +701,9 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   };
   pdl_wait();
   pdl_launch_dependents();
+  // Launch count of the exchange between clusters: stable until every CTA of
+  // this launch has finished (the last one to finish advances it).
+  const uint32_t gen = NC > 1 ? ld_relaxed_gpu(&sync[0]) : 0u;
   cluster_arrive_relaxed();
   if (warp == 0 && lane == 0) issue(min(C::kRing1, 2 * T));
   cluster_wait();
@@ -906,15 +947,92 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
         }
         *reinterpret_cast<uint4*>(blob + off_img) = pack8(acc);
       }
+      if (XC && NC > 1) {
+        // (3b) the head spans NC clusters: publish these rows (this cluster's
+        // sums) in the exchange area, wait for the CTAs of the same rank in
+        // the other clusters to publish theirs, and sum the NC copies in
+        // ascending cluster order (every cluster gets the same bits).
+        uint8_t* mine = xchg + (static_cast<size_t>(bh) * NC + cl) * C::kBlobBytes;
+        named_bar_sync(3, 256);
+        for (int js = ct; js < 2 * rows * 8; js += 256) {
+          const int a = js / (rows * 8), rem = js % (rows * 8);
+          const uint32_t off = a * C::kBlobAtomBytes + (n0 + rem / 8) * 128 + (rem % 8) * 16;
+          *reinterpret_cast<uint4*>(mine + off) = *reinterpret_cast<const uint4*>(blob + off);
+        }
+        __threadfence();
+        named_bar_sync(3, 256);
+        uint32_t* flags = sync + 2;
+        if (leader) st_release_gpu(&flags[bh * P + blockIdx.x], gen + 1);
+        if (ct < 32) {
+          int g = 1;
+          if (lane < NC && lane != cl) {
+            const uint32_t* f = &flags[bh * P + lane * S + rank];
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(f) < gen + 1) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_error(status, kDeviceTimeout);
+                g = 0;
+                break;
+              }
+            }
+          }
+          g = __all_sync(0xffffffffu, g);
+          if (leader && !g) comb_flag = 1;
+        }
+        named_bar_sync(3, 256);
+        if (comb_flag == 0) {
+          const uint8_t* base = xchg + static_cast<size_t>(bh) * NC * C::kBlobBytes;
+          for (int js0 = ct; js0 < 2 * rows * 8; js0 += 256 * 4) {
+            uint4 w[4][C::kMaxClusters];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int js = js0 + 256 * e;
+              if (js < 2 * rows * 8) {
+                const int a = js / (rows * 8), rem = js % (rows * 8);
+                const uint32_t off = a * C::kBlobAtomBytes + (n0 + rem / 8) * 128 + (rem % 8) * 16;
+#pragma unroll
+                for (int c = 0; c < C::kMaxClusters; ++c)
+                  if (c < NC)
+                    w[e][c] = c == cl ? *reinterpret_cast<const uint4*>(blob + off)
+                                      : ld_cg_v4(base + static_cast<size_t>(c) * C::kBlobBytes + off);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int js = js0 + 256 * e;
+              if (js < 2 * rows * 8) {
+                const int a = js / (rows * 8), rem = js % (rows * 8);
+                const uint32_t off = a * C::kBlobAtomBytes + (n0 + rem / 8) * 128 + (rem % 8) * 16;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+                for (int c = 0; c < C::kMaxClusters; ++c)
+                  if (c < NC) {
+                    const uint32_t wv[4] = {w[e][c].x, w[e][c].y, w[e][c].z, w[e][c].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+                      acc[2 * i] += x.x;
+                      acc[2 * i + 1] += x.y;
+                    }
+                  }
+                *reinterpret_cast<uint4*>(blob + off) = pack8(acc);
+              }
+            }
+          }
+        }
+      }
       fence_proxy_async_smem();
       named_bar_sync(3, 256);
-      if (ct < 2 * (S - 1)) {
+      if (comb_flag == 0 && ct < 2 * (S - 1)) {
         const int o = (rank + 1 + (ct >> 1)) % S, a = ct & 1;
         const uint32_t off = a * C::kBlobAtomBytes + n0 * 128;
         bulk_copy_to_cluster(mapa_shared(smem_u32(blob) + off, o), blob + off, static_cast<uint32_t>(rows) * 128u,
                              mapa_shared(smem_u32(&blob_full), o));
       }
       if (leader) mbar_arrive(&blob_full);   // this CTA's own rows are in place
+      ok = comb_flag == 0;
     }
     if (ok) {
       // (4) outputs: each warp its rows' half of the value columns, staged
@@ -964,63 +1082,105 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  if (XC && NC > 1 && threadIdx.x == 0) {
+    // the last CTA of the launch to get here advances the launch count
+    __threadfence();
+    const uint32_t total = gridDim.x * gridDim.y;
+    if (atomicAdd(&sync[1], 1u) == total - 1) {
+      sync[1] = 0;
+      __threadfence();
+      st_release_gpu(&sync[0], gen + 1);
+    }
+  }
   cluster_sync_all();
 }
 
-// Largest cluster size S <= min(8, tiles) for which B*H clusters of `kern`
-// fit on the device at once (one wave), per device and kernel; 1 when none
-// does.
-int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int tiles) {
+// Clusters of `kern` (cluster size s, `smem` bytes, `threads` threads) that
+// can be resident at once on the current device; cached per device, kernel
+// and size.
+int max_active_clusters(const void* kern, uint32_t smem, int threads, int s) {
   static std::mutex mu;
   static const void* key[16];
-  static int cache[64][16][9];
-  static bool have[64][16][9] = {};
+  static int cache[64][16][17];
+  static bool have[64][16][17] = {};
   static int nkeys = 0;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  if (s < 1 || s > 16 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
-    return 1;
+    return 0;
   }
   std::lock_guard<std::mutex> lock(mu);
   int k = 0;
   while (k < nkeys && key[k] != kern) ++k;
   if (k == nkeys) {
-    if (nkeys == 16) return 1;
+    if (nkeys == 16) return 0;
     key[nkeys++] = kern;
   }
-  const int smax = tiles < 8 ? tiles : 8;
-  for (int s = smax; s >= 2; --s) {
-    if (!have[dev][k][s]) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(static_cast<unsigned>(s), 1);
-      cfg.blockDim = dim3(threads);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = static_cast<unsigned>(s);
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int m = 0;
-      if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        m = 0;
-      }
-      cache[dev][k][s] = m;
-      have[dev][k][s] = true;
+  if (!have[dev][k][s]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(s), 1);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int m = 0;
+    if (ensure_smem_attr(kern, smem) != cudaSuccess || cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      m = 0;
     }
-    if (cache[dev][k][s] >= BH) return s;
+    cache[dev][k][s] = m;
+    have[dev][k][s] = true;
   }
+  return cache[dev][k][s];
+}
+
+// D = 64: one cluster per head, the largest size S <= min(8, tiles) for
+// which B*H clusters fit on the device at once (one wave); 1 when none does.
+int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int tiles) {
+  const int smax = tiles < 8 ? tiles : 8;
+  for (int s = smax; s >= 2; --s)
+    if (max_active_clusters(kern, smem, threads, s) >= BH) return s;
   return 1;
 }
 
+// D = 128: P CTAs per head in NC = P / S clusters of S.  One cluster per
+// head (the largest S <= min(8, tiles) whose B*H clusters fit at once) unless
+// that leaves more than half of the SMs idle; then heads are spread over up to
+// four clusters (P <= 16, every CTA of the launch resident at once, since the
+// clusters of a head wait for one another).  The exchange between clusters
+// goes through L2 and costs several microseconds under full memory load, so
+// it only pays where one cluster per head would use few SMs (few heads).
+// Heads that outnumber the SMs run one CTA each, in waves.
+void geometry_t(long long BH, int tiles, int num_sms, int* P_out, int* S_out) {
+  const void* kern = reinterpret_cast<const void*>(fused_t_kernel<0, false>);
+  const int s1 = pick_cluster(kern, CfgT::kSmemBytes, CfgT::kThreads, BH, tiles);
+  *P_out = s1;
+  *S_out = s1;
+  if (BH * s1 * 2 >= num_sms) return;
+  const long long pmax = std::min<long long>(std::min(tiles, 16), num_sms / std::max<long long>(BH, 1));
+  for (long long P = pmax; P > s1; --P) {
+    if (BH * P > kSyncFlags) continue;
+    for (int S = static_cast<int>(std::min<long long>(P, 8)); S >= 1; --S) {
+      if (P % S != 0 || P / S > CfgT::kMaxClusters) continue;
+      if (max_active_clusters(kern, CfgT::kSmemBytes, CfgT::kThreads, S) >= BH * (P / S)) {
+        *P_out = static_cast<int>(P);
+        *S_out = S;
+        return;
+      }
+    }
+  }
+}
+
 template <class C, class Kern>
-cudaError_t launch_fused(const LaunchArgs& a, Kern kern) {
+cudaError_t launch_fused(const LaunchArgs& a, Kern kern, int P, int S, uint32_t* sync, uint8_t* xchg) {
   const Plan& p = *a.p;
   cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
-  const int S = pick_cluster(reinterpret_cast<const void*>(kern), C::kSmemBytes, C::kThreads, p.BH, p.tiles);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(S);
@@ -1029,24 +1189,52 @@ cudaError_t launch_fused(const LaunchArgs& a, Kern kern) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(p.BH));
+  cfg.gridDim = dim3(static_cast<unsigned>(P), static_cast<unsigned>(p.BH));
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = a.stream;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
-  return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
+  if constexpr (std::is_same<C, CfgT>::value)
+    return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, sync, xchg, p.N, p.tiles,
+                              p.eps);
+  else
+    return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
 }
 
 }  // namespace
 
+void noncausal_geometry(Plan* p, size_t* xchg_bytes) {
+  *xchg_bytes = 0;
+  if (p->D == 128) {
+    geometry_t(p->BH, std::max(p->tiles, 1), p->num_sms, &p->ctas_per_head, &p->cluster);
+    const int nc = p->ctas_per_head / p->cluster;
+    if (nc > 1) *xchg_bytes = static_cast<size_t>(p->BH) * nc * CfgT::kBlobBytes;
+  } else {
+    const void* kern = reinterpret_cast<const void*>(fused_kernel<64, 0>);
+    const int s = pick_cluster(kern, Cfg<64>::kSmemBytes, Cfg<64>::kThreads, p->BH, std::max(p->tiles, 1));
+    p->ctas_per_head = s;
+    p->cluster = s;
+  }
+}
+
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
   const Plan& p = *a.p;
-  if (p.F != 0) return cudaErrorNotSupported;
-  if (p.D == 128) return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0>) : launch_fused<CfgT>(a, fused_t_kernel<1>);
+  if (p.F != 0 || p.ctas_per_head < 1 || p.cluster < 1) return cudaErrorNotSupported;
+  uint32_t* sync = reinterpret_cast<uint32_t*>(a.ws + p.off_sync);
+  uint8_t* xchg = reinterpret_cast<uint8_t*>(a.ws + p.off_xchg);
+  const int P = p.ctas_per_head, S = p.cluster;
+  if (p.D == 128) {
+    if (P > S)
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, true>, P, S, sync, xchg);
+    return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false>, P, S, sync, xchg)
+                       : launch_fused<CfgT>(a, fused_t_kernel<1, false>, P, S, sync, xchg);
+  }
   if (p.D == 64)
-    return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>) : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>);
+    return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>, P, S, sync, xchg)
+                       : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>, P, S, sync, xchg);
   return cudaErrorNotSupported;
 }
 

@@ -93,7 +93,7 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
   p->tiles = static_cast<int>(cdiv(N, la::kTileTokens));
   p->num_sms = num_sms > 0 ? num_sms : 148;
   const long long BH = std::max<long long>(p->BH, 1);
-  size_t partial_floats = 0, ksum_floats = 0, final_bytes = 0, final_ksum_bytes = 0, blob_total = 0;
+  size_t partial_floats = 0, ksum_floats = 0, final_bytes = 0, final_ksum_bytes = 0, blob_total = 0, xchg_bytes = 0;
   if (h->dtype == LA_F32) {
     // Enough (head, split, feature-block) blocks for ~2 waves; splits of whole
     // 16-token chunks (non-causal) or >= 64 tokens (causal).
@@ -110,9 +110,11 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
       final_ksum_bytes = static_cast<size_t>(BH) * p->Fe * 4;
     }
   } else if (!causal && F == 0) {
-    // One thread-block cluster per head; the cluster size is chosen at launch
-    // from the device's cluster occupancy.  The combine runs through
-    // distributed shared memory, so only the workspace header is used.
+    // Each head is split over clusters of CTAs chosen from the device's
+    // cluster occupancy; the combine runs through distributed shared memory
+    // inside a cluster and, where a head spans several clusters, through an
+    // exchange area in the workspace.
+    la::noncausal_geometry(p, &xchg_bytes);
   } else if (causal) {
     // Segments of whole 128-token chunks, about one CTA per SM in all; every
     // segment but the last leaves its state sum, [D + 1][D] fp32.
@@ -143,11 +145,13 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
   }
   size_t off = 0;
   p->off_status = off;        off += la::kStatusBytes;
+  p->off_sync = off;          off += la::kSyncBytes;
   p->off_partial = off;       off = align256(off + partial_floats * 4);
   p->off_ksum_partial = off;  off = align256(off + ksum_floats * 4);
   p->off_final = off;         off = align256(off + final_bytes);
   p->off_final_ksum = off;    off = align256(off + final_ksum_bytes);
   p->off_blob = off;          off = align256(off + blob_total);
+  p->off_xchg = off;          off = align256(off + xchg_bytes);
   p->bytes = off;
 }
 
@@ -216,8 +220,9 @@ bool on_current_device(const void* p) {
 
 namespace la {
 
-// Plan of the fused cluster kernel (la_forward_noalloc): the combine runs
-// through distributed shared memory, so the workspace is only the status word.
+// Plan of the fused kernel for la_forward_noalloc: the same geometry as
+// la_forward's (so both give the same bits); the scratch holds the header and
+// the exchange area between the clusters of a head.
 void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int num_sms, Plan* p) {
   memset(p, 0, sizeof(*p));
   p->dtype = LA_BF16;
@@ -226,9 +231,13 @@ void plan_bf16_noncausal(int B, int H, int N, int D, int fmap, float eps, int nu
   p->BH = static_cast<long long>(B) * H;
   p->tiles = static_cast<int>(cdiv(N, la::kTileTokens));
   p->num_sms = num_sms > 0 ? num_sms : 148;
+  size_t xchg_bytes = 0;
+  la::noncausal_geometry(p, &xchg_bytes);
   size_t off = 0;
   p->off_status = off;        off += la::kStatusBytes;
+  p->off_sync = off;          off += la::kSyncBytes;
   p->off_partial = p->off_ksum_partial = p->off_final = p->off_final_ksum = p->off_blob = off;
+  p->off_xchg = off;          off = align256(off + xchg_bytes);
   p->bytes = off;
 }
 

@@ -15,9 +15,14 @@ constexpr int kDeviceTimeout = 6;                            // == LA_ERR_TIMEOU
 
 constexpr int kTileTokens = 128;   // tokens per tensor-core tile (MMA M or K)
 
-// Workspace header: a 256-byte status area, zeroed when the workspace is bound.
+// Workspace header, zeroed by the first call that uses a newly bound
+// workspace: a 256-byte status area, then the synchronisation words of the
+// bf16 non-causal kernel's exchange between clusters (a launch counter, a
+// done counter and one flag per CTA; see bf16_noncausal.cu).
 constexpr size_t kStatusBytes = 256;
-constexpr size_t kHeaderBytes = kStatusBytes;
+constexpr size_t kSyncBytes = 4096;
+constexpr size_t kHeaderBytes = kStatusBytes + kSyncBytes;
+constexpr int kSyncFlags = static_cast<int>(kSyncBytes / 4) - 2;   // CTAs a cross-cluster launch may have
 
 // Everything la_forward decides on the host, shared with la_workspace_bytes.
 struct Plan {
@@ -32,8 +37,10 @@ struct Plan {
   int seg_len;     // tokens per split/segment
   int num_sms;
   int apply_ctas, apply_tps;   // bf16 projected: apply CTAs per head, 128-token tiles each
+  // bf16 non-causal: CTAs per head, made of clusters of `cluster` CTAs
+  int ctas_per_head, cluster;
   // workspace layout (byte offsets from the workspace base, 256-aligned)
-  size_t off_status, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, bytes;
+  size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, off_xchg, bytes;
   size_t blob_bytes;   // bf16 [kv | ksum | 0]^T image per head (projected path)
 };
 
@@ -74,6 +81,10 @@ cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes);
 // f32 CUDA-core path (all modes).
 cudaError_t launch_f32(const LaunchArgs& a);
 // bf16 tensor-core paths.
+// CTAs per head and cluster size of the bf16 non-causal kernel for p's shape
+// on the current device (from its cluster occupancy), and the bytes of the
+// exchange area between the clusters of a head (0 when a head is one cluster).
+void noncausal_geometry(Plan* p, size_t* xchg_bytes);
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a);
 cudaError_t launch_bf16_causal(const LaunchArgs& a);
 cudaError_t launch_bf16_projected(const LaunchArgs& a);

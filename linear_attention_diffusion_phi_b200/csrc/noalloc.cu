@@ -19,9 +19,11 @@ namespace {
 
 constexpr size_t kScratchBytes = LA_NOALLOC_SCRATCH_BYTES;
 
-// Scratch for la_forward_noalloc: the status word of its kernel (written on a
-// device-side timeout, read by nobody).  In host code this name is only a handle for
-// cudaGetSymbolAddress, never a device address.
+// Scratch for la_forward_noalloc, laid out as la_forward's workspace of the
+// same problem: the status word of its kernel (written on a device-side
+// timeout, read by nobody), the synchronisation words of the exchange between
+// clusters (zero at load) and the exchange area.  In host code this name is
+// only a handle for cudaGetSymbolAddress, never a device address.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -169,6 +169,55 @@ def test_bf16_deterministic_and_guard_bands():
     assert torch.all(sentinel[:pad] == -12345.0) and torch.all(sentinel[pad + n:] == -12345.0)
 
 
+HEADER_BYTES = 256 + 4096    # workspace header: status word, synchronisation words
+XCHG_CASES = [dict(B=1, H=2, N=4607), dict(B=1, H=1, N=8192, fmap="relu"), dict(B=3, H=3, N=2100),
+              dict(B=1, H=4, N=65536)]
+
+
+@pytest.mark.parametrize("case", XCHG_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_heads_over_several_clusters(case):
+    """Few heads, long sequences: each head is spread over several thread-block
+    clusters whose partial states meet in an exchange area of the workspace
+    (la_workspace_bytes grows beyond the header by 36 KB per head and
+    cluster).  Every output element against the oracle (sampled rows for the
+    64k sequence), and the same bits over repeated calls and over CUDA-graph
+    replays, which advance the launch count the clusters synchronise on."""
+    import torch
+    case = dict(case)
+    w = Workload("xchg", D=128, seed=71, **case)
+    q, k, v, _ = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps)
+    need = la.la_workspace_bytes(op.handle, w.B, w.H, w.N, 128, 0, 0)
+    assert need > HEADER_BYTES and (need - HEADER_BYTES) % 36864 == 0
+    assert (need - HEADER_BYTES) // 36864 in [w.B * w.H * c for c in (2, 3, 4)]
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = op(qd, kd, vd)
+    first = out.clone()
+    for _ in range(2):
+        assert torch.equal(op(qd, kd, vd, out=out), first)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        op(qd, kd, vd, out=out)
+    for _ in range(5):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
+    del g
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    if w.N <= 8192:
+        assert_parity(first.cpu(), oracle_full(w, q, k, v, None), "bf16")
+    else:
+        rows = np.array([0, 1, 4095, 4096, 20000, 32767, 32768, 50001, w.N - 2, w.N - 1])
+        got = as_float64(first.cpu())[:, :, rows]
+        ref = np.stack([np.stack([ora.brute_force_rows(as_float64(q)[b, h], as_float64(k)[b, h],
+                                                       as_float64(v)[b, h], rows, w.fmap, w.eps, False)
+                                  for h in range(w.H)]) for b in range(w.B)])
+        assert_parity(got, ref, "bf16")
+
+
 def test_bf16_weights_property():
     """N <= D and V = I: output row i is the normalised weight row: entries
     >= 0, rows sum to ~1 under elu+1, and agree with the oracle."""
@@ -447,7 +496,9 @@ def test_overlapping_output_is_refused_before_launch():
         la.LA_ERR_INVALID_ARG
     big = torch.empty(2 * qd.numel() + ws.numel(), dtype=torch.bfloat16, device=dev)
     op2 = la.LinearAttention(torch.bfloat16, "elu", w.eps)
-    assert la.la_set_workspace(op2.handle, big.data_ptr(), 256) == la.LA_OK
+    need = la.la_workspace_bytes(op2.handle, 1, 2, 1000, 128, 0, 0)
+    assert 0 < need <= ws.numel() * ws.element_size()
+    assert la.la_set_workspace(op2.handle, big.data_ptr(), need) == la.LA_OK
     assert la.la_forward(op2.handle, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), big.data_ptr(), *args) == \
         la.LA_ERR_INVALID_ARG
     torch.cuda.synchronize()
