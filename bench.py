@@ -71,14 +71,14 @@ def algorithmic_flops(w):
 
 
 # DRAM traffic per step (dram__bytes_read.sum + dram__bytes_write.sum summed
-# over the step's launches, one ncu --set full capture each; the summaries are
-# in profiles/).  Reported only while the device code (the kernel file and the
+# over the step's launches, from one ncu capture per workload; the summaries
+# and their commands are in profiles/).  Reported only while the device code (the kernel file and the
 # device headers it includes) still hashes to what was captured; else null.
 DEVICE_HEADERS = ("bf16_common.cuh", "sm100.cuh")
 NCU_TRAFFIC = {
-    "flux1024": (89_287_168, ("bf16_noncausal.cu",), "09cb7e3d60d8e95f"),
-    "causal32k": (722_496_256, ("bf16_causal.cu",), "0827122f020f8286"),
-    "proj256": (102_777_344, ("bf16_proj.cu", "bf16_image.cu"), "af511b8a7d19cef5"),
+    "flux1024": (88_776_704, ("bf16_noncausal.cu",), "c0ee3835e613a30f"),
+    "flux2048_cfg": (780_772_096, ("bf16_noncausal.cu",), "c0ee3835e613a30f"),
+    "causal32k": (716_144_384, ("bf16_causal.cu",), "3e37cbf7e846ccac"),
 }
 
 
@@ -102,7 +102,7 @@ def captured_traffic(w):
 def kernels_per_step(w, sms):
     """(description, launches) of the library's kernels for one forward."""
     if w.dtype == "bf16" and not w.F and not w.causal:
-        return "fused_kernel (one cluster launch per step)", 1
+        return "fused_t_kernel (one cluster launch per step)" if w.D == 128 else "fused_kernel (one cluster launch per step)", 1
     if w.dtype == "bf16" and w.F:
         return "proj_state_kernel + proj_combine_kernel + proj_apply_kernel (three launches per step)", 3
     if w.dtype == "bf16" and w.causal:
