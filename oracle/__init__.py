@@ -7,9 +7,14 @@ from .la_oracle import (  # noqa: F401
     brute_force_rows,
     feature_map,
     forward,
+    landmark_count,
+    landmark_head,
+    landmark_positions,
     linear_causal_head,
     linear_noncausal_head,
     phi_elu1,
     phi_relu,
     rows,
+    sigmoid,
+    ttr_forward,
 )

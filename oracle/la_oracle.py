@@ -210,3 +210,82 @@ def rows(q, k, v, b, h, idx, fmap="elu", eps=1e-6, causal=False, W=None):
                             np.asarray(k[b, h], dtype=np.float64),
                             np.asarray(v[b, h], dtype=np.float64),
                             list(idx), fmap, eps, causal, _head_W(W, h))
+
+
+# --------------------------------------------------------------------------
+# The TTR student layer (page "Flux2TTRTrainer", "How the distillation works"):
+# a linear-time kernel branch (the grouped form above) and a small
+# exact-softmax branch over "landmark" tokens, blended by a bounded weight.
+# The page names the landmark knobs (fraction, min, max; "Inputs worth
+# setting") but gives neither the selection rule nor the blend form.
+# Readings taken here:
+#   * L landmarks, evenly spaced over the sequence: token floor(l N / L) for
+#     l = 0..L-1, with L = clamp(round(fraction N), min, max), then clamped to
+#     [1, N] (round half up);
+#   * the landmark branch is exact softmax attention of every query over the
+#     landmark keys and values, scores q_i . k_j / sqrt(D) (the scale of the
+#     attention the layer replaces), no feature map and no projection;
+#   * the bounded weight is alpha_h = sigmoid(g_h) for a per-head logit g_h,
+#     out = alpha_h * landmark branch + (1 - alpha_h) * kernel branch;
+#   * non-causal only (the layer replaces Flux's bidirectional attention).
+# --------------------------------------------------------------------------
+
+def landmark_count(n, fraction, lo, hi):
+    """Number of landmarks: round(fraction * n) clamped to [lo, hi], then to [1, n]."""
+    want = int(np.floor(fraction * n + 0.5))
+    return max(1, min(n, max(lo, min(hi, want))))
+
+
+def landmark_positions(n, count):
+    """Token indices of ``count`` evenly spaced landmarks among ``n`` tokens."""
+    return [(l * n) // count for l in range(count)]
+
+
+def sigmoid(g):
+    """1 / (1 + exp(-g)), evaluated without overflow for large |g|."""
+    g = float(g)
+    if g >= 0.0:
+        return 1.0 / (1.0 + np.exp(-g))
+    e = np.exp(g)
+    return e / (1.0 + e)
+
+
+def landmark_head(q, k, v, positions):
+    """Exact softmax attention of every query row over the landmark rows.
+
+    scores s_il = q_i . k_{p_l} / sqrt(D); weights softmax_l(s_il) (per query,
+    over the landmarks); returns weights @ v[positions], [N, Dv] float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kl = np.asarray(k, dtype=np.float64)[positions]
+    vl = np.asarray(v, dtype=np.float64)[positions]
+    s = (q @ kl.T) / np.sqrt(q.shape[1])
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    return (e / e.sum(axis=1, keepdims=True)) @ vl
+
+
+def ttr_forward(q, k, v, gate, n_landmarks, fmap="elu", eps=1e-6, W=None):
+    """The blended layer over all heads; ``gate`` holds one logit per head.
+
+    Returns float64 [B, H, N, Dv]: alpha_h landmark + (1 - alpha_h) kernel.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    _check(q, k, v, fmap, eps)
+    B, H, N, _ = q.shape
+    gate = np.asarray(gate, dtype=np.float64).reshape(-1)
+    if gate.shape[0] != H:
+        raise ValueError("one gate logit per head")
+    if not 1 <= n_landmarks <= N:
+        raise ValueError("n_landmarks must be in [1, N]")
+    pos = landmark_positions(N, n_landmarks)
+    out = np.empty(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            a = sigmoid(gate[h])
+            lin = linear_noncausal_head(q[b, h], k[b, h], v[b, h], fmap, eps, _head_W(W, h))
+            lm = landmark_head(q[b, h], k[b, h], v[b, h], pos)
+            out[b, h] = a * lm + (1.0 - a) * lin
+    return out

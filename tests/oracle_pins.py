@@ -19,6 +19,7 @@ from fractions import Fraction
 import numpy as np
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+SCALAR_KEYS = ("fmap", "eps", "landmarks", "gate0", "gate1")
 
 
 # ---------------------------------------------------------------- fixtures --
@@ -33,7 +34,7 @@ def load_golden(name):
             if not line:
                 continue
             parts = line.split()
-            if parts[0] in ("fmap", "eps"):
+            if parts[0] in SCALAR_KEYS:
                 sections[parts[0]] = parts[1]
                 cur = None
             elif len(parts) == 1 and not _is_number(parts[0]):
@@ -42,7 +43,10 @@ def load_golden(name):
             else:
                 sections[cur].append([float(Fraction(p)) for p in parts])
     out = {"fmap": sections["fmap"], "eps": float(Fraction(sections["eps"]))}
-    for key in ("q", "k", "v", "W", "out_noncausal", "out_causal"):
+    for key in ("landmarks", "gate0", "gate1"):
+        if key in sections:
+            out[key] = sections[key]
+    for key in ("q", "k", "v", "W", "out_noncausal", "out_causal", "out_head0", "out_head1"):
         if key in sections:
             out[key] = np.array(sections[key], dtype=np.float64)
     return out
@@ -317,6 +321,102 @@ def pin_projection_reduction(ora):
     _close(got[0, 0], (w @ v[0, 0]) / (w.sum(axis=1) + 1e-6)[:, None], rtol=1e-12)
 
 
+# ------------------------------------------------------ the TTR layer pins --
+# Page "Flux2TTRTrainer", "How the distillation works": a kernel branch and an
+# exact-softmax branch over landmark tokens blended by a bounded weight; the
+# landmark rule, the softmax scale and the blend form are the readings stated
+# in the oracle (evenly spaced landmarks, q.k/sqrt(D), sigmoid(g) on the
+# landmark branch).
+
+def _gate(tok):
+    return math.log(3.0) if tok == "ln3" else float(Fraction(tok))
+
+
+def pin_ttr_golden(ora):
+    """Hand-derived worked example (tests/golden/ttr_blend_rational.txt): two
+    heads with the same inputs and gates 0 and ln 3 (alpha = 1/2 and 3/4)."""
+    g = load_golden("ttr_blend_rational.txt")
+    q = np.stack([g["q"], g["q"]])[None]
+    k = np.stack([g["k"], g["k"]])[None]
+    v = np.stack([g["v"], g["v"]])[None]
+    gate = [_gate(g["gate0"]), _gate(g["gate1"])]
+    got = ora.ttr_forward(q, k, v, gate, int(g["landmarks"]), g["fmap"], g["eps"])
+    _close(got[0, 0], g["out_head0"], rtol=1e-14, atol=1e-15)
+    _close(got[0, 1], g["out_head1"], rtol=1e-14, atol=1e-15)
+
+
+def pin_landmark_rule(ora):
+    """Evenly spaced landmark tokens and the clamped count, by hand."""
+    assert list(ora.landmark_positions(10, 4)) == [0, 2, 5, 7]
+    assert list(ora.landmark_positions(4, 2)) == [0, 2]
+    assert list(ora.landmark_positions(5, 5)) == [0, 1, 2, 3, 4]
+    assert list(ora.landmark_positions(4608, 128))[:3] == [0, 36, 72]
+    assert ora.landmark_count(4608, 1 / 32, 16, 128) == 128     # 144 capped at the max
+    assert ora.landmark_count(100, 1 / 32, 16, 128) == 16       # 3 raised to the min
+    assert ora.landmark_count(10, 0.5, 16, 128) == 10           # the min capped at N
+    assert ora.landmark_count(1000, 0.1, 16, 128) == 100
+    assert ora.landmark_count(3, 0.0, 0, 5) == 1                # at least one landmark
+    assert ora.landmark_count(30, 0.05, 0, 64) == 2             # 1.5 rounds half up
+
+
+def pin_sigmoid_values(ora):
+    """The bounded weight: sigmoid(0) = 1/2, sigmoid(+-ln 3) = 3/4, 1/4,
+    and finite, in (0, 1) or at its limits, for huge logits."""
+    _close(ora.sigmoid(0.0), 0.5, rtol=0, atol=1e-16)
+    _close(ora.sigmoid(math.log(3.0)), 0.75, rtol=1e-15, atol=0)
+    _close(ora.sigmoid(-math.log(3.0)), 0.25, rtol=1e-15, atol=0)
+    assert ora.sigmoid(800.0) == 1.0 and ora.sigmoid(-800.0) == 0.0
+    for g in (-30.0, -2.5, 0.3, 7.0):
+        assert 0.0 < ora.sigmoid(g) < 1.0
+
+
+def pin_landmark_all_tokens_is_attention(ora):
+    """With every token a landmark the softmax branch is plain scaled
+    dot-product attention: the library routine (default scale 1/sqrt(D))."""
+    import torch
+    rng = _rng(41)
+    for n, d in ((37, 8), (5, 3)):
+        q, k, v = rng.standard_normal((3, n, d))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None])[0].numpy()
+        _close(ora.landmark_head(q, k, v, list(range(n))), ref, rtol=1e-12)
+        pos = ora.landmark_positions(n, n)
+        _close(ora.landmark_head(q, k, v, pos), ref, rtol=1e-12)
+
+
+def pin_landmark_invariances(ora):
+    """Shifting every landmark key by one vector u shifts each query's scores
+    by a constant (q.u / sqrt(D)): the softmax, and so the branch, is
+    unchanged.  Scaling V scales the branch; weights are convex, so every
+    output lies between the smallest and largest landmark value."""
+    rng = _rng(43)
+    q, k, v = rng.standard_normal((3, 40, 6))
+    pos = ora.landmark_positions(40, 7)
+    base = ora.landmark_head(q, k, v, pos)
+    _close(ora.landmark_head(q, k + rng.standard_normal(6), v, pos), base, rtol=1e-11)
+    _close(ora.landmark_head(q, k, 3.0 * v, pos), 3.0 * base, rtol=1e-12)
+    vl = v[pos]
+    assert np.all(base <= vl.max(axis=0) + 1e-12) and np.all(base >= vl.min(axis=0) - 1e-12)
+
+
+def pin_ttr_blend_limits(ora):
+    """A logit far above zero leaves the landmark branch alone, far below it
+    the kernel branch alone; in between every output lies between the two
+    branches (a convex blend)."""
+    rng = _rng(47)
+    q, k, v = rng.standard_normal((3, 2, 3, 50, 8))
+    q, k, v = q[None, 0], k[None, 0], v[None, 0]
+    n_l = 9
+    pos = ora.landmark_positions(50, n_l)
+    lin = ora.forward(q, k, v, "elu", 1e-6)
+    lm = np.stack([ora.landmark_head(q[0, h], k[0, h], v[0, h], pos) for h in range(3)])[None]
+    _close(ora.ttr_forward(q, k, v, [60.0, 60.0, 60.0], n_l, "elu", 1e-6), lm, rtol=1e-12)
+    _close(ora.ttr_forward(q, k, v, [-60.0, -60.0, -60.0], n_l, "elu", 1e-6), lin, rtol=1e-12)
+    mid = ora.ttr_forward(q, k, v, [0.4, -1.3, 2.2], n_l, "elu", 1e-6)
+    lo, hi = np.minimum(lin, lm), np.maximum(lin, lm)
+    assert np.all(mid >= lo - 1e-12) and np.all(mid <= hi + 1e-12)
+
+
 ALL_PINS = [
     pin_feature_maps,
     pin_feature_map_vs_torch,
@@ -330,4 +430,10 @@ ALL_PINS = [
     pin_invariances,
     pin_relu_zero_denominator,
     pin_projection_reduction,
+    pin_ttr_golden,
+    pin_landmark_rule,
+    pin_sigmoid_values,
+    pin_landmark_all_tokens_is_attention,
+    pin_landmark_invariances,
+    pin_ttr_blend_limits,
 ]

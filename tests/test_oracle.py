@@ -46,6 +46,17 @@ MUTANTS = [
     ("projection_after_map", "        x = x @ np.asarray(W, dtype=np.float64)\n    if fmap == \"elu\":\n        return phi_elu1(x)",
      "        pass\n    if fmap == \"elu\":\n        return phi_elu1(x) if W is None else phi_elu1(x) @ np.asarray(W, dtype=np.float64)"),
     ("projection_head_zero", "return W if W.ndim == 2 else W[h]", "return W if W.ndim == 2 else W[0]"),
+    ("ttr_alpha_on_kernel_branch", "out[b, h] = a * lm + (1.0 - a) * lin", "out[b, h] = a * lin + (1.0 - a) * lm"),
+    ("landmark_no_scale", "s = (q @ kl.T) / np.sqrt(q.shape[1])", "s = q @ kl.T"),
+    ("landmark_softmax_over_queries", "s = s - s.max(axis=1, keepdims=True)\n    e = np.exp(s)\n    return (e / e.sum(axis=1, keepdims=True)) @ vl",
+     "s = s - s.max(axis=0, keepdims=True)\n    e = np.exp(s)\n    return (e / e.sum(axis=0, keepdims=True)) @ vl"),
+    ("landmark_positions_shifted", "return [(l * n) // count for l in range(count)]",
+     "return [min(n - 1, (l * n) // count + 1) for l in range(count)]"),
+    ("landmark_count_no_clamp", "return max(1, min(n, max(lo, min(hi, want))))", "return max(1, min(n, want))"),
+    ("landmark_count_rounds_down", "want = int(np.floor(fraction * n + 0.5))", "want = int(np.floor(fraction * n))"),
+    ("sigmoid_wrong_sign", "return 1.0 / (1.0 + np.exp(-g))", "return 1.0 / (1.0 + np.exp(g))"),
+    ("landmark_values_from_keys", "vl = np.asarray(v, dtype=np.float64)[positions]",
+     "vl = np.asarray(k, dtype=np.float64)[positions]"),
 ]
 
 
