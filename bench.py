@@ -339,9 +339,10 @@ def parity_samples(w):
     return [(b, h, sl) for b, h in heads[:2]]
 
 
-def parity_block(w, q, k, v, W, got):
+def parity_block(w, q, k, v, W, got, ttr=None):
     """Error figures of the GPU output `got` against the float64 oracle on
-    the sampled heads / rows (CPU torch tensors of the stored values)."""
+    the sampled heads / rows (CPU torch tensors of the stored values); with
+    `ttr` = (landmark count, logits), against the oracle's TTR layer."""
     from linear_attention_diffusion_phi_b200.inputs import as_float64
     from oracle import la_oracle as ora
     qf, kf, vf, Wf = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
@@ -349,7 +350,10 @@ def parity_block(w, q, k, v, W, got):
     for b, h, rows in parity_samples(w):
         g = as_float64(got[b, h])
         Wh = None if Wf is None else Wf[h:h + 1]
-        if rows is None:
+        if ttr is not None:
+            ref = ora.ttr_forward(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1],
+                                  [ttr[1][h]], ttr[0], w.fmap, w.eps, Wh)[0, 0]
+        elif rows is None:
             ref = ora.forward(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1], w.fmap, w.eps,
                               w.causal, Wh)[0, 0]
         else:
@@ -384,11 +388,14 @@ class Timed:
     shifted along the sequence, so every step reads memory the previous steps
     did not touch), the operator, and CUDA graphs of its steps."""
 
-    def __init__(self, w, dev, rank, graphs=True):
+    def __init__(self, w, dev, rank, graphs=True, ttr=None):
         import torch
         import linear_attention_diffusion_phi_b200 as la
         from linear_attention_diffusion_phi_b200.inputs import make_inputs
         self.w = w
+        # (landmark count, logits): time the TTR layer instead of la_forward
+        self.ttr = ttr
+        self.gate = None if ttr is None else torch.tensor(ttr[1], dtype=torch.float32, device=dev)
         dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.set_bytes = 4 * w.B * w.H * w.N * w.D * (2 if w.dtype == "bf16" else 4)
         self.nsets = max(2, -(-3 * L2_BYTES // self.set_bytes))
@@ -411,7 +418,10 @@ class Timed:
 
     def step(self, i):
         q, k, v, o = self.sets[i % self.nsets]
-        self.op(q, k, v, out=o)
+        if self.ttr is None:
+            self.op(q, k, v, out=o)
+        else:
+            self.op.ttr(q, k, v, self.ttr[0], self.gate, out=o)
 
     def capture(self):
         import torch
@@ -514,7 +524,16 @@ def roofline(w, per_step_s, hbm, tflops, src, sms):
     return roof, launches
 
 
-EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k")
+EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr")
+# The TTR layer on the flux1024 shape: 128 landmarks (the page's knobs at
+# fraction 1/32, min 16, max 128) and one logit per head, spread over [-2, 2].
+TTR_LANDMARKS = (1 / 32, 16, 128)
+
+
+def ttr_params(w):
+    """(landmark count, per-head logits) of the TTR layer on workload w."""
+    import linear_attention_diffusion_phi_b200 as la
+    return la.la_landmark_count(w.N, *TTR_LANDMARKS), [float(x) for x in np.linspace(-2.0, 2.0, w.H)]
 
 
 def main():
@@ -599,9 +618,10 @@ def main():
     extras = []
     if ws == 1 and not args.no_extra and w.name == "flux1024":
         for name in EXTRA_WORKLOADS:
-            x = WORKLOADS[name]
+            ttr = name.endswith("_ttr")
+            x = WORKLOADS[name[:-4] if ttr else name]
             try:
-                tx = Timed(x, dev, rank, graphs=not args.no_graph)
+                tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None)
                 xsteps = max(args.steps, 100)
                 tx.steps_hint = xsteps
                 smp = ClockSampler(local)
@@ -611,13 +631,21 @@ def main():
                 xclk = smp.stop()
                 assert tx.op.sync_status() == la.LA_OK, "device-side error during the timed region"
                 xroof, xl = roofline(x, xms / 1e3 / xsteps, hbm, tflops, src, sms)
+                if ttr:
+                    # two launches; the roofline is the layer's: q, k, v read
+                    # once and out written once (the landmark pass adds a read
+                    # of q and a read and write of out on top)
+                    xl = 2
+                    xroof["kernel"] = "fused_t_kernel + landmark_blend_kernel (two launches per step)"
+                    xroof["traffic"] = None
+                    xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
                 ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
                        "causal": x.causal, "dtype": x.dtype, "steps": xsteps, "ms_per_step": xms / xsteps,
                        "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
                        "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
                        "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
                 if not args.no_parity:
-                    ent["parity"] = parity_block(x, *tx.host, tx.output0())
+                    ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr)
                 tx.close()
                 del tx
             except Exception as e:   # an extra figure never costs the headline line

@@ -146,6 +146,33 @@ la_status_t la_forward_host(la_handle_t handle, const void* q_host, const void* 
  * LA_ERR_CUDA. */
 la_status_t la_sync_status(la_handle_t handle, void* stream);
 
+/* The TTR student layer (page "Flux2TTRTrainer", "How the distillation
+ * works"): the kernel branch of la_forward (non-causal, F = 0 or a projection
+ * bound as for la_forward) fused with an exact-softmax branch over landmark
+ * tokens, blended by a bounded weight.  The page gives neither the landmark
+ * rule nor the blend; this library reads them as: n_landmarks tokens evenly
+ * spaced, token floor(l N / n_landmarks) for l = 0 .. n_landmarks - 1; scores
+ * q_i . k_l / sqrt(D) (the scale of the attention the layer replaces),
+ * softmax over the landmarks per query, weights applied to the landmark value
+ * rows; out = a_h * softmax branch + (1 - a_h) * kernel branch with
+ * a_h = 1 / (1 + exp(-gate[h])), gate a device array of H floats (one logit per
+ * head, 4-byte aligned, sharing no byte with out or the workspace).
+ * Supported: LA_BF16 handles, D = 128, 1 <= n_landmarks <= min(N, 128)
+ * (n_landmarks outside [1, N] gives LA_ERR_INVALID_ARG, above 128
+ * LA_ERR_UNSUPPORTED).  Two launches on `stream`: the kernel branch into out,
+ * then the landmark branch, which reads q, the landmark rows of k and v and
+ * out, and rewrites out blended.  Same workspace, errors and determinism as
+ * la_forward. */
+la_status_t la_forward_ttr(la_handle_t handle, const void* q, const void* k, const void* v, void* out, int B,
+                           int H, int N, int D, int F, int feature_map, float eps, int n_landmarks,
+                           const float* gate, void* stream);
+
+/* Landmark count of the page's knobs (landmark fraction, min, max; page
+ * "Flux2TTRTrainer", "Inputs worth setting"): round(fraction * N) (half up)
+ * clamped to [min_count, max_count], then to [1, N].  0 for invalid arguments
+ * (N < 1, fraction < 0 or NaN, min_count < 0, max_count < 1). */
+int la_landmark_count(int N, float fraction, int min_count, int max_count);
+
 /* Size of the static scratch array behind la_forward_noalloc (8 MiB).  A
  * device holds it from the moment the library's code is loaded on it (at the
  * latest, the first la_forward_noalloc call there) until the process exits. */

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 
 EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
             "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version",
-            "la_forward_noalloc")
+            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count")
 
 
 class LAError(RuntimeError):
@@ -60,11 +60,14 @@ def lib():
     L.la_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
     L.la_sync_status.argtypes = [vp, vp]
     L.la_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
+    L.la_forward_ttr.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]
+    L.la_landmark_count.argtypes = [i32, f32, i32, i32]
+    L.la_landmark_count.restype = i32
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_version.argtypes = []
     for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
-                 "la_forward_host", "la_sync_status", "la_forward_noalloc"):
+                 "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -110,6 +113,15 @@ def la_forward_noalloc(q, k, v, out, B, H, N, D, feature_map, eps, stream):
     """bf16 non-causal forward whose scratch is a static device array inside the
     library, for callers that cannot allocate device memory."""
     return lib().la_forward_noalloc(q, k, v, out, B, H, N, D, feature_map, eps, stream)
+
+
+def la_forward_ttr(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, n_landmarks, gate, stream):
+    """The TTR layer: kernel branch blended with exact softmax over landmarks."""
+    return lib().la_forward_ttr(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, n_landmarks, gate, stream)
+
+
+def la_landmark_count(N, fraction, min_count, max_count):
+    return lib().la_landmark_count(N, fraction, min_count, max_count)
 
 
 def la_sync_status(handle, stream):
@@ -218,6 +230,26 @@ class LinearAttention:
             s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
             check(la_forward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              B, H, N, D, self.F, self.fmap, self.eps, self.causal, s), "la_forward")
+        return out
+
+    def ttr(self, q, k, v, n_landmarks, gate, out=None, stream=None):
+        """The TTR layer (la_forward_ttr): ``gate`` is a float32 CUDA tensor of
+        one logit per head; non-causal operators only."""
+        if self.causal:
+            raise ValueError("the TTR layer is non-causal")
+        if out is None:
+            out = self.torch.empty_like(q)
+        self._check_tensors(q, k, v, out)
+        B, H, N, D = q.shape
+        if gate.dtype != self.torch.float32 or gate.numel() != H or not gate.is_contiguous() \
+                or gate.device != q.device:
+            raise ValueError(f"gate: expected {H} contiguous float32 values on {q.device}")
+        with self.torch.cuda.device(q.device):
+            self._bind_workspace(B, H, N, D, q.device)
+            s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
+            check(la_forward_ttr(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 B, H, N, D, self.F, self.fmap, self.eps, int(n_landmarks), gate.data_ptr(), s),
+                  "la_forward_ttr")
         return out
 
     def sync_status(self, stream=None):

@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libla_phi.so")
 
-SOURCES = ["la_api.cpp", "f32_kernels.cu", "bf16_noncausal.cu", "bf16_causal.cu", "bf16_proj.cu", "bf16_image.cu", "noalloc.cu"]
+SOURCES = ["la_api.cpp", "f32_kernels.cu", "bf16_noncausal.cu", "bf16_causal.cu", "bf16_proj.cu", "bf16_image.cu",
+           "bf16_landmark.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", f"-I{INCLUDE}", f"-I{CSRC}"]

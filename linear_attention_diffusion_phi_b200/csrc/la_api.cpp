@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "la.h"
@@ -346,8 +347,13 @@ la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
   return LA_OK;
 }
 
-la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H, int N,
-                       int D, int F, int fmap, float eps, int causal, void* stream) {
+namespace {
+
+// la_forward, and with `gate` the landmark branch of la_forward_ttr blended
+// into out right after the kernel branch (same stream, same tensor maps).
+la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H,
+                         int N, int D, int F, int fmap, float eps, int causal, void* stream, const void* gate,
+                         int n_landmarks) {
   if (!h) return LA_ERR_INVALID_ARG;
   la_status_t st = check_shape(h, B, H, N, D, F, fmap, eps, causal);
   if (st != LA_OK) return st;
@@ -420,6 +426,7 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
       a.tm_w = &tw;
     }
     err = causal ? la::launch_bf16_causal(a) : (F > 0 ? la::launch_bf16_projected(a) : la::launch_bf16_noncausal(a));
+    if (err == cudaSuccess && gate) err = la::launch_bf16_landmark(a, gate, n_landmarks);
   }
   if (err == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
   if (err != cudaSuccess) {
@@ -427,6 +434,41 @@ la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* 
     return LA_ERR_CUDA;
   }
   return LA_OK;
+}
+
+}  // namespace
+
+la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                       int D, int F, int fmap, float eps, int causal, void* stream) {
+  return forward_impl(h, q, k, v, out, B, H, N, D, F, fmap, eps, causal, stream, nullptr, 0);
+}
+
+int la_landmark_count(int N, float fraction, int min_count, int max_count) {
+  if (N < 1 || !(fraction >= 0.f) || min_count < 0 || max_count < 1) return 0;
+  const double want = std::floor(static_cast<double>(fraction) * N + 0.5);
+  long long n = want > 2e9 ? 2000000000LL : static_cast<long long>(want);
+  n = std::max<long long>(min_count, std::min<long long>(max_count, n));
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(N, n)));
+}
+
+la_status_t la_forward_ttr(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H,
+                           int N, int D, int F, int fmap, float eps, int n_landmarks, const float* gate,
+                           void* stream) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  la_status_t st = check_shape(h, B, H, N, D, F, fmap, eps, 0);
+  if (st != LA_OK) return st;
+  if (h->dtype != LA_BF16 || D != 128) return LA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return LA_OK;
+  if (n_landmarks < 1 || n_landmarks > N) return LA_ERR_INVALID_ARG;
+  if (n_landmarks > 128) return LA_ERR_UNSUPPORTED;
+  if (!gate || (reinterpret_cast<uintptr_t>(gate) & 3u) != 0) return LA_ERR_INVALID_ARG;
+  // out is rewritten by the blend while every CTA reads the gate logits
+  const size_t nb = static_cast<size_t>(B) * H * N * D * 2;
+  if (out && la::overlap(out, nb, gate, static_cast<size_t>(H) * 4)) return LA_ERR_INVALID_ARG;
+  if (h->ws && la::overlap(h->ws, h->ws_bytes, gate, static_cast<size_t>(H) * 4)) return LA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (la::current_sm100(&sms) && !la::on_current_device(gate)) return LA_ERR_INVALID_ARG;
+  return forward_impl(h, q, k, v, out, B, H, N, D, F, fmap, eps, 0, stream, gate, n_landmarks);
 }
 
 la_status_t la_forward_host(la_handle_t h, const void* q_host, const void* k_host, const void* v_host,

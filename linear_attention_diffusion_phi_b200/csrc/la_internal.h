@@ -87,6 +87,9 @@ cudaError_t launch_f32(const LaunchArgs& a);
 void noncausal_geometry(Plan* p, size_t* xchg_bytes);
 cudaError_t launch_bf16_noncausal(const LaunchArgs& a);
 cudaError_t launch_bf16_causal(const LaunchArgs& a);
+// The landmark branch of the TTR layer blended in place into a.out (which
+// holds the kernel branch); gate: device float[H] logits; 1 <= n <= 128.
+cudaError_t launch_bf16_landmark(const LaunchArgs& a, const void* gate, int n_landmarks);
 cudaError_t launch_bf16_projected(const LaunchArgs& a);
 // Sums fp32 partials (kv^T [D][fpart] and ksum [fpart] per (head, split, part))
 // into the apply's bf16 [kv | ksum | 0]^T image, K-major, D + 16 rows.

@@ -216,3 +216,40 @@ def test_binding_checks_tensors_before_calling():
         la.LinearAttention(torch.bfloat16, W=torch.zeros(2, 128, 256, dtype=torch.bfloat16))
     with pytest.raises(ValueError, match="W: expected"):
         la.LinearAttention(torch.float32, W=torch.zeros(256))
+
+
+def test_landmark_count_matches_the_rule():
+    """la_landmark_count (host logic) against the oracle's landmark rule:
+    round(fraction N) half up, clamped to [min, max], then to [1, N]."""
+    from oracle import la_oracle as ora
+    import numpy as np
+    rng = np.random.default_rng(5)
+    cases = [(4608, 1 / 32, 16, 128), (100, 1 / 32, 16, 128), (10, 0.5, 16, 128), (30, 0.05, 0, 64),
+             (3, 0.0, 0, 5), (1, 0.9, 0, 1), (65536, 0.001, 8, 128)]
+    for _ in range(200):
+        cases.append((int(rng.integers(1, 20000)), float(rng.choice([0.25, 0.125, 1 / 32, 0.01, 0.0625])),
+                      int(rng.integers(0, 40)), int(rng.integers(1, 300))))
+    for n, f, lo, hi in cases:
+        assert la.la_landmark_count(n, f, lo, hi) == ora.landmark_count(n, float(np.float32(f)), lo, hi), (n, f, lo, hi)
+    assert la.la_landmark_count(0, 0.1, 1, 8) == 0
+    assert la.la_landmark_count(10, -0.1, 1, 8) == 0
+    assert la.la_landmark_count(10, float("nan"), 1, 8) == 0
+    assert la.la_landmark_count(10, 0.1, -1, 8) == 0
+    assert la.la_landmark_count(10, 0.1, 1, 0) == 0
+
+
+def test_ttr_argument_checks_on_the_host(handles):
+    """la_forward_ttr refuses what it does not support before touching a
+    device: fp32 handles, D != 128, causal-free checks of the landmark count
+    and of the gate pointer."""
+    f = lambda h, D, L, gate: la.la_forward_ttr(h, 0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, D, 0,
+                                               la.LA_PHI_ELU1, 1e-6, L, gate, None)
+    assert f(handles["f32"], 128, 8, 0x3000) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 64, 8, 0x3000) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 128, 0, 0x3000) == la.LA_ERR_INVALID_ARG       # no landmark
+    assert f(handles["bf16"], 128, 257, 0x3000) == la.LA_ERR_INVALID_ARG     # more than N
+    assert f(handles["bf16"], 128, 200, 0x3000) == la.LA_ERR_UNSUPPORTED     # more than 128
+    assert f(handles["bf16"], 128, 8, None) == la.LA_ERR_INVALID_ARG         # no gate
+    assert f(handles["bf16"], 128, 8, 0x3002) == la.LA_ERR_INVALID_ARG       # misaligned gate
+    assert la.la_forward_ttr(handles["bf16"], 0, 0, 0, 0, 0, 2, 256, 128, 0, la.LA_PHI_ELU1, 1e-6, 8,
+                             0x3000, None) == la.LA_OK                       # empty problem

@@ -218,6 +218,62 @@ def test_bf16_heads_over_several_clusters(case):
         assert_parity(got, ref, "bf16")
 
 
+TTR_CASES = [
+    dict(B=1, H=2, N=300, L=16, gates=(0.3, -1.2)),
+    dict(B=1, H=2, N=1000, L=64, fmap="relu", gates=(2.0, -0.5)),
+    dict(B=1, H=3, N=4607, L=128, gates=(0.0, 1.0, -1.0)),
+    dict(B=2, H=2, N=129, L=1, gates=(5.0, -5.0)),
+    dict(B=1, H=2, N=256, L=128, gates=(25.0, -25.0)),     # landmark branch alone, kernel branch alone
+    dict(B=1, H=2, N=77, L=77, gates=(0.7, 0.7)),          # every token a landmark
+    dict(B=1, H=2, N=500, L=40, F=256, gates=(0.2, -0.4)),  # projected kernel branch
+]
+
+
+@pytest.mark.parametrize("case", TTR_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items() if k != "gates"))
+def test_ttr_layer(case):
+    """The TTR layer (kernel branch + exact softmax over evenly spaced
+    landmarks, sigmoid-bounded blend; page "Flux2TTRTrainer", "How the
+    distillation works") against the oracle's float64 definition of it,
+    every output element, and the same bits on a second call."""
+    import torch
+    case = dict(case)
+    gates, n_l = case.pop("gates"), case.pop("L")
+    w = Workload("ttr", D=128, seed=97, **case)
+    q, k, v, W = make_inputs(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps, False, None if W is None else W.to(dev))
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    g = torch.tensor(gates, dtype=torch.float32, device=dev)
+    out = op.ttr(qd, kd, vd, n_l, g)
+    again = op.ttr(qd, kd, vd, n_l, g)
+    torch.cuda.synchronize()
+    assert torch.equal(out, again)
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    ref = ora.ttr_forward(as_float64(q), as_float64(k), as_float64(v), list(gates), n_l, w.fmap, w.eps,
+                          None if W is None else as_float64(W))
+    assert_parity(out.cpu(), ref, "bf16")
+
+
+def test_ttr_flux1024():
+    """The flux1024 shape with 128 landmarks (the count the page's knobs give
+    at fraction 1/32, min 16, max 128) and a logit per head."""
+    import torch
+    w = WORKLOADS["flux1024"]
+    q, k, v, _ = make_inputs(w)
+    n_l = la.la_landmark_count(w.N, 1 / 32, 16, 128)
+    assert n_l == 128
+    gates = np.linspace(-2.0, 2.0, w.H)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps)
+    out = op.ttr(q.to(dev), k.to(dev), v.to(dev), n_l, torch.tensor(gates, dtype=torch.float32, device=dev))
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    ref = ora.ttr_forward(as_float64(q), as_float64(k), as_float64(v), gates, n_l, w.fmap, w.eps)
+    assert_parity(out.cpu(), ref, "bf16", "flux1024 TTR, 128 landmarks (all elements)")
+
+
 def test_bf16_weights_property():
     """N <= D and V = I: output row i is the normalised weight row: entries
     >= 0, rows sum to ~1 under elu+1, and agree with the oracle."""
