@@ -49,13 +49,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const float* __restrict__ gate, int* status, int H, int N, int tiles, int L) {
   extern __shared__ uint8_t smem_raw[];
   // qfull / ofull: a Q tile / a kernel-branch output tile has arrived in slot
-  // s; qempty: the S MMA has read the Q tile; oempty: the blended tile has been
-  // read by its TMA store.  Group g (tiles u with u % 2 == g) owns slot g.
-  __shared__ __align__(8) uint64_t qfull[2], ofull[2], qempty[2], oempty[2];
+  // s; qempty: the S MMA has read the Q tile.  Group g (tiles u with
+  // u % 2 == g) owns slot g; it reloads its output slot itself once the store
+  // of its previous tile has read it.
+  __shared__ __align__(8) uint64_t qfull[2], ofull[2], qempty[2];
   // sfull: S in tensor memory; pready: the weights P written over S;
   // ofull_acc: O in tensor memory; tfree: the group has read O (its tensor
   // memory may take the tile after next).
   __shared__ __align__(8) uint64_t sfull[2], pready[2], ofull_acc[2], tfree[2];
+  // lm_ready: the landmark keys and values are in shared memory
+  __shared__ __align__(8) uint64_t lm_ready;
   __shared__ uint32_t tmem_slot;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -79,12 +82,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&qfull[i], 1);
       mbar_init(&ofull[i], 1);
       mbar_init(&qempty[i], 1);
-      mbar_init(&oempty[i], 1);
       mbar_init(&sfull[i], 1);
       mbar_init(&pready[i], 4);
       mbar_init(&ofull_acc[i], 1);
       mbar_init(&tfree[i], 4);
     }
+    mbar_init(&lm_ready, 8);
     fence_mbarrier_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_out);
@@ -93,74 +96,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  // The kernel branch (the previous launch on the stream) wrote `out`: wait for
-  // it before any global access.
-  pdl_wait();
-  pdl_launch_dependents();
-  // Gather the landmark rows of this head (token floor(l N / L)); rows L..Lp-1
-  // are zero, so their scores are masked below and their values add nothing.
-  {
-    const size_t head = static_cast<size_t>(bh) * N * kD;
-    for (int i = threadIdx.x; i < Lp * 16; i += kThreads) {
-      const int l = i >> 4, c = i & 15;
-      uint4 kk = make_uint4(0u, 0u, 0u, 0u), vv = kk;
-      if (l < L) {
-        const size_t row = head + static_cast<size_t>((static_cast<long long>(l) * N) / L) * kD + c * 8;
-        kk = *reinterpret_cast<const uint4*>(k + row);
-        vv = *reinterpret_cast<const uint4*>(v + row);
-      }
-      *reinterpret_cast<uint4*>(kl + lm_off(l, c)) = kk;
-      *reinterpret_cast<uint4*>(vl + lm_off(l, c)) = vv;
-    }
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // The kernel branch (the previous launch on the stream) wrote `out`: wait for
+  // it before any global access.
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // -------------------------------------------------------- producer
     if (lane == 0) {
       for (int u = 0; u < T; ++u) {
         const int s = u & 1;
-        if (u >= 2 && (!mbar_wait(&qempty[s], ((u >> 1) - 1) & 1, status) ||
-                       !mbar_wait(&oempty[s], ((u >> 1) - 1) & 1, status)))
-          break;
+        if (u >= 2 && !mbar_wait(&qempty[s], ((u >> 1) - 1) & 1, status)) break;
         const int row = (tile0 + u) * kTileTokens;
         mbar_arrive_expect_tx(&qfull[s], kTileBytes);
         tma_load_3d(qs + s * kTileBytes, &tm_q, &qfull[s], 0, row, bh);
         tma_load_3d(qs + s * kTileBytes + kBoxBytes, &tm_q, &qfull[s], 64, row, bh);
-        mbar_arrive_expect_tx(&ofull[s], kTileBytes);
-        tma_load_3d(os + s * kTileBytes, &tm_out, &ofull[s], 0, row, bh);
-        tma_load_3d(os + s * kTileBytes + kBoxBytes, &tm_out, &ofull[s], 64, row, bh);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer
+    // -------------------------------------------------- MMA issuers
+    // Lane 0 issues the S MMAs, lane 1 the O MMAs, each tracking (commit) its
+    // own: an O MMA waits only for its tile's weights, never behind the next
+    // tile's S MMA and what that one waits for.
+    const uint32_t idesc_s = idesc_bf16_f32(128, Lp, 0, 0);       // A = Q (K-major), B = K_L (K-major)
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, kD, 0, 1);   // A = P (tensor memory), B = V_L (MN-major)
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, Lp, 0, 0);   // A = Q (K-major), B = K_L (K-major)
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kD, 0, 1);   // A = P (tensor memory), B = V_L (MN-major)
       const uint64_t kdesc = smem_desc_sw128(smem_u32(kl), 16, 1024);
-      const uint64_t vdesc = smem_desc_sw128(smem_u32(vl), lm_atom, 1024);
-      auto issue_o = [&](int u) {
-        const int g = u & 1;
-        if (!mbar_wait(&pready[g], (u >> 1) & 1, status)) return false;
-        tc_fence_after();
-        const uint32_t p = tmem + g * 256, o = tmem + g * 256 + 128;
-        umma_ts<0>(o, p, vdesc, idesc_o);
-        for (int kk = 1; kk < Lp / 16; ++kk) umma_ts<1>(o, p + 8 * kk, desc_add(vdesc, 2048 * kk), idesc_o);
-        umma_commit(&ofull_acc[g]);
-        return true;
-      };
-      bool ok = true;
+      bool ok = mbar_wait(&lm_ready, 0, status);
       for (int u = 0; u < T && ok; ++u) {
         const int g = u & 1;
         if (!mbar_wait(&qfull[g], (u >> 1) & 1, status) ||
-            (u >= 2 && !mbar_wait(&tfree[g], ((u >> 1) - 1) & 1, status))) {
-          ok = false;
+            (u >= 2 && !mbar_wait(&tfree[g], ((u >> 1) - 1) & 1, status)))
           break;
-        }
         tc_fence_after();
         const uint64_t qdesc = smem_desc_sw128(smem_u32(qs + g * kTileBytes), 16, 1024);
         const uint32_t sacc = tmem + g * 256;
@@ -171,11 +142,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                      desc_add(kdesc, (kk >> 2) * lm_atom + (kk & 3) * 32), idesc_s);
         umma_commit(&qempty[g]);
         umma_commit(&sfull[g]);
-        if (u >= 1) ok = issue_o(u - 1);
       }
-      if (ok && T > 0) issue_o(T - 1);
+    } else if (lane == 1) {
+      const uint64_t vdesc = smem_desc_sw128(smem_u32(vl), lm_atom, 1024);
+      for (int u = 0; u < T; ++u) {
+        const int g = u & 1;
+        if (!mbar_wait(&pready[g], (u >> 1) & 1, status)) break;
+        tc_fence_after();
+        const uint32_t p = tmem + g * 256, o = tmem + g * 256 + 128;
+        umma_ts<0>(o, p, vdesc, idesc_o);
+        for (int kk = 1; kk < Lp / 16; ++kk) umma_ts<1>(o, p + 8 * kk, desc_add(vdesc, 2048 * kk), idesc_o);
+        umma_commit(&ofull_acc[g]);
+      }
     }
   } else {
+    // Gather the landmark rows of this head (token floor(l N / L)) while the
+    // first tiles load; rows L..Lp-1 are zero, so their scores are masked
+    // below and their values add nothing.
+    {
+      // 256 threads, 2048 16-byte chunks of each at most: all of a thread's
+      // loads are issued before its stores, so they overlap
+      const size_t head = static_cast<size_t>(bh) * N * kD;
+      constexpr int kPer = kMaxLandmarks * 16 / (kThreads - 64);
+      uint4 kk[kPer], vv[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x - 64 + j * (kThreads - 64), l = i >> 4, c = i & 15;
+        kk[j] = vv[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (l < L) {
+          const size_t row = head + static_cast<size_t>((static_cast<long long>(l) * N) / L) * kD + c * 8;
+          kk[j] = *reinterpret_cast<const uint4*>(k + row);
+          vv[j] = *reinterpret_cast<const uint4*>(v + row);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x - 64 + j * (kThreads - 64), l = i >> 4, c = i & 15;
+        if (l < Lp) {
+          *reinterpret_cast<uint4*>(kl + lm_off(l, c)) = kk[j];
+          *reinterpret_cast<uint4*>(vl + lm_off(l, c)) = vv[j];
+        }
+      }
+      fence_proxy_async_smem();   // read by the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lm_ready);
+    }
     // -------------------------------------- softmax, blend and store
     const int g = (warp - 2) >> 2;         // group: tiles u with u % 2 == g
     const int q4 = warp & 3;               // tensor-memory lane quarter
@@ -183,41 +194,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = warp == 2 + 4 * g && lane == 0;   // lane 0 of the group's first warp
     const uint32_t lanes = static_cast<uint32_t>(32 * q4) << 16;
     const float a = 1.0f / (1.0f + expf(-gate[bh % H]));
+    auto load_out = [&](int u) {   // the kernel branch's output tile u into slot g
+      const int row = (tile0 + u) * kTileTokens;
+      mbar_arrive_expect_tx(&ofull[g], kTileBytes);
+      tma_load_3d(os + g * kTileBytes, &tm_out, &ofull[g], 0, row, bh);
+      tma_load_3d(os + g * kTileBytes + kBoxBytes, &tm_out, &ofull[g], 64, row, bh);
+    };
+    if (leader && g < T) load_out(g);
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));   // log2(e) / sqrt(D)
     for (int u = g; u < T; u += 2) {
       const int it = u >> 1;
       if (!warp_wait(&sfull[g], it & 1, status)) break;
       tc_fence_after();
       const uint32_t srow = tmem + g * 256 + lanes;
-      // row max over the landmarks (padded columns excluded)
+      // the row of S in two halves of 64 columns (columns from L on are
+      // masked): first its maximum, then the weights exp((s - m) / sqrt(D)),
+      // rounded to bf16; the sum is taken over the rounded weights, so
+      // numerator and denominator see the same ones.  P goes over S in place:
+      // two weights per column.
       float m = -INFINITY;
-      for (int c0 = 0; c0 < Lp; c0 += 32) {
-        float x[32];
-        tmem_ld32(srow + c0, x);
+#pragma unroll
+      for (int h0 = 0; h0 < kMaxLandmarks; h0 += 64) {
+        float x[64];
+        tmem_ld32(srow + h0, *reinterpret_cast<float(*)[32]>(x));
+        tmem_ld32(srow + h0 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c0 + e < L) m = fmaxf(m, x[e]);
+        for (int e = 0; e < 64; ++e)
+          if (h0 + e < L) m = fmaxf(m, x[e]);
       }
-      // weights exp((s - m) / sqrt(D)), rounded to bf16; the sum is taken over
-      // the rounded weights, so numerator and denominator see the same ones
       float sum = 0.f;
-      for (int c0 = 0; c0 < Lp; c0 += 32) {
-        float x[32];
-        tmem_ld32(srow + c0, x);
-        tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = c0 + 2 * e < L ? ex2_approx((x[2 * e] - m) * sl2) : 0.f;
-          const float p1 = c0 + 2 * e + 1 < L ? ex2_approx((x[2 * e + 1] - m) * sl2) : 0.f;
+      for (int h0 = 0; h0 < kMaxLandmarks; h0 += 64) {
+        float x[64];
+        tmem_ld32(srow + h0, *reinterpret_cast<float(*)[32]>(x));
+        tmem_ld32(srow + h0 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+        tmem_wait_ld();
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = h0 + 2 * e;
+          const float p0 = c < L ? ex2_approx((x[2 * e] - m) * sl2) : 0.f;
+          const float p1 = c + 1 < L ? ex2_approx((x[2 * e + 1] - m) * sl2) : 0.f;
           const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
           const float2 f = __bfloat1622float2(b);
           sum += f.x + f.y;
           w[e] = *reinterpret_cast<const uint32_t*>(&b);
         }
-        // P over S in place: two weights per column, column c0 / 2 on
-        tmem_st16(srow + c0 / 2, w);
+        tmem_st32(srow + h0 / 2, w);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -229,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O in four runs of 32 columns, each blended into 4 chunks of the row
       const float scale = a / sum;
       uint8_t* ob = os + g * kTileBytes;
-#pragma unroll
+#pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + g * 256 + 128 + lanes + c0, o);
@@ -263,8 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_3d(&tm_out, ob, 0, row, bh);
         tma_store_3d(&tm_out, ob + kBoxBytes, 64, row, bh);
         bulk_commit_group();
-        bulk_wait_group_read<0>();
-        mbar_arrive(&oempty[g]);
+        if (u + 2 < T) {
+          bulk_wait_group_read<0>();   // the store has read the slot
+          load_out(u + 2);
+        }
       }
     }
     if (leader) bulk_wait_group<0>();
