@@ -14,14 +14,14 @@
 // shared memory in the layout a TMA tile has (row = landmark, 128-byte
 // swizzle): the B operand of  S = Q K_L^T  (K-major) and of  O = P V_L
 // (MN-major).  Per tile: TMA brings the Q tile and the kernel branch's output
-// tile; one thread issues the S MMA (tensor memory, fp32); four warps turn
+// tile; one thread issues the S MMA (tensor memory, fp32); eight warps turn
 // each row of S into softmax weights (row max, exp2, rounded to bf16, summed)
 // and write them back into the same tensor-memory columns as the A operand of
 // the O MMA; the same warps read O, divide by the weight sum, blend with the
 // kernel branch's row in shared memory and TMA-store the tile.  Two such
-// groups of four warps take alternate tiles, each with its own tensor memory
-// (S/P 128 columns, O 128 columns), so one group's softmax overlaps the
-// other's loads and MMAs.
+// groups of eight warps (two per row, one half of the columns each) take
+// alternate tiles, each with its own tensor memory (S/P 128 columns, O 128
+// columns), so one group's softmax overlaps the other's loads and MMAs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -40,7 +40,7 @@ constexpr int kMaxLandmarks = 128;
 constexpr uint32_t kTileBytes = 128u * kD * 2u;                  // one 128-row bf16 tile
 constexpr uint32_t kLmBytes = kMaxLandmarks * kD * 2u;           // landmark keys (or values)
 constexpr uint32_t kSmemBytes = 2 * kLmBytes + 4 * kTileBytes + 1024;
-constexpr int kThreads = 32 * 10;                                // producer, MMA, 2 x 4 softmax warps
+constexpr int kThreads = 32 * 18;                                // producer, MMA, 2 x 8 softmax warps
 constexpr uint32_t kTmemCols = 512;                              // per group: S/P 128, O 128
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // lm_ready: the landmark keys and values are in shared memory
   __shared__ __align__(8) uint64_t lm_ready;
   __shared__ uint32_t tmem_slot;
+  // per group and column half: each row's partial max and weight sum
+  __shared__ float row_max[2][2][128], row_sum[2][2][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -83,11 +85,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ofull[i], 1);
       mbar_init(&qempty[i], 1);
       mbar_init(&sfull[i], 1);
-      mbar_init(&pready[i], 4);
+      mbar_init(&pready[i], 8);
       mbar_init(&ofull_acc[i], 1);
-      mbar_init(&tfree[i], 4);
+      mbar_init(&tfree[i], 8);
     }
-    mbar_init(&lm_ready, 8);
+    mbar_init(&lm_ready, 16);
     fence_mbarrier_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_out);
@@ -150,8 +152,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&pready[g], (u >> 1) & 1, status)) break;
         tc_fence_after();
         const uint32_t p = tmem + g * 256, o = tmem + g * 256 + 128;
+        // P: landmarks 0..63 at columns 0..31, 64..127 at columns 64..95
         umma_ts<0>(o, p, vdesc, idesc_o);
-        for (int kk = 1; kk < Lp / 16; ++kk) umma_ts<1>(o, p + 8 * kk, desc_add(vdesc, 2048 * kk), idesc_o);
+        for (int kk = 1; kk < Lp / 16; ++kk)
+          umma_ts<1>(o, p + 8 * kk + (kk >= 4 ? 32 : 0), desc_add(vdesc, 2048 * kk), idesc_o);
         umma_commit(&ofull_acc[g]);
       }
     }
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // first tiles load; rows L..Lp-1 are zero, so their scores are masked
     // below and their values add nothing.
     {
-      // 256 threads, 2048 16-byte chunks of each at most: all of a thread's
+      // 512 threads, 2048 16-byte chunks of each at most: all of a thread's
       // loads are issued before its stores, so they overlap
       const size_t head = static_cast<size_t>(bh) * N * kD;
       constexpr int kPer = kMaxLandmarks * 16 / (kThreads - 64);
@@ -188,10 +192,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&lm_ready);
     }
     // -------------------------------------- softmax, blend and store
-    const int g = (warp - 2) >> 2;         // group: tiles u with u % 2 == g
+    // Group g (warps 2 + 8 g .. 9 + 8 g) takes tiles u with u % 2 == g; two
+    // warps per tensor-memory lane quarter, each one half of a row's columns.
+    const int g = (warp - 2) >> 3;
+    const int ch = ((warp - 2) >> 2) & 1;  // column half
     const int q4 = warp & 3;               // tensor-memory lane quarter
     const int r = 32 * q4 + lane;          // row of the tile
-    const bool leader = warp == 2 + 4 * g && lane == 0;   // lane 0 of the group's first warp
+    const bool leader = warp == 2 + 8 * g && lane == 0;   // lane 0 of the group's first warp
     const uint32_t lanes = static_cast<uint32_t>(32 * q4) << 16;
     const float a = 1.0f / (1.0f + expf(-gate[bh % H]));
     auto load_out = [&](int u) {   // the kernel branch's output tile u into slot g
@@ -202,38 +209,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if (leader && g < T) load_out(g);
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));   // log2(e) / sqrt(D)
+    const int c_lo = 64 * ch;              // this warp's score columns c_lo .. c_lo + 63
     for (int u = g; u < T; u += 2) {
       const int it = u >> 1;
       if (!warp_wait(&sfull[g], it & 1, status)) break;
       tc_fence_after();
       const uint32_t srow = tmem + g * 256 + lanes;
-      // the row of S in two halves of 64 columns (columns from L on are
-      // masked): first its maximum, then the weights exp((s - m) / sqrt(D)),
-      // rounded to bf16; the sum is taken over the rounded weights, so
-      // numerator and denominator see the same ones.  P goes over S in place:
-      // two weights per column.
+      // Softmax of the row, columns from L on masked: each warp the maximum of
+      // its half, exchanged; then its weights exp((s - m) / sqrt(D)) rounded
+      // to bf16 and their sum, exchanged before the blend (the sum is over the
+      // rounded weights, so numerator and denominator see the same ones).
+      // The weights go over this warp's own scores, two per column: landmarks
+      // 0..63 at columns 0..31, 64..127 at columns 64..95.
       float m = -INFINITY;
 #pragma unroll
-      for (int h0 = 0; h0 < kMaxLandmarks; h0 += 64) {
-        float x[64];
-        tmem_ld32(srow + h0, *reinterpret_cast<float(*)[32]>(x));
-        tmem_ld32(srow + h0 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+      for (int h0 = 0; h0 < 64; h0 += 32) {
+        float x[32];
+        tmem_ld32(srow + c_lo + h0, x);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (h0 + e < L) m = fmaxf(m, x[e]);
+        for (int e = 0; e < 32; ++e)
+          if (c_lo + h0 + e < L) m = fmaxf(m, x[e]);
       }
+      row_max[g][ch][r] = m;
+      named_bar_sync(1 + g, 256);
+      m = fmaxf(m, row_max[g][ch ^ 1][r]);
       float sum = 0.f;
 #pragma unroll
-      for (int h0 = 0; h0 < kMaxLandmarks; h0 += 64) {
-        float x[64];
-        tmem_ld32(srow + h0, *reinterpret_cast<float(*)[32]>(x));
-        tmem_ld32(srow + h0 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+      for (int h0 = 0; h0 < 64; h0 += 32) {
+        float x[32];
+        tmem_ld32(srow + c_lo + h0, x);
         tmem_wait_ld();
-        uint32_t w[32];
+        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = h0 + 2 * e;
+        for (int e = 0; e < 16; ++e) {
+          const int c = c_lo + h0 + 2 * e;
           const float p0 = c < L ? ex2_approx((x[2 * e] - m) * sl2) : 0.f;
           const float p1 = c + 1 < L ? ex2_approx((x[2 * e + 1] - m) * sl2) : 0.f;
           const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
@@ -241,24 +251,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum += f.x + f.y;
           w[e] = *reinterpret_cast<const uint32_t*>(&b);
         }
-        tmem_st32(srow + h0 / 2, w);
+        tmem_st16(srow + c_lo + h0 / 2, w);
       }
+      row_sum[g][ch][r] = sum;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&pready[g]);
-      // O, then the blend with the kernel branch's row
+      // O, then the blend with the kernel branch's row: this warp's half of
+      // the value columns, 32 at a time, each run blended into 4 chunks
       if (!warp_wait(&ofull_acc[g], it & 1, status) || !warp_wait(&ofull[g], it & 1, status)) break;
       tc_fence_after();
-      // O in four runs of 32 columns, each blended into 4 chunks of the row
+      named_bar_sync(1 + g, 256);          // both halves' sums are written
+      sum += row_sum[g][ch ^ 1][r];
       const float scale = a / sum;
       uint8_t* ob = os + g * kTileBytes;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + g * 256 + 128 + lanes + c0, o);
         tmem_wait_ld();
-        if (c0 == kD - 32) {
+        if (c0 == 64 * ch + 32) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tfree[g]);   // S/P and O of this group are read
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      named_bar_sync(1 + g, 128);
+      named_bar_sync(1 + g, 256);
       if (leader) {
         const int row = (tile0 + u) * kTileTokens;
         tma_store_3d(&tm_out, ob, 0, row, bh);
