@@ -573,6 +573,10 @@ __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
 
 // XC: a head may span several clusters (the exchange through L2 is compiled
 // in only then).
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
+
 template <int FMAP, bool XC>
 __global__ void __launch_bounds__(CfgT::kThreads, 1)
     fused_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -580,6 +584,10 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
                    int* status, uint32_t* sync, uint8_t* xchg, int N, int tiles, float eps) {
   using C = CfgT;
   constexpr int D = C::D;
+  // Warps that apply phi to the K tiles: with elu+1 (an exponential per
+  // element) the combine warps, idle in phase 1, join the eight phi warps;
+  // relu is cheap enough for eight.
+  constexpr int kKWarps = FMAP == 0 ? 16 : 8;
   extern __shared__ uint8_t smem_raw[];
   // full: a K or Q tile has arrived (waited on by the phi warps, every phase
   // in order); vfull: a V tile has arrived (MMA issuer); empty: a phase-1
@@ -632,11 +640,11 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     for (int i = 0; i < C::kRing1; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&vfull[i], 1);
-      mbar_init(&empty[i], (i & 1) == 0 ? C::kPhiWarps : 1);
+      mbar_init(&empty[i], (i & 1) == 0 ? kKWarps : 1);
       mbar_init(&qfree[i], C::kPhiWarps);
     }
     for (int i = 0; i < C::kABufs; ++i) {
-      mbar_init(&aready[i], C::kPhiWarps);
+      mbar_init(&aready[i], kKWarps);
       mbar_init(&aempty[i], 1);
     }
     mbar_init(&p1full, 1);
@@ -708,6 +716,61 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   if (warp == 0 && lane == 0) issue(min(C::kRing1, 2 * T));
   cluster_wait();
 
+  // phi on the K tiles into tensor memory, by kKWarps warps (kKWarps / 4 per
+  // lane quarter): warp (qd, kq) takes features 32 qd .. 32 qd + 31 (two
+  // 16-lane halves) of tokens kq * kTok .. kq * kTok + kTok - 1 (16-token blocks).
+  auto k_phase = [&]() {
+    constexpr int kTok = 128 / (kKWarps / 4), kBlocks = kTok / 16;
+    const int qd = warp & 3, kq = (warp - 2) >> 2;
+    const int lm = lane >> 3, lr = lane & 7;
+    for (int t = 0; t < T; ++t) {
+      const int s = (2 * t) % C::kRing1, b = t % C::kABufs;
+      if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
+      const uint32_t base = smem_u32(slot_ptr(s));
+      uint32_t x[2][kBlocks][4];
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < kBlocks; ++tb) {
+          // matrix lm: tokens +8 (lm >> 1), features +8 (lm & 1); row lr
+          const int tok = kTok * kq + 16 * tb + 8 * (lm >> 1) + lr;
+          const int cc = 4 * qd + 2 * fh + (lm & 1);
+          ldsm_x4_trans(base + swz_off(tok, cc), x[fh][tb]);
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);   // the K tile is in registers
+      // key rows past the sequence end must not reach kv or ksum
+      const int valid = min(kTileTokens, N - (tile0 + t) * kTileTokens);
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < kBlocks; ++tb)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            uint32_t w = phi_pair<FMAP>(x[fh][tb][r]);
+            if (valid < kTileTokens) {
+              const int tok = kTok * kq + 16 * tb + 8 * (r >> 1) + 2 * (lane & 3);
+              w &= (tok < valid ? 0x0000FFFFu : 0u) | (tok + 1 < valid ? 0xFFFF0000u : 0u);
+            }
+            x[fh][tb][r] = w;
+          }
+      if (t >= C::kABufs && !warp_wait(&aempty[b], ((t / C::kABufs) - 1) & 1, status)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int fh = 0; fh < 2; ++fh)
+#pragma unroll
+        for (int tb = 0; tb < kBlocks; ++tb)
+          tmem_st_16x128b_x2(tmem + (static_cast<uint32_t>(32 * qd + 16 * fh) << 16) + C::kABuf0 +
+                                 b * C::kABufCols + kTok / 2 * kq + 8 * tb,
+                             x[fh][tb]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[b]);
+    }
+    return true;
+  };
+
   if (warp == 0) {
     if (lane == 0) issue(3 * T);
   } else if (warp == 1) {
@@ -770,61 +833,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     // ------------------------------------------------------- phi warps
     // Tensor-memory lane quarter qd (the warp's accessible lanes); half hf.
     const int qd = warp & 3, hf = (warp - 2) >> 2;
-    bool ok = true;
-    // K tiles: features 32 qd .. 32 qd + 31 (two 16-lane halves), tokens
-    // 64 hf .. 64 hf + 63 (four 16-token blocks)
-    const int lm = lane >> 3, lr = lane & 7;
-    for (int t = 0; t < T && ok; ++t) {
-      const int s = (2 * t) % C::kRing1, b = t % C::kABufs;
-      if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) {
-        ok = false;
-        break;
-      }
-      const uint32_t base = smem_u32(slot_ptr(s));
-      uint32_t x[2][4][4];
-#pragma unroll
-      for (int fh = 0; fh < 2; ++fh)
-#pragma unroll
-        for (int tb = 0; tb < 4; ++tb) {
-          // matrix lm: tokens +8 (lm >> 1), features +8 (lm & 1); row lr
-          const int tok = 64 * hf + 16 * tb + 8 * (lm >> 1) + lr;
-          const int cc = 4 * qd + 2 * fh + (lm & 1);
-          ldsm_x4_trans(base + swz_off(tok, cc), x[fh][tb]);
-        }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);   // the K tile is in registers
-      // key rows past the sequence end must not reach kv or ksum
-      const int valid = min(kTileTokens, N - (tile0 + t) * kTileTokens);
-#pragma unroll
-      for (int fh = 0; fh < 2; ++fh)
-#pragma unroll
-        for (int tb = 0; tb < 4; ++tb)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            uint32_t w = phi_pair<FMAP>(x[fh][tb][r]);
-            if (valid < kTileTokens) {
-              const int tok = 64 * hf + 16 * tb + 8 * (r >> 1) + 2 * (lane & 3);
-              w &= (tok < valid ? 0x0000FFFFu : 0u) | (tok + 1 < valid ? 0xFFFF0000u : 0u);
-            }
-            x[fh][tb][r] = w;
-          }
-      if (t >= C::kABufs && !warp_wait(&aempty[b], ((t / C::kABufs) - 1) & 1, status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int fh = 0; fh < 2; ++fh)
-#pragma unroll
-        for (int tb = 0; tb < 4; ++tb)
-          tmem_st_16x128b_x2(tmem + (static_cast<uint32_t>(32 * qd + 16 * fh) << 16) + C::kABuf0 +
-                                 b * C::kABufCols + 32 * hf + 8 * tb,
-                             x[fh][tb]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&aready[b]);
-    }
+    bool ok = k_phase();
     // Q tiles: token row 32 qd + lane, features 64 hf .. 64 hf + 63
     const int i = 32 * qd + lane;
     const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
@@ -852,7 +861,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&aready[b]);
+      if (lane == 0) mbar_arrive_n(&aready[b], kKWarps / 8);   // counted like the K-tile warps
     }
   } else {
     // ----------------------------------------- combine, then the outputs
@@ -861,13 +870,13 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     const bool leader = ct == 0;
     const int q = warp & 3;
     const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
-    bool got = true;
+    bool got = kKWarps == 16 ? k_phase() : true;
     auto sync_ok = [&](bool mine) {
       if (leader && !mine) comb_flag = 1;
       named_bar_sync(3, 256);
       return comb_flag == 0;
     };
-    if (leader) got = mbar_wait(&p1full, 0, status);
+    if (leader && got) got = mbar_wait(&p1full, 0, status);
     bool ok = sync_ok(got);
     if (ok) {
       // (1) the partial [kv | ksum] (lane = feature, column = value) into
