@@ -63,11 +63,14 @@ __device__ __forceinline__ void load_tile128(void* dst, const CUtensorMap* m, ui
 
 // ====================================================== kernel 1: the state
 
+// K ring of three slots: a slot holds K_t until the K W MMA has read it, then
+// phi(K_t) (written over it by the phi warps) until the state MMAs have read
+// that; V ring of two.
+constexpr int kS1RK = 3;
 constexpr uint32_t kS1OffW = 0;                       // W half: two 64-feature atoms [128 d][64 f]
-constexpr uint32_t kS1OffPhi = kS1OffW + kT32;        // phi(K) half: two atoms [128 t][64 f]
-constexpr uint32_t kS1OffOnes = kS1OffPhi + kT32;     // ones: K-major [16 rows][128 t], 4 KB
+constexpr uint32_t kS1OffOnes = kS1OffW + kT32;       // ones: K-major [16 rows][128 t], 4 KB
 constexpr uint32_t kS1OffK = kS1OffOnes + 4096;
-constexpr uint32_t kS1OffV = kS1OffK + 2 * kT32;
+constexpr uint32_t kS1OffV = kS1OffK + kS1RK * kT32;
 constexpr uint32_t kS1Smem = kS1OffV + 2 * kT32 + 1024;
 constexpr int kS1Threads = 64 + 32 * kPhiWarps;
 constexpr uint32_t kS1ColKv = 256, kS1ColKs = 384;   // kv^T (128 columns), ksum (16)
@@ -79,8 +82,10 @@ __global__ void __launch_bounds__(kS1Threads, 1)
                       float* __restrict__ part_ks, int* status, int N, int H, int w_per_head, int tiles,
                       int tps) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t wfull, kfull[2], kempty[2], vfull[2], vempty[2], kwfull[2], kwfree[2];
-  __shared__ __align__(8) uint64_t phiready, phifree, accfull;
+  __shared__ __align__(8) uint64_t wfull, kfull[kS1RK], kempty[kS1RK], vfull[2], vempty[2], kwfull[2], kwfree[2];
+  // phiready[t & 1]: phi(K_t) written; two barriers, as phi may run one tile
+  // ahead of the state MMAs that wait for it
+  __shared__ __align__(8) uint64_t phiready[2], accfull;
   __shared__ uint32_t tmem_slot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, bh = blockIdx.y, fh = blockIdx.z, nsplit = gridDim.x;
@@ -88,21 +93,23 @@ __global__ void __launch_bounds__(kS1Threads, 1)
   const int T = min(tiles, tile0 + tps) - tile0;   // >= 1
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wsm = smem + kS1OffW;
-  uint8_t* phik = smem + kS1OffPhi;
   uint8_t* ones = smem + kS1OffOnes;
+  auto k_slot = [&](int t) { return smem + kS1OffK + (t % kS1RK) * kT32; };
 
   if (threadIdx.x == 0) {
     mbar_init(&wfull, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kS1RK; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&vfull[i], 1);
       mbar_init(&vempty[i], 1);
       mbar_init(&kwfull[i], 1);
       mbar_init(&kwfree[i], kPhiWarps);
     }
-    mbar_init(&phiready, kPhiWarps);
-    mbar_init(&phifree, 1);
+    mbar_init(&phiready[0], kPhiWarps);
+    mbar_init(&phiready[1], kPhiWarps);
     mbar_init(&accfull, 1);
     fence_mbarrier_init();
     prefetch_tmap(&tm_k);
@@ -133,11 +140,10 @@ __global__ void __launch_bounds__(kS1Threads, 1)
       tma_load_3d(wsm, &tm_w, &wfull, fh * kFH, 0, wz);
       tma_load_3d(wsm + kBoxBytes, &tm_w, &wfull, fh * kFH + 64, 0, wz);
       for (int t = 0; t < T; ++t) {
-        const int s = t & 1, row = (tile0 + t) * kTileTokens;
-        const uint32_t par = ((t >> 1) - 1) & 1;
-        if (t >= 2 && !mbar_wait(&kempty[s], par, status)) break;
-        load_tile128(smem + kS1OffK + s * kT32, &tm_k, &kfull[s], row, bh);
-        if (t >= 2 && !mbar_wait(&vempty[s], par, status)) break;
+        const int s = t & 1, sk = t % kS1RK, row = (tile0 + t) * kTileTokens;
+        if (t >= kS1RK && !mbar_wait(&kempty[sk], ((t / kS1RK) - 1) & 1, status)) break;
+        load_tile128(k_slot(t), &tm_k, &kfull[sk], row, bh);
+        if (t >= 2 && !mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, status)) break;
         load_tile128(smem + kS1OffV + s * kT32, &tm_v, &vfull[s], row, bh);
       }
     }
@@ -148,13 +154,14 @@ __global__ void __launch_bounds__(kS1Threads, 1)
       constexpr uint32_t id_kv = idesc_bf16_f32(kD, kFH, 1, 1);    // V^T phi(K): both MN-major
       constexpr uint32_t id_ks = idesc_bf16_f32(kFH, 16, 1, 0);    // phi(K)^T 1: A MN-major, B K-major
       const uint64_t wdesc = smem_desc_sw128(smem_u32(wsm), kBoxBytes, 1024);
-      const uint64_t pdesc = smem_desc_sw128(smem_u32(phik), kBoxBytes, 1024);
       const uint64_t odesc = smem_desc_sw128(smem_u32(ones), 16, 1024);
-      // kv^T and ksum of tile u from phi(K) in shared memory
+      // kv^T and ksum of tile u from phi(K_u), in K_u's slot
       auto issue_kv = [&](int u) -> bool {
         const int s = u & 1;
-        if (!mbar_wait(&phiready, u & 1, status) || !mbar_wait(&vfull[s], (u >> 1) & 1, status)) return false;
+        if (!mbar_wait(&phiready[s], (u >> 1) & 1, status) || !mbar_wait(&vfull[s], (u >> 1) & 1, status))
+          return false;
         tc_fence_after();
+        const uint64_t pdesc = smem_desc_sw128(smem_u32(k_slot(u)), kBoxBytes, 1024);
         const uint64_t vdesc = smem_desc_sw128(smem_u32(smem + kS1OffV + s * kT32), kBoxBytes, 1024);
         if (u == 0) {
           umma_ss<0>(tmem + kS1ColKv, vdesc, pdesc, id_kv);
@@ -170,27 +177,26 @@ __global__ void __launch_bounds__(kS1Threads, 1)
                      id_ks);
         }
         umma_commit(&vempty[s]);
-        umma_commit(&phifree);
+        umma_commit(&kempty[u % kS1RK]);
         return true;
       };
       bool ok = mbar_wait(&wfull, 0, status);
       for (int t = 0; t < T && ok; ++t) {
         const int s = t & 1;
         // K W_half for tile t into buffer s, once the phi warps have read its previous use
-        if (!mbar_wait(&kfull[s], (t >> 1) & 1, status) ||
+        if (!mbar_wait(&kfull[t % kS1RK], (t / kS1RK) & 1, status) ||
             (t >= 2 && !mbar_wait(&kwfree[s], ((t >> 1) - 1) & 1, status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t kdesc = smem_desc_sw128(smem_u32(smem + kS1OffK + s * kT32), 16, 1024);
+        const uint64_t kdesc = smem_desc_sw128(smem_u32(k_slot(t)), 16, 1024);
         const uint32_t d = tmem + s * 128;
         umma_ss<0>(d, kdesc, wdesc, id_kw);
 #pragma unroll
         for (int k = 1; k < kD / 16; ++k)
           umma_ss<1>(d, desc_add(kdesc, (k >> 2) * kBoxBytes + (k & 3) * 32), desc_add(wdesc, 2048 * k), id_kw);
-        umma_commit(&kwfull[s]);
-        umma_commit(&kempty[s]);
+        umma_commit(&kwfull[s]);   // also: the K tile has been read, phi may go over it
         // the state MMAs of the previous tile, while phi works on this one
         if (t >= 1 && !issue_kv(t - 1)) {
           ok = false;
@@ -202,14 +208,16 @@ __global__ void __launch_bounds__(kS1Threads, 1)
     }
   } else {
     // ------------------------------------------ phi warps: K W -> phi(K)
-    // Two warps per lane quarter; each takes 64 of the 128 features.
+    // Two warps per lane quarter; each takes 64 of the 128 features.  phi(K_t)
+    // goes over K_t in its slot (the K W MMA has read it once kwfull fires),
+    // so phi of tile t runs while the state MMAs of tile t - 1 read theirs.
     const int qd = warp & 3, hw = (warp - 2) >> 2, r = 32 * qd + lane;
     const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
-    uint8_t* dst = phik + hw * kBoxBytes + r * 128;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int s = t & 1;
-      if (!warp_wait(&kwfull[s], (t >> 1) & 1, status) || (t >= 1 && !warp_wait(&phifree, (t - 1) & 1, status))) {
+      uint8_t* dst = k_slot(t) + hw * kBoxBytes + r * 128;
+      if (!warp_wait(&kwfull[s], (t >> 1) & 1, status)) {
         ok = false;
         break;
       }
@@ -234,7 +242,7 @@ __global__ void __launch_bounds__(kS1Threads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&phiready);
+      if (lane == 0) mbar_arrive(&phiready[s]);
     }
     // read-out: warps 2..5 cover the four lane quarters
     if (ok && warp < 6 && warp_wait(&accfull, 0, status)) {
