@@ -345,27 +345,30 @@ __global__ void __launch_bounds__(kS3Threads, 1)
       constexpr uint32_t id_ap = idesc_bf16_f32(128, kNB, 0, 0);   // phi(Q) [kv | ksum]
       const uint64_t wdesc = smem_desc_sw128(smem_u32(wsm), kBoxBytes, 1024);
       const uint64_t idesc_img = smem_desc_sw128(smem_u32(img), 16, 1024);
-      bool ok = mbar_wait(&wfull, 0, status) && mbar_wait(&imgfull, 0, status);
+      // Q W for feature half h of tile t (use g = 2 t + h of the one Q W
+      // buffer, once the phi warps have read use g - 1)
+      auto issue_qw = [&](int t, int h) -> bool {
+        const int g = 2 * t + h;
+        if (g > 0 && !mbar_wait(&qwfree, (g - 1) & 1, status)) return false;
+        tc_fence_after();
+        const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + kS3OffQ + (t & 1) * kT32), 16, 1024);
+        const uint64_t wh = desc_add(wdesc, h * kT32);
+        umma_ss<0>(tmem, qdesc, wh, id_qw);
+#pragma unroll
+        for (int k = 1; k < kD / 16; ++k)
+          umma_ss<1>(tmem, desc_add(qdesc, (k >> 2) * kBoxBytes + (k & 3) * 32), desc_add(wh, 2048 * k), id_qw);
+        umma_commit(&qwfull);
+        return true;
+      };
+      // Order on the tensor pipe: Q W (t, 1), Q W (t + 1, 0), then O of tile
+      // t, so phi of the next tile's first half runs during O.
+      bool ok = mbar_wait(&wfull, 0, status) && mbar_wait(&imgfull, 0, status) && mbar_wait(&qfull[0], 0, status) &&
+                issue_qw(0, 0);
       for (int t = 0; t < T && ok; ++t) {
         const int s = t & 1;
-        if (!mbar_wait(&qfull[s], (t >> 1) & 1, status)) break;
-        const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + kS3OffQ + s * kT32), 16, 1024);
-        for (int h = 0; h < 2; ++h) {
-          const int g = 2 * t + h;   // use of the Q W buffer
-          if (g > 0 && !mbar_wait(&qwfree, (g - 1) & 1, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t wh = desc_add(wdesc, h * kT32);
-          umma_ss<0>(tmem, qdesc, wh, id_qw);
-#pragma unroll
-          for (int k = 1; k < kD / 16; ++k)
-            umma_ss<1>(tmem, desc_add(qdesc, (k >> 2) * kBoxBytes + (k & 3) * 32), desc_add(wh, 2048 * k), id_qw);
-          umma_commit(&qwfull);
-        }
-        if (!ok) break;
+        if (!issue_qw(t, 1)) break;
         umma_commit(&qempty[s]);
+        if (t + 1 < T && (!mbar_wait(&qfull[(t + 1) & 1], ((t + 1) >> 1) & 1, status) || !issue_qw(t + 1, 0))) break;
         // O = phi(Q) [kv | ksum | 0]: 16 feature steps, A from tensor memory
         if (!mbar_wait(&phiqready, t & 1, status) || (t > 0 && !mbar_wait(&oempty, (t - 1) & 1, status))) break;
         tc_fence_after();
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(kS3Threads, 1)
       bool ok = true;
       for (int h = 0; h < 2; ++h) {
         const int g = 2 * t + h;
-        if (!warp_wait(&qwfull, g & 1, status) || (h == 0 && t > 0 && !warp_wait(&phiqfree, (t - 1) & 1, status))) {
+        if (!warp_wait(&qwfull, g & 1, status)) {
           ok = false;
           break;
         }
@@ -401,6 +404,13 @@ __global__ void __launch_bounds__(kS3Threads, 1)
         uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) w[e] = phi2_f32<FMAP>(v[2 * e], v[2 * e + 1]);
+        // phi of the first half is computed while the previous tile's output
+        // MMAs still read phi(Q); it is stored once they are done
+        if (h == 0 && t > 0 && !warp_wait(&phiqfree, (t - 1) & 1, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         // features 128 h + 64 hw .. : packed columns 64 h + 32 hw ..
         tmem_st32(tmem + kS3ColPhi + 64 * h + 32 * hw + lanes, w);
         tmem_wait_st();
