@@ -76,9 +76,11 @@ def algorithmic_flops(w):
 # device headers it includes) still hashes to what was captured; else null.
 DEVICE_HEADERS = ("bf16_common.cuh", "sm100.cuh")
 NCU_TRAFFIC = {
-    "flux1024": (88_776_704, ("bf16_noncausal.cu",), "c0ee3835e613a30f"),
-    "flux2048_cfg": (780_772_096, ("bf16_noncausal.cu",), "c0ee3835e613a30f"),
+    "flux1024": (88_649_216, ("bf16_noncausal.cu",), "d1510f5b4c6763ac"),
+    "flux2048_cfg": (780_859_648, ("bf16_noncausal.cu",), "d1510f5b4c6763ac"),
     "causal32k": (716_144_384, ("bf16_causal.cu",), "3e37cbf7e846ccac"),
+    "proj256": (99_814_016, ("bf16_proj.cu", "bf16_image.cu"), "4d91d4572082bf07"),
+    "flux1024_ttr": (146_939_456, ("bf16_noncausal.cu", "bf16_landmark.cu"), "ba5a94f6fc141518"),
 }
 
 
@@ -91,8 +93,8 @@ def source_hash(kernel_files):
     return h.hexdigest()[:16]
 
 
-def captured_traffic(w):
-    entry = NCU_TRAFFIC.get(w.name)
+def captured_traffic(w, name=None):
+    entry = NCU_TRAFFIC.get(name or w.name)
     if entry is None:
         return None
     nbytes, kernel_files, digest = entry
@@ -104,7 +106,7 @@ def kernels_per_step(w, sms):
     if w.dtype == "bf16" and not w.F and not w.causal:
         return "fused_t_kernel (one cluster launch per step)" if w.D == 128 else "fused_kernel (one cluster launch per step)", 1
     if w.dtype == "bf16" and w.F:
-        return "proj_state_kernel + proj_combine_kernel + proj_apply_kernel (three launches per step)", 3
+        return "proj_state_kernel + image_combine_kernel + proj_apply_kernel (three launches per step)", 3
     if w.dtype == "bf16" and w.causal:
         tiles = max(1, -(-w.N // 128))
         want = max(1, sms // (w.B * w.H))
@@ -660,7 +662,7 @@ def main():
                     # of q and a read and write of out on top)
                     xl = 2
                     xroof["kernel"] = "fused_t_kernel + landmark_blend_kernel (two launches per step)"
-                    xroof["traffic"] = None
+                    xroof["traffic"] = captured_traffic(x, name)
                     xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
                 ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
                        "causal": x.causal, "dtype": x.dtype, "steps": xsteps, "ms_per_step": xms / xsteps,

@@ -14,7 +14,7 @@
 //                        warps into shared memory (bf16), then
 //                        kv^T += V^T phi(K) (M = D, N = 128) and
 //                        ksum += phi(K)^T 1 (M = 128 features, N = 16).
-//   image_combine_kernel (bf16_split.cu) sums the splits in ascending order
+//   image_combine_kernel (bf16_image.cu) sums the splits in ascending order
 //                        (fp32) into the apply's B operand [kv | ksum | 0]^T,
 //                        bf16, K-major, 128-byte swizzle (144 rows x 256).
 //   proj_apply_kernel    grid (ctas, B H): W_h and the image stay in shared
