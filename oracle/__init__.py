@@ -5,8 +5,10 @@ from .la_oracle import (  # noqa: F401
     brute_force,
     brute_force_head,
     brute_force_rows,
+    e4m3_decode,
     feature_map,
     forward,
+    forward_e4m3,
     landmark_count,
     landmark_head,
     landmark_positions,

@@ -289,3 +289,41 @@ def ttr_forward(q, k, v, gate, n_landmarks, fmap="elu", eps=1e-6, W=None):
             lm = landmark_head(q[b, h], k[b, h], v[b, h], pos)
             out[b, h] = a * lm + (1.0 - a) * lin
     return out
+
+
+# --------------------------------------------------------------------------
+# FP8 storage of Q, K and V (page "FLUXNATION", section "What it does": an
+# FP8 CUDA kernel).  Readings: FP8 is the E4M3 format of the OCP 8-bit
+# floating-point specification in its finite form (sign bit, four exponent
+# bits with bias 7, three mantissa bits; no infinities; exponent 1111 with
+# mantissa 111 is NaN; largest finite value 448), and each tensor carries one
+# fp32 scale, its stored values being scale x code value.  The layer itself is
+# unchanged: it runs on the dequantised tensors.
+# --------------------------------------------------------------------------
+
+def e4m3_decode(codes):
+    """Float64 values of E4M3 codes (uint8 array of any shape).
+
+    Exponent field e and mantissa field m: (1 + m/8) 2^(e-7) for e >= 1,
+    (m/8) 2^-6 for e = 0 (subnormals); the sign bit negates; e = 15 with
+    m = 7 is NaN.
+    """
+    c = np.asarray(codes).astype(np.int64)
+    if np.any((c < 0) | (c > 255)):
+        raise ValueError("E4M3 codes are bytes")
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((c & 0x80) != 0, -mag, mag)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def forward_e4m3(q8, k8, v8, scales, fmap="elu", eps=1e-6):
+    """The non-causal layer on E4M3-stored Q, K, V (uint8 [B, H, N, D] codes).
+
+    ``scales`` = (scale_q, scale_k, scale_v): each tensor is dequantised as
+    scale x e4m3_decode(codes) before ``forward``.  Returns float64.
+    """
+    sq, sk, sv = (float(x) for x in scales)
+    return forward(sq * e4m3_decode(q8), sk * e4m3_decode(k8), sv * e4m3_decode(v8), fmap, eps, causal=False)
+

@@ -417,6 +417,60 @@ def pin_ttr_blend_limits(ora):
     assert np.all(mid >= lo - 1e-12) and np.all(mid <= hi + 1e-12)
 
 
+
+# ------------------------------------------------------- FP8 (E4M3) storage --
+
+def _torch_e4m3(codes):
+    """Values of E4M3 codes by torch's float8_e4m3fn conversion (a library routine)."""
+    import torch
+    c = torch.from_numpy(np.ascontiguousarray(np.asarray(codes, dtype=np.uint8)))
+    return c.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def pin_e4m3_vs_torch(ora):
+    """All 256 codes decode as torch's float8_e4m3fn does (NaN where it has NaN)."""
+    c = np.arange(256, dtype=np.uint8)
+    got, want = ora.e4m3_decode(c), _torch_e4m3(c)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def pin_e4m3_format_facts(ora):
+    """Landmarks of the E4M3 format: 448 the largest finite value, 2^-9 the
+    smallest subnormal, 2^-6 the smallest normal, 1.0 at exponent field 7,
+    signed zeros, NaN only at S.1111.111, magnitudes increasing with the code,
+    and the sign bit negating."""
+    d = ora.e4m3_decode
+    c = np.arange(256, dtype=np.uint8)
+    v = d(c)
+    assert d(np.uint8(0x7E)) == 448.0 and d(np.uint8(0xFE)) == -448.0
+    assert d(np.uint8(0x01)) == 2.0 ** -9 and d(np.uint8(0x07)) == 7 * 2.0 ** -9
+    assert d(np.uint8(0x08)) == 2.0 ** -6 and d(np.uint8(0x38)) == 1.0 and d(np.uint8(0xB8)) == -1.0
+    assert d(np.uint8(0x00)) == 0.0 and np.signbit(d(np.uint8(0x80)))
+    assert list(np.flatnonzero(np.isnan(v))) == [0x7F, 0xFF]
+    assert np.all(np.diff(v[:0x7F]) > 0)
+    assert np.array_equal(v[0x80:0xFF], -v[:0x7F])
+
+
+def pin_e4m3_forward(ora):
+    """The layer on E4M3 storage is the layer on scale x decoded codes (decoded
+    here by the library routine), and V's scale scales the output."""
+    rng = _rng(41)
+    shape = (1, 2, 37, 8)
+    codes = [rng.integers(0, 256, size=shape).astype(np.uint8) for _ in range(3)]
+    for cc in codes:
+        cc[(cc & 0x7F) == 0x7F] = 0x3A   # no NaN codes
+        cc[(cc & 0x78) >= 0x50] &= 0xC7  # keep magnitudes below about 8
+    scales = (0.75, 0.125, 1.5)
+    for fmap in ("elu", "relu"):
+        want = ora.forward(*(s * _torch_e4m3(cc) for s, cc in zip(scales, codes)), fmap, 1e-6)
+        got = ora.forward_e4m3(*codes, scales, fmap, 1e-6)
+        _close(got, want, rtol=1e-12)
+    twice = ora.forward_e4m3(*codes, (0.75, 0.125, 3.0), "elu", 1e-6)
+    _close(twice, 2.0 * ora.forward_e4m3(*codes, scales, "elu", 1e-6), rtol=1e-12)
+
+
 ALL_PINS = [
     pin_feature_maps,
     pin_feature_map_vs_torch,
@@ -436,4 +490,7 @@ ALL_PINS = [
     pin_landmark_all_tokens_is_attention,
     pin_landmark_invariances,
     pin_ttr_blend_limits,
+    pin_e4m3_vs_torch,
+    pin_e4m3_format_facts,
+    pin_e4m3_forward,
 ]

@@ -55,6 +55,13 @@ MUTANTS = [
     ("landmark_count_no_clamp", "return max(1, min(n, max(lo, min(hi, want))))", "return max(1, min(n, want))"),
     ("landmark_count_rounds_down", "want = int(np.floor(fraction * n + 0.5))", "want = int(np.floor(fraction * n))"),
     ("sigmoid_wrong_sign", "return 1.0 / (1.0 + np.exp(-g))", "return 1.0 / (1.0 + np.exp(g))"),
+    ("e4m3_bias_eight", "np.exp2(e - 7.0)", "np.exp2(e - 8.0)"),
+    ("e4m3_no_subnormals", "np.where(e == 0, (m / 8.0) * 2.0 ** -6,", "np.where(e < 0, (m / 8.0) * 2.0 ** -6,"),
+    ("e4m3_subnormal_scale", "(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7"),
+    ("e4m3_sign_ignored", "val = np.where((c & 0x80) != 0, -mag, mag)", "val = mag"),
+    ("e4m3_no_nan", "return np.where((e == 15) & (m == 7), np.nan, val)", "return val"),
+    ("e4m3_scales_swapped", "forward(sq * e4m3_decode(q8), sk * e4m3_decode(k8)", "forward(sk * e4m3_decode(q8), sq * e4m3_decode(k8)"),
+    ("e4m3_value_scale_dropped", "sv * e4m3_decode(v8)", "e4m3_decode(v8)"),
     ("landmark_values_from_keys", "vl = np.asarray(v, dtype=np.float64)[positions]",
      "vl = np.asarray(k, dtype=np.float64)[positions]"),
 ]
