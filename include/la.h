@@ -167,6 +167,26 @@ la_status_t la_forward_ttr(la_handle_t handle, const void* q, const void* k, con
                            int H, int N, int D, int F, int feature_map, float eps, int n_landmarks,
                            const float* gate, void* stream);
 
+/* FP8 storage (page "FLUXNATION", "What it does": an FP8 CUDA kernel): the
+ * non-causal F = 0 forward of la_forward with q, k and v stored as E4M3 codes
+ * and one fp32 scale per tensor; the layer runs on scale_q x q, scale_k x k
+ * and scale_v x v.  The page names FP8 only; this library reads it as the
+ * finite E4M3 of the OCP 8-bit floating-point format (sign, four exponent
+ * bits with bias 7, three mantissa bits; largest value 448; S.1111.111 is NaN
+ * and yields NaN wherever it reaches the output) with per-tensor scales.
+ * q, k, v: device uint8 [B, H, N, D] codes, 16-byte aligned, read only (they
+ * may coincide).  out: device bf16 [B, H, N, D], 16-byte aligned, sharing no
+ * byte with q, k, v or the workspace (else LA_ERR_INVALID_ARG).  Scales
+ * finite and > 0 (else LA_ERR_INVALID_ARG).  Supported: LA_BF16 handles,
+ * D = 128 (else LA_ERR_UNSUPPORTED).  Each dequantised value is rounded to
+ * bf16 before the feature map (exact for power-of-two scales, at most 2^-9
+ * relative otherwise); accumulation is fp32 as for bf16 inputs.  Workspace:
+ * la_workspace_bytes of the same B, H, N, D with F = 0 and causal = 0.
+ * One launch on `stream`; errors and determinism as la_forward. */
+la_status_t la_forward_e4m3(la_handle_t handle, const void* q, const void* k, const void* v, float scale_q,
+                            float scale_k, float scale_v, void* out, int B, int H, int N, int D,
+                            int feature_map, float eps, void* stream);
+
 /* Landmark count of the page's knobs (landmark fraction, min, max; page
  * "Flux2TTRTrainer", "Inputs worth setting"): round(fraction * N) (half up)
  * clamped to [min_count, max_count], then to [1, N].  0 for invalid arguments

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 
 EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
             "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version",
-            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count")
+            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count", "la_forward_e4m3")
 
 
 class LAError(RuntimeError):
@@ -61,13 +61,14 @@ def lib():
     L.la_sync_status.argtypes = [vp, vp]
     L.la_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
     L.la_forward_ttr.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]
+    L.la_forward_e4m3.argtypes = [vp, vp, vp, vp, f32, f32, f32, vp, i32, i32, i32, i32, i32, f32, vp]
     L.la_landmark_count.argtypes = [i32, f32, i32, i32]
     L.la_landmark_count.restype = i32
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_version.argtypes = []
     for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
-                 "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr"):
+                 "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr", "la_forward_e4m3"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -118,6 +119,12 @@ def la_forward_noalloc(q, k, v, out, B, H, N, D, feature_map, eps, stream):
 def la_forward_ttr(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, n_landmarks, gate, stream):
     """The TTR layer: kernel branch blended with exact softmax over landmarks."""
     return lib().la_forward_ttr(handle, q, k, v, out, B, H, N, D, F, feature_map, eps, n_landmarks, gate, stream)
+
+
+def la_forward_e4m3(handle, q, k, v, scale_q, scale_k, scale_v, out, B, H, N, D, feature_map, eps, stream):
+    """Non-causal forward on E4M3-stored q, k, v with one scale per tensor; out bf16."""
+    return lib().la_forward_e4m3(handle, q, k, v, scale_q, scale_k, scale_v, out, B, H, N, D, feature_map, eps,
+                                 stream)
 
 
 def la_landmark_count(N, fraction, min_count, max_count):
@@ -250,6 +257,38 @@ class LinearAttention:
             check(la_forward_ttr(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                  B, H, N, D, self.F, self.fmap, self.eps, int(n_landmarks), gate.data_ptr(), s),
                   "la_forward_ttr")
+        return out
+
+    def e4m3(self, q, k, v, scales, out=None, stream=None):
+        """Forward on E4M3-stored inputs (la_forward_e4m3): ``q``, ``k``, ``v``
+        are uint8 (or float8_e4m3fn) CUDA tensors of codes, ``scales`` the
+        three fp32 scales; ``out`` is bf16.  Non-causal, F = 0, bf16 operators."""
+        if self.causal or self.F:
+            raise ValueError("E4M3 storage: non-causal operators without a projection only")
+        if q.dim() != 4:
+            raise ValueError(f"q: expected [B, H, N, D], got shape {tuple(q.shape)}")
+        codes = []
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            if t.dtype == getattr(self.torch, "float8_e4m3fn", None):
+                t = t.view(self.torch.uint8)
+            if t.dtype != self.torch.uint8:
+                raise ValueError(f"{name}: dtype {t.dtype}, expected uint8 E4M3 codes")
+            if t.shape != q.shape or not t.is_contiguous() or t.device.type != "cuda" or t.device != q.device:
+                raise ValueError(f"{name}: expected a contiguous {tuple(q.shape)} tensor on {q.device}")
+            codes.append(t)
+        if out is None:
+            out = self.torch.empty(q.shape, dtype=self.torch.bfloat16, device=q.device)
+        if out.dtype != self.torch.bfloat16 or out.shape != q.shape or not out.is_contiguous() \
+                or out.device != q.device:
+            raise ValueError(f"out: expected a contiguous bfloat16 {tuple(q.shape)} tensor on {q.device}")
+        sq, sk, sv = (float(x) for x in scales)
+        B, H, N, D = q.shape
+        with self.torch.cuda.device(q.device):
+            self._bind_workspace(B, H, N, D, q.device)
+            s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
+            check(la_forward_e4m3(self.handle, codes[0].data_ptr(), codes[1].data_ptr(), codes[2].data_ptr(),
+                                  sq, sk, sv, out.data_ptr(), B, H, N, D, self.fmap, self.eps, s),
+                  "la_forward_e4m3")
         return out
 
     def sync_status(self, stream=None):

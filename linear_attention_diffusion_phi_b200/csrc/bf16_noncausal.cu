@@ -35,6 +35,7 @@
 // by 16-byte asynchronous remote stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -577,23 +578,54 @@ __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
 
-template <int FMAP, bool XC>
+// 16 E4M3 codes (one 16-byte chunk, lowest feature in the lowest byte) times
+// `scale`, rounded to bf16: features 0..7 into lo, 8..15 into hi.  The codes
+// are widened exactly to f16 by the hardware conversion, the product is
+// formed in fp32.
+__device__ __forceinline__ void e4m3x16_to_bf16(uint4 raw, float scale, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t f16x2;
+      const uint16_t two = static_cast<uint16_t>(w[i] >> (16 * h));
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(two));
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
+      const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+      o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// E8: q, k and v are E4M3 codes (tensor maps of bytes, 128 x 128 boxes) with
+// one scale each; out is bf16 as for bf16 inputs.
+template <int FMAP, bool XC, bool E8>
 __global__ void __launch_bounds__(CfgT::kThreads, 1)
     fused_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                   int* status, uint32_t* sync, uint8_t* xchg, int N, int tiles, float eps) {
+                   int* status, uint32_t* sync, uint8_t* xchg, int N, int tiles, float eps, float sq, float sk,
+                   float sv) {
   using C = CfgT;
   constexpr int D = C::D;
   // Warps that apply phi to the K tiles: with elu+1 (an exponential per
   // element) the combine warps, idle in phase 1, join the eight phi warps;
-  // relu is cheap enough for eight.
-  constexpr int kKWarps = FMAP == 0 ? 16 : 8;
+  // relu is cheap enough for eight.  With E4M3 inputs the combine warps
+  // widen the K and V tiles to bf16 in phase 1 instead.
+  constexpr int kKWarps = FMAP == 0 && !E8 ? 16 : 8;
+  constexpr uint32_t kCodeTileBytes = kTileTokens * C::D;   // one E4M3 tile
   extern __shared__ uint8_t smem_raw[];
   // full: a K or Q tile has arrived (waited on by the phi warps, every phase
   // in order); vfull: a V tile has arrived (MMA issuer); empty: a phase-1
   // slot is free again (a K slot once the phi warps have read it, a V slot
   // once its MMAs are done); qfree: a Q tile has been read by the phi warps.
   __shared__ __align__(8) uint64_t full[C::kRing1], vfull[C::kRing1], empty[C::kRing1], qfree[C::kRing1];
+  // E8: an E4M3 K or V tile has landed in its slot (the widening warps then
+  // rewrite the slot as bf16 and arrive on full or vfull)
+  __shared__ __align__(8) uint64_t landed[C::kRing1];
   // A buffers in tensor memory, used in turn by the T key tiles and then the
   // T query tiles: written by the phi warps (aready), read by the MMAs (aempty).
   __shared__ __align__(8) uint64_t aready[C::kABufs], aempty[C::kABufs];
@@ -642,6 +674,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       mbar_init(&vfull[i], 1);
       mbar_init(&empty[i], (i & 1) == 0 ? kKWarps : 1);
       mbar_init(&qfree[i], C::kPhiWarps);
+      mbar_init(&landed[i], 1);
     }
     for (int i = 0; i < C::kABufs; ++i) {
       mbar_init(&aready[i], kKWarps);
@@ -700,10 +733,18 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       const int tile = p1 ? seq / 2 : u;
       uint64_t* bar = is_v ? &vfull[s] : &full[s];
       uint8_t* dst = slot_ptr(s);
-      mbar_arrive_expect_tx(bar, C::kSlotBytes);
+      if constexpr (E8) {
+        // the codes fill the first 16 KB of the slot; K and V are widened
+        // in place before full / vfull, Q is read as codes by the phi warps
+        if (p1) bar = &landed[s];
+        mbar_arrive_expect_tx(bar, kCodeTileBytes);
+        tma_load_3d(dst, m, bar, 0, (tile0 + tile) * kTileTokens, bh);
+      } else {
+        mbar_arrive_expect_tx(bar, C::kSlotBytes);
 #pragma unroll
-      for (int b = 0; b < C::kBoxes; ++b)
-        tma_load_3d(dst + b * kBoxBytes, m, bar, 64 * b, (tile0 + tile) * kTileTokens, bh);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_3d(dst + b * kBoxBytes, m, bar, 64 * b, (tile0 + tile) * kTileTokens, bh);
+      }
       ++seq;
     }
   };
@@ -842,10 +883,25 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       if (!warp_wait(&full[s], q_full_round(u) & 1, status)) break;
       const uint8_t* src = slot_ptr(s);
       uint4 x[8];
+      if constexpr (E8) {
+        // codes of features 64 hf .. 64 hf + 63: four 16-byte chunks of the
+        // 128-byte row (128-byte swizzle), widened to bf16 times sq
+        uint4 raw[4];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
+        for (int m = 0; m < 4; ++m) {
+          const int c = 4 * hf + m;
+          raw[m] = *reinterpret_cast<const uint4*>(src + i * 128 + ((c ^ (i & 7)) << 4));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
+#pragma unroll
+        for (int m = 0; m < 4; ++m) e4m3x16_to_bf16(raw[m], sq, x[2 * m], x[2 * m + 1]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
+      }
       uint32_t w[32];
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -870,7 +926,43 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     const bool leader = ct == 0;
     const int q = warp & 3;
     const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
-    bool got = kKWarps == 16 ? k_phase() : true;
+    // E8: widen every K and V tile in place (codes times sk or sv, rounded to
+    // bf16, in the layout of a bf16 tile), in the order they were issued.
+    // Every warp meets both barriers of every tile even after a wait has
+    // given up (the output is then undefined and the status word says so).
+    auto widen = [&]() {
+      bool good = true;
+      for (int j = 0; j < 2 * T; ++j) {
+        const int s = j % C::kRing1;
+        uint8_t* slot = slot_ptr(s);
+        good = good && warp_wait(&landed[s], (j / C::kRing1) & 1, status);
+        uint4 raw[4];
+        if (good) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int unit = ct + 256 * r, row = unit >> 3, c = unit & 7;
+            raw[r] = *reinterpret_cast<const uint4*>(slot + row * 128 + ((c ^ (row & 7)) << 4));
+          }
+        }
+        named_bar_sync(3, 256);   // the whole tile is in registers
+        if (good) {
+          const float sc = (j & 1) ? sv : sk;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int unit = ct + 256 * r, row = unit >> 3, c = unit & 7;
+            uint4 lo, hi;
+            e4m3x16_to_bf16(raw[r], sc, lo, hi);
+            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c)) = lo;
+            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c + 1)) = hi;
+          }
+        }
+        fence_proxy_async_smem();   // V tiles feed the tensor core
+        named_bar_sync(3, 256);
+        if (good && leader) mbar_arrive((j & 1) ? &vfull[s] : &full[s]);
+      }
+      return good;
+    };
+    bool got = E8 ? widen() : (kKWarps == 16 ? k_phase() : true);
     auto sync_ok = [&](bool mine) {
       if (leader && !mine) comb_flag = 1;
       named_bar_sync(3, 256);
@@ -1166,7 +1258,7 @@ int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int
 // it only pays where one cluster per head would use few SMs (few heads).
 // Heads that outnumber the SMs run one CTA each, in waves.
 void geometry_t(long long BH, int tiles, int num_sms, int* P_out, int* S_out) {
-  const void* kern = reinterpret_cast<const void*>(fused_t_kernel<0, false>);
+  const void* kern = reinterpret_cast<const void*>(fused_t_kernel<0, false, false>);
   const int s1 = pick_cluster(kern, CfgT::kSmemBytes, CfgT::kThreads, BH, tiles);
   *P_out = s1;
   *S_out = s1;
@@ -1207,7 +1299,7 @@ cudaError_t launch_fused(const LaunchArgs& a, Kern kern, int P, int S, uint32_t*
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
   if constexpr (std::is_same<C, CfgT>::value)
     return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, sync, xchg, p.N, p.tiles,
-                              p.eps);
+                              p.eps, a.scale_q, a.scale_k, a.scale_v);
   else
     return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
 }
@@ -1235,12 +1327,20 @@ cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
   uint8_t* xchg = reinterpret_cast<uint8_t*>(a.ws + p.off_xchg);
   const int P = p.ctas_per_head, S = p.cluster;
   if (p.D == 128) {
+    if (a.e4m3) {
+      if (P > S)
+        return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, true>, P, S, sync, xchg)
+                           : launch_fused<CfgT>(a, fused_t_kernel<1, true, true>, P, S, sync, xchg);
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, true>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, false, true>, P, S, sync, xchg);
+    }
     if (P > S)
-      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true>, P, S, sync, xchg)
-                         : launch_fused<CfgT>(a, fused_t_kernel<1, true>, P, S, sync, xchg);
-    return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false>, P, S, sync, xchg)
-                       : launch_fused<CfgT>(a, fused_t_kernel<1, false>, P, S, sync, xchg);
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, false>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, true, false>, P, S, sync, xchg);
+    return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, false>, P, S, sync, xchg)
+                       : launch_fused<CfgT>(a, fused_t_kernel<1, false, false>, P, S, sync, xchg);
   }
+  if (a.e4m3) return cudaErrorNotSupported;
   if (p.D == 64)
     return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>, P, S, sync, xchg)
                        : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>, P, S, sync, xchg);

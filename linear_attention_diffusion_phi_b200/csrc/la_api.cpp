@@ -192,6 +192,23 @@ bool encode_bf16_3d(CUtensorMap* m, const void* base, long long outer, long long
   return r == CUDA_SUCCESS;
 }
 
+// [outer, rows, cols] tensor of bytes (E4M3 codes), box [1, 128, 128] with
+// the 128-byte swizzle: one box is a whole 128 x 128 tile.
+bool encode_u8_3d(CUtensorMap* m, const void* base, long long outer, long long rows, long long cols,
+                  long long outer_stride_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(outer_stride_elems)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
@@ -350,10 +367,11 @@ la_status_t la_set_workspace(la_handle_t h, void* ptr, size_t bytes) {
 namespace {
 
 // la_forward, and with `gate` the landmark branch of la_forward_ttr blended
-// into out right after the kernel branch (same stream, same tensor maps).
+// into out right after the kernel branch (same stream, same tensor maps);
+// with `scales` (q, k, v scales) the inputs are E4M3 codes (la_forward_e4m3).
 la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H,
                          int N, int D, int F, int fmap, float eps, int causal, void* stream, const void* gate,
-                         int n_landmarks) {
+                         int n_landmarks, const float* scales = nullptr) {
   if (!h) return LA_ERR_INVALID_ARG;
   la_status_t st = check_shape(h, B, H, N, D, F, fmap, eps, causal);
   if (st != LA_OK) return st;
@@ -370,13 +388,14 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   {
     const size_t es = h->dtype == LA_F32 ? 4 : 2;
     const size_t nb = static_cast<size_t>(B) * H * N * D * es;
+    const size_t nin = static_cast<size_t>(B) * H * N * D * (scales ? 1 : es);   // bytes of q, k or v
     const size_t wb = F == 0 ? 0
                       : (h->w_head_stride ? static_cast<size_t>(H - 1) * h->w_head_stride : 0) * es +
                             static_cast<size_t>(D) * F * es;
     const void* ins[3] = {q, k, v};
     for (const void* x : ins) {
-      if (la::overlap(out, nb, x, nb)) return LA_ERR_INVALID_ARG;
-      if (h->ws && la::overlap(h->ws, h->ws_bytes, x, nb)) return LA_ERR_INVALID_ARG;
+      if (la::overlap(out, nb, x, nin)) return LA_ERR_INVALID_ARG;
+      if (h->ws && la::overlap(h->ws, h->ws_bytes, x, nin)) return LA_ERR_INVALID_ARG;
     }
     if (F > 0 && la::overlap(out, nb, h->W, wb)) return LA_ERR_INVALID_ARG;
     if (h->ws && (la::overlap(h->ws, h->ws_bytes, out, nb) || (F > 0 && la::overlap(h->ws, h->ws_bytes, h->W, wb))))
@@ -415,9 +434,16 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
     CUtensorMap tq, tk, tv, to, tw;
     const long long BH = p.BH;
     const long long hs = static_cast<long long>(N) * D;
-    if (!encode_bf16_3d(&tq, q, BH, N, D, hs, 128) || !encode_bf16_3d(&tk, k, BH, N, D, hs, 128) ||
-        !encode_bf16_3d(&tv, v, BH, N, D, hs, 128) || !encode_bf16_3d(&to, out, BH, N, D, hs, 128))
+    if (scales) {
+      if (!encode_u8_3d(&tq, q, BH, N, D, hs) || !encode_u8_3d(&tk, k, BH, N, D, hs) ||
+          !encode_u8_3d(&tv, v, BH, N, D, hs) || !encode_bf16_3d(&to, out, BH, N, D, hs, 128))
+        return LA_ERR_CUDA;
+      a.e4m3 = true;
+      a.scale_q = scales[0]; a.scale_k = scales[1]; a.scale_v = scales[2];
+    } else if (!encode_bf16_3d(&tq, q, BH, N, D, hs, 128) || !encode_bf16_3d(&tk, k, BH, N, D, hs, 128) ||
+               !encode_bf16_3d(&tv, v, BH, N, D, hs, 128) || !encode_bf16_3d(&to, out, BH, N, D, hs, 128)) {
       return LA_ERR_CUDA;
+    }
     a.tm_q = &tq; a.tm_k = &tk; a.tm_v = &tv; a.tm_out = &to;
     if (F > 0) {
       const long long nW = h->w_head_stride ? H : 1;
@@ -441,6 +467,19 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
 la_status_t la_forward(la_handle_t h, const void* q, const void* k, const void* v, void* out, int B, int H, int N,
                        int D, int F, int fmap, float eps, int causal, void* stream) {
   return forward_impl(h, q, k, v, out, B, H, N, D, F, fmap, eps, causal, stream, nullptr, 0);
+}
+
+la_status_t la_forward_e4m3(la_handle_t h, const void* q, const void* k, const void* v, float scale_q,
+                            float scale_k, float scale_v, void* out, int B, int H, int N, int D, int fmap, float eps,
+                            void* stream) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  la_status_t st = check_shape(h, B, H, N, D, 0, fmap, eps, 0);
+  if (st != LA_OK) return st;
+  const float sc[3] = {scale_q, scale_k, scale_v};
+  for (float x : sc)
+    if (!(x > 0.f) || !std::isfinite(x)) return LA_ERR_INVALID_ARG;
+  if (h->dtype != LA_BF16 || D != 128) return LA_ERR_UNSUPPORTED;
+  return forward_impl(h, q, k, v, out, B, H, N, D, 0, fmap, eps, 0, stream, nullptr, 0, sc);
 }
 
 int la_landmark_count(int N, float fraction, int min_count, int max_count) {

@@ -60,6 +60,10 @@ struct LaunchArgs {
   const CUtensorMap* tm_v;
   const CUtensorMap* tm_out;
   const CUtensorMap* tm_w;
+  // q, k and v stored as E4M3 codes (tm_q, tm_k, tm_v are then maps of
+  // bytes), dequantised as scale x code value; out stays bf16
+  bool e4m3;
+  float scale_q, scale_k, scale_v;
 };
 
 // Host helpers defined in la_api.cpp for other host translation units.

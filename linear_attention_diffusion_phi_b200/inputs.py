@@ -87,3 +87,33 @@ def as_float64(t):
         return None
     import torch
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+def e4m3_scale(a):
+    """Power-of-two scale that keeps the largest |a| / scale at or below 448,
+    the largest finite E4M3 value (1.0 for an all-zero array)."""
+    amax = float(np.abs(a).max()) if a.size else 0.0
+    if amax == 0.0:
+        return 1.0
+    return float(2.0 ** np.ceil(np.log2(amax / 448.0)))
+
+
+def make_e4m3_inputs(w: Workload, seed=None):
+    """E4M3 storage of the workload's q, k, v: (q8, k8, v8, scales).
+
+    The values are drawn as for ``make_inputs``, divided by a per-tensor
+    power-of-two scale (``e4m3_scale``) and rounded to the nearest code by
+    torch's float8_e4m3fn conversion; q8, k8, v8 are uint8 CPU tensors of the
+    codes and ``scales`` the three scales, so that the stored tensors are
+    scale x code value.
+    """
+    import torch
+    q, k, v, _ = _draw(w, seed)
+    codes, scales = [], []
+    for a in (q, k, v):
+        s = e4m3_scale(a)
+        t = torch.from_numpy(np.ascontiguousarray(a / np.float32(s)))
+        codes.append(t.to(torch.float8_e4m3fn).view(torch.uint8).contiguous())
+        scales.append(s)
+    return codes[0], codes[1], codes[2], tuple(scales)
+

@@ -253,3 +253,19 @@ def test_ttr_argument_checks_on_the_host(handles):
     assert f(handles["bf16"], 128, 8, 0x3002) == la.LA_ERR_INVALID_ARG       # misaligned gate
     assert la.la_forward_ttr(handles["bf16"], 0, 0, 0, 0, 0, 2, 256, 128, 0, la.LA_PHI_ELU1, 1e-6, 8,
                              0x3000, None) == la.LA_OK                       # empty problem
+
+
+def test_e4m3_argument_checks_on_the_host(handles):
+    """la_forward_e4m3 refuses what it does not support before touching a
+    device: scales that are not finite and positive, fp32 handles, D != 128,
+    bad shapes; an empty problem is a no-op."""
+    nan, inf = float("nan"), float("inf")
+    f = lambda h, D, sq, sk, sv, fmap=la.LA_PHI_ELU1: la.la_forward_e4m3(
+        h, 0x1000, 0x1000, 0x1000, sq, sk, sv, 0x2000, 1, 2, 256, D, fmap, 1e-6, None)
+    for bad in ((0.0, 1.0, 1.0), (1.0, -1.0, 1.0), (1.0, 1.0, nan), (inf, 1.0, 1.0)):
+        assert f(handles["bf16"], 128, *bad) == la.LA_ERR_INVALID_ARG, bad
+    assert f(handles["f32"], 128, 1.0, 1.0, 1.0) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 64, 1.0, 1.0, 1.0) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 128, 1.0, 1.0, 1.0, fmap=7) == la.LA_ERR_INVALID_ARG
+    assert la.la_forward_e4m3(handles["bf16"], 0, 0, 0, 1.0, 1.0, 1.0, 0, 0, 2, 256, 128, la.LA_PHI_ELU1,
+                              1e-6, None) == la.LA_OK                        # empty problem

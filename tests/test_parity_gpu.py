@@ -10,7 +10,7 @@ import pytest
 
 import linear_attention_diffusion_phi_b200 as la
 from linear_attention_diffusion_phi_b200 import build as la_build
-from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, Workload, as_float64, make_inputs
+from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, Workload, as_float64, make_e4m3_inputs, make_inputs
 from oracle import la_oracle as ora
 
 pytestmark = pytest.mark.gpu
@@ -592,3 +592,68 @@ def test_pointer_not_on_current_device_is_refused():
     assert torch.all(out == 0)
     assert torch.equal(op(qd, kd, vd), ref)
     op.close()
+
+
+# ------------------------------------------------ E4M3 storage of q, k and v --
+
+E8_CASES = [
+    dict(B=1, H=2, N=1, fmap="elu"),
+    dict(B=1, H=3, N=100, fmap="relu"),
+    dict(B=2, H=2, N=128, fmap="elu"),
+    dict(B=1, H=4, N=1000, fmap="elu"),
+    dict(B=2, H=3, N=333, fmap="relu"),
+    dict(B=1, H=1, N=20000, fmap="elu"),    # one head over several clusters
+    dict(B=1, H=2, N=9000, fmap="relu"),    # few heads, several clusters each
+    dict(B=3, H=40, N=300, fmap="elu"),     # more heads than fit at once
+]
+
+
+def run_e4m3(w, q8, k8, v8, scales, runs=1):
+    import torch
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.bfloat16, w.fmap, w.eps, False)
+    qd, kd, vd = q8.to(dev), k8.to(dev), v8.to(dev)
+    outs = [op.e4m3(qd, kd, vd, scales).cpu() for _ in range(runs)]
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    return outs if runs > 1 else outs[0]
+
+
+def check_e4m3(w, label=None):
+    q8, k8, v8, scales = make_e4m3_inputs(w)
+    got = run_e4m3(w, q8, k8, v8, scales)
+    ref = ora.forward_e4m3(q8.numpy(), k8.numpy(), v8.numpy(), scales, w.fmap, w.eps)
+    return assert_parity(got, ref, "bf16", label)
+
+
+@pytest.mark.parametrize("case", E8_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_e4m3_shapes(case):
+    w = Workload("e4m3_case", case["B"], case["H"], case["N"], 128, fmap=case["fmap"], seed=2100 + case["N"])
+    check_e4m3(w)
+
+
+def test_flux1024_e4m3_full():
+    check_e4m3(WORKLOADS["flux1024"], "flux1024_e4m3 (all elements)")
+
+
+def test_flux2048_cfg_e4m3_full():
+    check_e4m3(WORKLOADS["flux2048_cfg"], "flux2048_cfg_e4m3 (all elements)")
+
+
+def test_e4m3_equals_bf16_path_on_dequantised_values():
+    """With power-of-two scales every dequantised value is a bf16 number, and
+    the E4M3 path widens it exactly before the same arithmetic: its output is
+    bitwise the bf16 path's output on those bf16 tensors; repeated calls give
+    the same bits."""
+    import torch
+    for fmap, N in (("elu", 4608), ("relu", 777), ("elu", 20000)):
+        w = WORKLOADS["flux1024"].with_(H=4 if N < 20000 else 1, N=N, fmap=fmap)
+        q8, k8, v8, scales = make_e4m3_inputs(w, seed=77 + N)
+        got = run_e4m3(w, q8, k8, v8, scales, runs=2)
+        assert torch.equal(got[0].view(torch.int16), got[1].view(torch.int16))
+        deq = [torch.from_numpy(s * ora.e4m3_decode(c.numpy())).to(torch.bfloat16) for s, c in zip(scales, (q8, k8, v8))]
+        for d, s, c in zip(deq, scales, (q8, k8, v8)):   # exact in bf16
+            assert np.array_equal(as_float64(d), s * ora.e4m3_decode(c.numpy()))
+        ref = run_gpu(w.with_(dtype="bf16"), *deq)
+        assert torch.equal(got[0].view(torch.int16), ref.view(torch.int16)), (fmap, N)
