@@ -56,9 +56,11 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def algorithmic_bytes(w):
+def algorithmic_bytes(w, e4m3=False):
     elem = 2 if w.dtype == "bf16" else 4
     t = w.B * w.H * w.N * w.D * elem
+    if e4m3:   # q, k, v one byte per element, out bf16
+        return 3 * w.B * w.H * w.N * w.D + t
     wbytes = (w.H * w.D * w.F * elem) if w.F else 0
     return 4 * t + wbytes    # read q, k, v once, write out once (+ W)
 
@@ -341,13 +343,18 @@ def parity_samples(w):
     return [(b, h, sl) for b, h in heads[:2]]
 
 
-def parity_block(w, q, k, v, W, got, ttr=None):
+def parity_block(w, q, k, v, W, got, ttr=None, e4m3=False):
     """Error figures of the GPU output `got` against the float64 oracle on
     the sampled heads / rows (CPU torch tensors of the stored values); with
-    `ttr` = (landmark count, logits), against the oracle's TTR layer."""
+    `ttr` = (landmark count, logits), against the oracle's TTR layer; with
+    `e4m3`, q, k, v are E4M3 codes and W holds their three scales."""
     from linear_attention_diffusion_phi_b200.inputs import as_float64
     from oracle import la_oracle as ora
-    qf, kf, vf, Wf = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
+    if e4m3:
+        qf, kf, vf = (s * ora.e4m3_decode(c.numpy()) for s, c in zip(W, (q, k, v)))
+        Wf = None
+    else:
+        qf, kf, vf, Wf = as_float64(q), as_float64(k), as_float64(v), as_float64(W)
     diffs, refs, n_rows = [], [], 0
     for b, h, rows in parity_samples(w):
         g = as_float64(got[b, h])
@@ -390,24 +397,34 @@ class Timed:
     shifted along the sequence, so every step reads memory the previous steps
     did not touch), the operator, and CUDA graphs of its steps."""
 
-    def __init__(self, w, dev, rank, graphs=True, ttr=None):
+    def __init__(self, w, dev, rank, graphs=True, ttr=None, e4m3=False):
         import torch
         import linear_attention_diffusion_phi_b200 as la
-        from linear_attention_diffusion_phi_b200.inputs import make_inputs
+        from linear_attention_diffusion_phi_b200.inputs import make_e4m3_inputs, make_inputs
         self.w = w
         # (landmark count, logits): time the TTR layer instead of la_forward
         self.ttr = ttr
         self.gate = None if ttr is None else torch.tensor(ttr[1], dtype=torch.float32, device=dev)
+        # e4m3: q, k, v stored as E4M3 codes with per-tensor scales (la_forward_e4m3)
+        self.e4m3 = e4m3
         dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-        self.set_bytes = 4 * w.B * w.H * w.N * w.D * (2 if w.dtype == "bf16" else 4)
+        self.set_bytes = algorithmic_bytes(w, e4m3) - (w.H * w.D * w.F * (2 if w.dtype == "bf16" else 4) if w.F else 0)
         self.nsets = max(2, -(-3 * L2_BYTES // self.set_bytes))
-        self.host = make_inputs(w, seed=input_seed(w, 0, rank))
-        q, k, v, W = self.host
+        if e4m3:
+            q, k, v, self.scales = make_e4m3_inputs(w, seed=input_seed(w, 0, rank))
+            W = None
+            self.host = (q, k, v, self.scales)
+            out_like = lambda: torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        else:
+            self.host = make_inputs(w, seed=input_seed(w, 0, rank))
+            q, k, v, W = self.host
+            out_like = None
         base = (q.to(dev), k.to(dev), v.to(dev))
-        self.sets = [base + (torch.empty_like(base[0]),)]
+        new_out = out_like or (lambda: torch.empty_like(base[0]))
+        self.sets = [base + (new_out(),)]
         for i in range(1, self.nsets):
             sh = (97 * i) % max(w.N, 1)
-            self.sets.append(tuple(torch.roll(x, shifts=sh, dims=2) for x in base) + (torch.empty_like(base[0]),))
+            self.sets.append(tuple(torch.roll(x, shifts=sh, dims=2) for x in base) + (new_out(),))
         self.op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, None if W is None else W.to(dev))
         self.graphs = graphs
         self.g_all = None
@@ -420,7 +437,9 @@ class Timed:
 
     def step(self, i):
         q, k, v, o = self.sets[i % self.nsets]
-        if self.ttr is None:
+        if self.e4m3:
+            self.op.e4m3(q, k, v, self.scales, out=o)
+        elif self.ttr is None:
             self.op(q, k, v, out=o)
         else:
             self.op.ttr(q, k, v, self.ttr[0], self.gate, out=o)
@@ -526,7 +545,18 @@ def roofline(w, per_step_s, hbm, tflops, src, sms):
     return roof, launches
 
 
-EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr")
+def roofline_e4m3(w, per_step_s, hbm, src, name):
+    """HBM roofline of the E4M3-input forward (one launch per step): q, k, v
+    read once at one byte per element, out written once in bf16."""
+    abytes = algorithmic_bytes(w, e4m3=True)
+    achieved = abytes / per_step_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": captured_traffic(w, name), "peak_source": f"{src} hbm_gbs", "frac_of": src,
+            "kernel": "fused_t_kernel, E4M3 inputs (one cluster launch per step)",
+            "algorithmic_bytes_per_step": abytes}
+
+
+EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr", "flux1024_e4m3", "flux2048_cfg_e4m3")
 # The TTR layer on the flux1024 shape: 128 landmarks (the page's knobs at
 # fraction 1/32, min 16, max 128) and one logit per head, spread over [-2, 2].
 TTR_LANDMARKS = (1 / 32, 16, 128)
@@ -644,9 +674,10 @@ def main():
     if ws == 1 and not args.no_extra and w.name == "flux1024":
         for name in EXTRA_WORKLOADS:
             ttr = name.endswith("_ttr")
-            x = WORKLOADS[name[:-4] if ttr else name]
+            e8 = name.endswith("_e4m3")
+            x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else name)]
             try:
-                tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None)
+                tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8)
                 xsteps = max(args.steps, 100)
                 tx.steps_hint = xsteps
                 smp = ClockSampler(local)
@@ -664,13 +695,16 @@ def main():
                     xroof["kernel"] = "fused_t_kernel + landmark_blend_kernel (two launches per step)"
                     xroof["traffic"] = captured_traffic(x, name)
                     xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
+                if e8:
+                    xroof = roofline_e4m3(x, xms / 1e3 / xsteps, hbm, src, name)
                 ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
-                       "causal": x.causal, "dtype": x.dtype, "steps": xsteps, "ms_per_step": xms / xsteps,
+                       "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
+                       "ms_per_step": xms / xsteps,
                        "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
                        "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
                        "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
                 if not args.no_parity:
-                    ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr)
+                    ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8)
                 tx.close()
                 del tx
             except Exception as e:   # an extra figure never costs the headline line

@@ -623,9 +623,11 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   // slot is free again (a K slot once the phi warps have read it, a V slot
   // once its MMAs are done); qfree: a Q tile has been read by the phi warps.
   __shared__ __align__(8) uint64_t full[C::kRing1], vfull[C::kRing1], empty[C::kRing1], qfree[C::kRing1];
-  // E8: an E4M3 K or V tile has landed in its slot (the widening warps then
-  // rewrite the slot as bf16 and arrive on full or vfull)
-  __shared__ __align__(8) uint64_t landed[C::kRing1];
+  // E8: an E4M3 tile has landed in the second half of its slot (landed), and
+  // a K or V tile has been widened to bf16 over the whole slot by the eight
+  // widening warps (wready; the phi warps and the MMA issuer wait on it in
+  // place of full and vfull)
+  __shared__ __align__(8) uint64_t landed[C::kRing1], wready[C::kRing1];
   // A buffers in tensor memory, used in turn by the T key tiles and then the
   // T query tiles: written by the phi warps (aready), read by the MMAs (aempty).
   __shared__ __align__(8) uint64_t aready[C::kABufs], aempty[C::kABufs];
@@ -661,7 +663,8 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   auto uses1 = [&](int phys) { return (2 * T + C::kRing1 - 1 - phys) / C::kRing1; };
   auto q_full_round = [&](int u) {   // phases of full[] before Q tile u
     const int s = u % C::kRing2;
-    return ((s & 1) == 0 ? uses1(s) : 0) + u / C::kRing2;
+    // (E4M3 K tiles complete wready, not full)
+    return ((s & 1) == 0 && !E8 ? uses1(s) : 0) + u / C::kRing2;
   };
   // image rows [row0(o), row0(o + 1)) are owned by cluster CTA o
   auto row0 = [&](int o) { return o * C::kRows / S; };
@@ -675,6 +678,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       mbar_init(&empty[i], (i & 1) == 0 ? kKWarps : 1);
       mbar_init(&qfree[i], C::kPhiWarps);
       mbar_init(&landed[i], 1);
+      mbar_init(&wready[i], 8);
     }
     for (int i = 0; i < C::kABufs; ++i) {
       mbar_init(&aready[i], kKWarps);
@@ -734,11 +738,11 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       uint64_t* bar = is_v ? &vfull[s] : &full[s];
       uint8_t* dst = slot_ptr(s);
       if constexpr (E8) {
-        // the codes fill the first 16 KB of the slot; K and V are widened
-        // in place before full / vfull, Q is read as codes by the phi warps
+        // the codes fill the second 16 KB of the slot: K and V are widened
+        // over the whole slot, Q is read as codes by the phi warps
         if (p1) bar = &landed[s];
         mbar_arrive_expect_tx(bar, kCodeTileBytes);
-        tma_load_3d(dst, m, bar, 0, (tile0 + tile) * kTileTokens, bh);
+        tma_load_3d(dst + kCodeTileBytes, m, bar, 0, (tile0 + tile) * kTileTokens, bh);
       } else {
         mbar_arrive_expect_tx(bar, C::kSlotBytes);
 #pragma unroll
@@ -766,7 +770,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     const int lm = lane >> 3, lr = lane & 7;
     for (int t = 0; t < T; ++t) {
       const int s = (2 * t) % C::kRing1, b = t % C::kABufs;
-      if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
+      if (!warp_wait(E8 ? &wready[s] : &full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
       const uint32_t base = smem_u32(slot_ptr(s));
       uint32_t x[2][kBlocks][4];
 #pragma unroll
@@ -825,7 +829,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       for (int t = 0; t < T; ++t) {
         const int sv = (2 * t + 1) % C::kRing1, b = t % C::kABufs;
         if (!mbar_wait(&aready[b], (t / C::kABufs) & 1, status) ||
-            !mbar_wait(&vfull[sv], ((2 * t + 1) / C::kRing1) & 1, status)) {
+            !mbar_wait(E8 ? &wready[sv] : &vfull[sv], ((2 * t + 1) / C::kRing1) & 1, status)) {
           ok = false;
           break;
         }
@@ -890,7 +894,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int c = 4 * hf + m;
-          raw[m] = *reinterpret_cast<const uint4*>(src + i * 128 + ((c ^ (i & 7)) << 4));
+          raw[m] = *reinterpret_cast<const uint4*>(src + kCodeTileBytes + i * 128 + ((c ^ (i & 7)) << 4));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
@@ -926,41 +930,40 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     const bool leader = ct == 0;
     const int q = warp & 3;
     const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
-    // E8: widen every K and V tile in place (codes times sk or sv, rounded to
+    // E8: widen every K and V tile to bf16 (codes times sk or sv, rounded to
     // bf16, in the layout of a bf16 tile), in the order they were issued.
-    // Every warp meets both barriers of every tile even after a wait has
-    // given up (the output is then undefined and the status word says so).
+    // Warp w takes rows 16 w .. 16 w + 15, eight lanes per row.  The codes of
+    // row r sit in the slot's second half exactly where the bf16 row r of
+    // features 64..127 goes, and only the eight lanes of row r touch either,
+    // so a __syncwarp between their reads and writes is all the ordering the
+    // rewrite needs; each warp then arrives on wready.
     auto widen = [&]() {
-      bool good = true;
+      const int w8 = warp - C::kCombWarp0, c = lane & 7;
       for (int j = 0; j < 2 * T; ++j) {
         const int s = j % C::kRing1;
         uint8_t* slot = slot_ptr(s);
-        good = good && warp_wait(&landed[s], (j / C::kRing1) & 1, status);
+        if (!warp_wait(&landed[s], (j / C::kRing1) & 1, status)) return false;
         uint4 raw[4];
-        if (good) {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int unit = ct + 256 * r, row = unit >> 3, c = unit & 7;
-            raw[r] = *reinterpret_cast<const uint4*>(slot + row * 128 + ((c ^ (row & 7)) << 4));
-          }
+        for (int r = 0; r < 4; ++r) {
+          const int row = 16 * w8 + 4 * r + (lane >> 3);
+          raw[r] = *reinterpret_cast<const uint4*>(slot + kCodeTileBytes + row * 128 + ((c ^ (row & 7)) << 4));
         }
-        named_bar_sync(3, 256);   // the whole tile is in registers
-        if (good) {
-          const float sc = (j & 1) ? sv : sk;
+        __syncwarp();
+        const float sc = (j & 1) ? sv : sk;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int unit = ct + 256 * r, row = unit >> 3, c = unit & 7;
-            uint4 lo, hi;
-            e4m3x16_to_bf16(raw[r], sc, lo, hi);
-            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c)) = lo;
-            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c + 1)) = hi;
-          }
+        for (int r = 0; r < 4; ++r) {
+          const int row = 16 * w8 + 4 * r + (lane >> 3);
+          uint4 lo, hi;
+          e4m3x16_to_bf16(raw[r], sc, lo, hi);
+          *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c)) = lo;
+          *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c + 1)) = hi;
         }
         fence_proxy_async_smem();   // V tiles feed the tensor core
-        named_bar_sync(3, 256);
-        if (good && leader) mbar_arrive((j & 1) ? &vfull[s] : &full[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wready[s]);
       }
-      return good;
+      return true;
     };
     bool got = E8 ? widen() : (kKWarps == 16 ? k_phase() : true);
     auto sync_ok = [&](bool mine) {
