@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads timed after the headline (1 GPU only)")
     ap.add_argument("--no-parity", action="store_true", help="skip the oracle comparison of sampled heads")
+    ap.add_argument("--extra-only", default=None, choices=list(EXTRA_WORKLOADS),
+                    help="time only this extra configuration and print its entry (for profiling runs)")
     return ap.parse_args()
 
 
@@ -568,6 +570,52 @@ def ttr_params(w):
     return la.la_landmark_count(w.N, *TTR_LANDMARKS), [float(x) for x in np.linspace(-2.0, 2.0, w.H)]
 
 
+def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
+    """Time one of EXTRA_WORKLOADS the way the headline is timed (at least 100
+    steps) and return its entry for the line's extra_configs."""
+    import torch
+    import linear_attention_diffusion_phi_b200 as la
+    from linear_attention_diffusion_phi_b200.inputs import WORKLOADS
+    ttr = name.endswith("_ttr")
+    e8 = name.endswith("_e4m3")
+    x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else name)]
+    try:
+        tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8)
+        xsteps = max(args.steps, 100)
+        tx.steps_hint = xsteps
+        smp = ClockSampler(local)
+        smp.start()
+        tx.warm(args.warmup, 0.3)
+        xms = tx.timed_ms(xsteps, stream, ws)
+        xclk = smp.stop()
+        assert tx.op.sync_status() == la.LA_OK, "device-side error during the timed region"
+        xroof, xl = roofline(x, xms / 1e3 / xsteps, hbm, tflops, src, sms)
+        if ttr:
+            # two launches; the roofline is the layer's: q, k, v read
+            # once and out written once (the landmark pass adds a read
+            # of q and a read and write of out on top)
+            xl = 2
+            xroof["kernel"] = "fused_t_kernel + landmark_blend_kernel (two launches per step)"
+            xroof["traffic"] = captured_traffic(x, name)
+            xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
+        if e8:
+            xroof = roofline_e4m3(x, xms / 1e3 / xsteps, hbm, src, name)
+        ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
+               "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
+               "ms_per_step": xms / xsteps,
+               "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
+               "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
+               "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
+        if not args.no_parity:
+            ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8)
+        tx.close()
+        del tx
+    except Exception as e:   # an extra figure never costs the headline line
+        ent = {"workload": name, "error": f"{type(e).__name__}: {e}"[:300]}
+    torch.cuda.empty_cache()
+    return ent
+
+
 def main():
     args = parse()
     from linear_attention_diffusion_phi_b200.inputs import WORKLOADS
@@ -594,6 +642,12 @@ def main():
     stream = torch.cuda.current_stream(dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     hbm, tflops, src = peaks()
+
+    if args.extra_only:
+        ent = run_extra(args.extra_only, args, dev, rank, local, stream, ws, hbm, tflops, src, sms)
+        if rank == 0:
+            print(json.dumps(ent))
+        return 0 if "error" not in ent else 1
 
     tw = Timed(w, dev, rank, graphs=not args.no_graph)
     tw.steps_hint = args.steps
@@ -673,44 +727,7 @@ def main():
     extras = []
     if ws == 1 and not args.no_extra and w.name == "flux1024":
         for name in EXTRA_WORKLOADS:
-            ttr = name.endswith("_ttr")
-            e8 = name.endswith("_e4m3")
-            x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else name)]
-            try:
-                tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8)
-                xsteps = max(args.steps, 100)
-                tx.steps_hint = xsteps
-                smp = ClockSampler(local)
-                smp.start()
-                tx.warm(args.warmup, 0.3)
-                xms = tx.timed_ms(xsteps, stream, ws)
-                xclk = smp.stop()
-                assert tx.op.sync_status() == la.LA_OK, "device-side error during the timed region"
-                xroof, xl = roofline(x, xms / 1e3 / xsteps, hbm, tflops, src, sms)
-                if ttr:
-                    # two launches; the roofline is the layer's: q, k, v read
-                    # once and out written once (the landmark pass adds a read
-                    # of q and a read and write of out on top)
-                    xl = 2
-                    xroof["kernel"] = "fused_t_kernel + landmark_blend_kernel (two launches per step)"
-                    xroof["traffic"] = captured_traffic(x, name)
-                    xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
-                if e8:
-                    xroof = roofline_e4m3(x, xms / 1e3 / xsteps, hbm, src, name)
-                ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
-                       "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
-                       "ms_per_step": xms / xsteps,
-                       "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
-                       "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
-                       "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
-                if not args.no_parity:
-                    ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8)
-                tx.close()
-                del tx
-            except Exception as e:   # an extra figure never costs the headline line
-                ent = {"workload": name, "error": f"{type(e).__name__}: {e}"[:300]}
-            extras.append(ent)
-            torch.cuda.empty_cache()
+            extras.append(run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms))
 
     if ws > 1:
         dist.destroy_process_group()
