@@ -80,11 +80,13 @@ def algorithmic_flops(w):
 # device headers it includes) still hashes to what was captured; else null.
 DEVICE_HEADERS = ("bf16_common.cuh", "sm100.cuh")
 NCU_TRAFFIC = {
-    "flux1024": (88_649_216, ("bf16_noncausal.cu",), "d1510f5b4c6763ac"),
-    "flux2048_cfg": (780_859_648, ("bf16_noncausal.cu",), "d1510f5b4c6763ac"),
+    "flux1024": (89_199_616, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
+    "flux2048_cfg": (780_559_872, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
     "causal32k": (716_144_384, ("bf16_causal.cu",), "3e37cbf7e846ccac"),
     "proj256": (99_814_016, ("bf16_proj.cu", "bf16_image.cu"), "4d91d4572082bf07"),
-    "flux1024_ttr": (146_939_456, ("bf16_noncausal.cu", "bf16_landmark.cu"), "ba5a94f6fc141518"),
+    "flux1024_ttr": (144_733_952, ("bf16_noncausal.cu", "bf16_landmark.cu"), "10a1909d84b22ba5"),
+    "flux1024_e4m3": (42_692_992, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
+    "flux2048_cfg_e4m3": (460_586_112, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
 }
 
 
