@@ -16,6 +16,7 @@ from .la_oracle import (  # noqa: F401
     linear_noncausal_head,
     phi_elu1,
     phi_relu,
+    phi_softmax,
     rows,
     sigmoid,
     ttr_forward,

@@ -34,12 +34,12 @@ feature axis last; W is [H, D, F] (one matrix per head) or [D, F] (shared).
 
 import numpy as np
 
-FEATURE_MAPS = ("elu", "relu")
+FEATURE_MAPS = ("elu", "relu", "softmax")
 
 
 # --------------------------------------------------------------------------
 # Feature maps (page "NNT Define Linear Attention", "The inputs": feature_map
-# is elu, mapped as elu(x)+1, or relu; both are non-negative).
+# is elu, mapped as elu(x)+1, relu or softmax; all are non-negative).
 # --------------------------------------------------------------------------
 
 def phi_elu1(x):
@@ -52,6 +52,18 @@ def phi_relu(x):
     """relu(x) = max(x, 0)."""
     x = np.asarray(x, dtype=np.float64)
     return np.maximum(x, 0.0)
+
+
+def phi_softmax(x):
+    """softmax over the feature axis (the last): exp(x_f - max) / sum_f' exp(x_f' - max).
+
+    Reading: the page lists softmax as a third feature map without naming its
+    axis; a feature map takes one token's vector to a non-negative vector of
+    features, so the softmax runs over that vector.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(x - x.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
 
 
 def feature_map(x, fmap, W=None):
@@ -68,6 +80,8 @@ def feature_map(x, fmap, W=None):
         return phi_elu1(x)
     if fmap == "relu":
         return phi_relu(x)
+    if fmap == "softmax":
+        return phi_softmax(x)
     raise ValueError(f"unknown feature map {fmap!r}")
 
 

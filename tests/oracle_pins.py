@@ -418,6 +418,44 @@ def pin_ttr_blend_limits(ora):
 
 
 
+
+# ------------------------------------------------------ softmax feature map --
+
+def pin_softmax_vs_scipy(ora):
+    """phi_softmax is scipy's softmax over the last axis (a library routine),
+    including rows whose entries are far beyond exp's range."""
+    from scipy.special import softmax
+    rng = _rng(51)
+    for scale in (1.0, 30.0, 800.0):
+        x = rng.standard_normal((3, 5, 17)) * scale
+        _close(ora.phi_softmax(x), softmax(x, axis=-1), rtol=1e-12, atol=1e-300)
+        _close(ora.feature_map(x, "softmax"), softmax(x, axis=-1), rtol=1e-12, atol=1e-300)
+
+
+def pin_softmax_closed_forms(ora):
+    """[0, ln 2, ln 3] -> [1/6, 2/6, 3/6]; a constant row -> 1/D; adding a
+    constant to a row changes nothing; the features of a row sum to 1."""
+    _close(ora.phi_softmax(np.log([1.0, 2.0, 3.0])), np.array([1.0, 2.0, 3.0]) / 6.0, rtol=1e-14)
+    _close(ora.phi_softmax(np.full((2, 8), 3.7)), np.full((2, 8), 1.0 / 8.0), rtol=1e-14)
+    x = _rng(52).standard_normal((4, 9))
+    _close(ora.phi_softmax(x + 11.0), ora.phi_softmax(x), rtol=1e-12)
+    _close(ora.phi_softmax(x).sum(axis=-1), np.ones(4), rtol=1e-14)
+
+
+def pin_softmax_equal_keys(ora):
+    """With every key row equal, every weight is s = phi(q_i).phi(k), so
+    out_i = s sum_j v_j / (N s + eps), for the grouped form and the definition."""
+    rng = _rng(53)
+    N, D = 7, 5
+    q = rng.standard_normal((1, 1, N, D))
+    k = np.broadcast_to(rng.standard_normal(D), (1, 1, N, D)).copy()
+    v = rng.standard_normal((1, 1, N, 3))
+    eps = 0.25
+    s = ora.phi_softmax(q[0, 0]) @ ora.phi_softmax(k[0, 0, 0])
+    want = (s[:, None] * v[0, 0].sum(axis=0)[None, :]) / (N * s[:, None] + eps)
+    _close(ora.forward(q, k, v, "softmax", eps)[0, 0], want, rtol=1e-12)
+    _close(ora.brute_force(q, k, v, "softmax", eps)[0, 0], want, rtol=1e-12)
+
 # ------------------------------------------------------- FP8 (E4M3) storage --
 
 def _torch_e4m3(codes):
@@ -493,4 +531,7 @@ ALL_PINS = [
     pin_e4m3_vs_torch,
     pin_e4m3_format_facts,
     pin_e4m3_forward,
+    pin_softmax_vs_scipy,
+    pin_softmax_closed_forms,
+    pin_softmax_equal_keys,
 ]

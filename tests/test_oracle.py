@@ -55,6 +55,11 @@ MUTANTS = [
     ("landmark_count_no_clamp", "return max(1, min(n, max(lo, min(hi, want))))", "return max(1, min(n, want))"),
     ("landmark_count_rounds_down", "want = int(np.floor(fraction * n + 0.5))", "want = int(np.floor(fraction * n))"),
     ("sigmoid_wrong_sign", "return 1.0 / (1.0 + np.exp(-g))", "return 1.0 / (1.0 + np.exp(g))"),
+    ("softmax_wrong_axis", "e = np.exp(x - x.max(axis=-1, keepdims=True))\n    return e / e.sum(axis=-1, keepdims=True)",
+     "e = np.exp(x - x.max(axis=0, keepdims=True))\n    return e / e.sum(axis=0, keepdims=True)"),
+    ("softmax_not_normalised", "return e / e.sum(axis=-1, keepdims=True)", "return e"),
+    ("softmax_wrong_sign", "e = np.exp(x - x.max(axis=-1, keepdims=True))", "e = np.exp(x.max(axis=-1, keepdims=True) - x)"),
+    ("softmax_is_elu", "    if fmap == \"softmax\":\n        return phi_softmax(x)", "    if fmap == \"softmax\":\n        return phi_elu1(x)"),
     ("e4m3_bias_eight", "np.exp2(e - 7.0)", "np.exp2(e - 8.0)"),
     ("e4m3_no_subnormals", "np.where(e == 0, (m / 8.0) * 2.0 ** -6,", "np.where(e < 0, (m / 8.0) * 2.0 ** -6,"),
     ("e4m3_subnormal_scale", "(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7"),
@@ -93,7 +98,7 @@ def test_oracle_rejects_bad_arguments():
     import numpy as np
     x = np.zeros((1, 1, 4, 2))
     with pytest.raises(ValueError):
-        la_oracle.forward(x, x, x, "softmax")
+        la_oracle.forward(x, x, x, "tanh")
     with pytest.raises(ValueError):
         la_oracle.forward(x, x, x, "elu", eps=-1.0)
     with pytest.raises(ValueError):
