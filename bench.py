@@ -560,7 +560,8 @@ def roofline_e4m3(w, per_step_s, hbm, src, name):
             "algorithmic_bytes_per_step": abytes}
 
 
-EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr", "flux1024_e4m3", "flux2048_cfg_e4m3")
+EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr", "flux1024_e4m3", "flux2048_cfg_e4m3",
+                   "flux1024_softmax")
 # The TTR layer on the flux1024 shape: 128 landmarks (the page's knobs at
 # fraction 1/32, min 16, max 128) and one logit per head, spread over [-2, 2].
 TTR_LANDMARKS = (1 / 32, 16, 128)
@@ -580,7 +581,10 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
     from linear_attention_diffusion_phi_b200.inputs import WORKLOADS
     ttr = name.endswith("_ttr")
     e8 = name.endswith("_e4m3")
-    x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else name)]
+    smx = name.endswith("_softmax")   # the same shapes with the softmax feature map
+    x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else (name[:-8] if smx else name))]
+    if smx:
+        x = x.with_(fmap="softmax")
     try:
         tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8)
         xsteps = max(args.steps, 100)
@@ -602,6 +606,8 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
             xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
         if e8:
             xroof = roofline_e4m3(x, xms / 1e3 / xsteps, hbm, src, name)
+        if smx:
+            xroof["traffic"] = captured_traffic(x, name)
         ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
                "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
                "ms_per_step": xms / xsteps,

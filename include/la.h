@@ -9,7 +9,11 @@
  *     out_i = phi(q_i)^T kv / (phi(q_i) . ksum + eps).
  * This equals the weighted sum  sum_j w_ij v_j / (sum_j w_ij + eps)  with
  * w_ij = phi(q_i) . phi(k_j); the N x N weight matrix is never formed.
- *   feature maps  LA_PHI_ELU1: elu(x)+1 (alpha = 1);  LA_PHI_RELU: max(x, 0)
+ *   feature maps  LA_PHI_ELU1: elu(x)+1 (alpha = 1);  LA_PHI_RELU: max(x, 0);
+ *                 LA_PHI_SOFTMAX: softmax over each row's feature vector,
+ *                 exp(x_f - max x) / sum_f' exp(x_f' - max x) (the page lists
+ *                 softmax without naming its axis; a feature map takes one
+ *                 token's vector to its features, so it runs over that vector)
  *   causal        query i sees keys j <= i (itself included)
  *   projection    F > 0: phi(x) = fmap(x W_h) with a D x F matrix per head
  *                 (page "Flux2TTRTrainer", "Inputs worth setting": feature_dim
@@ -75,7 +79,7 @@ typedef enum {
 } la_status_t;
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype_t;
-typedef enum { LA_PHI_ELU1 = 0, LA_PHI_RELU = 1 } la_feature_map_t;
+typedef enum { LA_PHI_ELU1 = 0, LA_PHI_RELU = 1, LA_PHI_SOFTMAX = 2 } la_feature_map_t;
 
 /* Create a handle for one storage dtype (LA_F32 or LA_BF16).  Allocates host
  * memory only.  LA_F32 runs fp32 CUDA-core kernels with fp32 accumulation;
@@ -123,6 +127,9 @@ la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
  * Supported: LA_F32: D <= 128, D % 4 == 0, F in {0, 256}.
  *            LA_BF16: D in {64, 128}; F in {0, 256} with D = 128 when F > 0;
  *            causal with F = 0 and D = 64.
+ *            LA_PHI_SOFTMAX: F = 0; on LA_BF16 non-causal with D = 128 only
+ *            (also through la_forward_ttr and la_forward_noalloc; not
+ *            la_forward_e4m3).  Other combinations: LA_ERR_UNSUPPORTED.
  * The result is deterministic: the same arguments give bitwise the same out. */
 la_status_t la_forward(la_handle_t handle, const void* q, const void* k, const void* v,
                        void* out, int B, int H, int N, int D, int F, int feature_map,

@@ -15,8 +15,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libla_phi.so")
 
 LA_F32, LA_BF16 = 0, 1
-LA_PHI_ELU1, LA_PHI_RELU = 0, 1
-FEATURE_MAPS = {"elu": LA_PHI_ELU1, "relu": LA_PHI_RELU}
+LA_PHI_ELU1, LA_PHI_RELU, LA_PHI_SOFTMAX = 0, 1, 2
+FEATURE_MAPS = {"elu": LA_PHI_ELU1, "relu": LA_PHI_RELU, "softmax": LA_PHI_SOFTMAX}
 
 LA_OK = 0
 (LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_MISALIGNED, LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_TIMEOUT,

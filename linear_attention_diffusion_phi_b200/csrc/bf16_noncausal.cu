@@ -601,6 +601,16 @@ __device__ __forceinline__ void e4m3x16_to_bf16(uint4 raw, float scale, uint4& l
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// Softmax features of two tokens' values of one feature (bf16x2, lower token
+// in the low half): exp(x - m) * rz with that token's row maximum m and
+// reciprocal exponential sum rz, rounded to bf16.
+__device__ __forceinline__ uint32_t softmax_pair(uint32_t w, float m0, float rz0, float m1, float rz1) {
+  const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  const __nv_bfloat162 r = __floats2bfloat162_rn(ex2_approx((x.x - m0) * kLog2e) * rz0,
+                                                 ex2_approx((x.y - m1) * kLog2e) * rz1);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // E8: q, k and v are E4M3 codes (tensor maps of bytes, 128 x 128 boxes) with
 // one scale each; out is bf16 as for bf16 inputs.
 template <int FMAP, bool XC, bool E8>
@@ -616,6 +626,11 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   // relu is cheap enough for eight.  With E4M3 inputs the combine warps
   // widen the K and V tiles to bf16 in phase 1 instead.
   constexpr int kKWarps = FMAP == 0 && !E8 ? 16 : 8;
+  // Softmax (FMAP 2): the combine warps compute each K row's maximum and
+  // reciprocal exponential sum in phase 1 (kst, a ring over K tiles; kstat
+  // when a tile's rows are in), and read the K slot too.
+  constexpr bool kSmx = FMAP == 2;
+  constexpr int kStatRing = 6;
   constexpr uint32_t kCodeTileBytes = kTileTokens * C::D;   // one E4M3 tile
   extern __shared__ uint8_t smem_raw[];
   // full: a K or Q tile has arrived (waited on by the phi warps, every phase
@@ -628,6 +643,8 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   // widening warps (wready; the phi warps and the MMA issuer wait on it in
   // place of full and vfull)
   __shared__ __align__(8) uint64_t landed[C::kRing1], wready[C::kRing1];
+  __shared__ __align__(8) uint64_t kstat[kStatRing];
+  __shared__ __align__(16) float2 kst[kSmx ? kStatRing * kTileTokens : 1];
   // A buffers in tensor memory, used in turn by the T key tiles and then the
   // T query tiles: written by the phi warps (aready), read by the MMAs (aempty).
   __shared__ __align__(8) uint64_t aready[C::kABufs], aempty[C::kABufs];
@@ -675,11 +692,12 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     for (int i = 0; i < C::kRing1; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&vfull[i], 1);
-      mbar_init(&empty[i], (i & 1) == 0 ? kKWarps : 1);
+      mbar_init(&empty[i], (i & 1) == 0 ? kKWarps + (kSmx ? 8 : 0) : 1);
       mbar_init(&qfree[i], C::kPhiWarps);
       mbar_init(&landed[i], 1);
       mbar_init(&wready[i], 8);
     }
+    for (int i = 0; i < kStatRing; ++i) mbar_init(&kstat[i], 8);
     for (int i = 0; i < C::kABufs; ++i) {
       mbar_init(&aready[i], kKWarps);
       mbar_init(&aempty[i], 1);
@@ -784,6 +802,10 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
         }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);   // the K tile is in registers
+      // softmax: this tile's row statistics (their ring entry is rewritten
+      // only after this warp has read the K slot of three tiles later)
+      const float2* st = kst + (t % kStatRing) * kTileTokens;
+      if (kSmx && !warp_wait(&kstat[t % kStatRing], (t / kStatRing) & 1, status)) return false;
       // key rows past the sequence end must not reach kv or ksum
       const int valid = min(kTileTokens, N - (tile0 + t) * kTileTokens);
 #pragma unroll
@@ -792,7 +814,14 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
         for (int tb = 0; tb < kBlocks; ++tb)
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            uint32_t w = phi_pair<FMAP>(x[fh][tb][r]);
+            uint32_t w;
+            if constexpr (kSmx) {
+              const int tk = kTok * kq + 16 * tb + 8 * (r >> 1) + 2 * (lane & 3);
+              const float4 mz = *reinterpret_cast<const float4*>(st + tk);   // tokens tk, tk + 1
+              w = softmax_pair(x[fh][tb][r], mz.x, mz.y, mz.z, mz.w);
+            } else {
+              w = phi_pair<FMAP>(x[fh][tb][r]);
+            }
             if (valid < kTileTokens) {
               const int tok = kTok * kq + 16 * tb + 8 * (r >> 1) + 2 * (lane & 3);
               w &= (tok < valid ? 0x0000FFFFu : 0u) | (tok + 1 < valid ? 0xFFFF0000u : 0u);
@@ -887,6 +916,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       if (!warp_wait(&full[s], q_full_round(u) & 1, status)) break;
       const uint8_t* src = slot_ptr(s);
       uint4 x[8];
+      float rowmax = 0.f;
       if constexpr (E8) {
         // codes of features 64 hf .. 64 hf + 63: four 16-byte chunks of the
         // 128-byte row (128-byte swizzle), widened to bf16 times sq
@@ -903,17 +933,45 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       } else {
 #pragma unroll
         for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
+        if constexpr (kSmx) {
+          // softmax: the row's maximum over all 128 features (the other
+          // half's chunks are read for it, before the slot is released)
+          __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&x[0].x);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const uint32_t o[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+            const uint4 y = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * (1 - hf) + m));
+            const uint32_t p[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              mx = __hmax2(mx, __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&o[e]),
+                                       *reinterpret_cast<const __nv_bfloat162*>(&p[e])));
+          }
+          rowmax = fmaxf(__low2float(mx), __high2float(mx));
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
       }
       uint32_t w[32];
+      if constexpr (kSmx) {
+        // exp(x - rowmax): the row's normaliser is not applied; with eps
+        // folded into ksum it cancels exactly
+        const float c = rowmax;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const uint4 y = phi_chunk<FMAP>(x[m]);
-        w[4 * m] = y.x;
-        w[4 * m + 1] = y.y;
-        w[4 * m + 2] = y.z;
-        w[4 * m + 3] = y.w;
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t o[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[4 * m + e] = softmax_pair(o[e], c, 1.f, c, 1.f);
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint4 y = phi_chunk<FMAP>(x[m]);
+          w[4 * m] = y.x;
+          w[4 * m + 1] = y.y;
+          w[4 * m + 2] = y.z;
+          w[4 * m + 3] = y.w;
+        }
       }
       if (j >= C::kABufs && !warp_wait(&aempty[b], ((j / C::kABufs) - 1) & 1, status)) break;
       tc_fence_after();
@@ -965,7 +1023,46 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       }
       return true;
     };
-    bool got = E8 ? widen() : (kKWarps == 16 ? k_phase() : true);
+    // softmax: each K row's maximum and reciprocal exponential sum, two
+    // threads per row (adjacent lanes, 64 features each), into kst
+    auto kstats = [&]() {
+      const int row = ct >> 1, hh = ct & 1;
+      for (int t = 0; t < T; ++t) {
+        const int s = (2 * t) % C::kRing1;
+        if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
+        const uint8_t* slot = slot_ptr(s);
+        uint4 x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(slot + swz_off(row, 8 * hh + m));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);   // the K tile is in registers
+        __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&x[0].x);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t o[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx = __hmax2(mx, *reinterpret_cast<const __nv_bfloat162*>(&o[e]));
+        }
+        float m0 = fmaxf(__low2float(mx), __high2float(mx));
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+        float z = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t o[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o[e]));
+            z += ex2_approx((v2.x - m0) * kLog2e) + ex2_approx((v2.y - m0) * kLog2e);
+          }
+        }
+        z += __shfl_xor_sync(0xffffffffu, z, 1);
+        if (hh == 0) kst[(t % kStatRing) * kTileTokens + row] = make_float2(m0, 1.f / z);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&kstat[t % kStatRing]);
+      }
+      return true;
+    };
+    bool got = E8 ? widen() : (kSmx ? kstats() : (kKWarps == 16 ? k_phase() : true));
     auto sync_ok = [&](bool mine) {
       if (leader && !mine) comb_flag = 1;
       named_bar_sync(3, 256);
@@ -1049,6 +1146,13 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
             acc[2 * e + 1] += x.y;
           }
         }
+        // softmax: eps joins every ksum entry once (after the last sum), so
+        // the apply's denominator is sum_f u_f (ksum_f + eps) for the
+        // unnormalised query features u
+        if (kSmx && !(XC && NC > 1) && n0 + rem / 8 >= D) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += eps;
+        }
         *reinterpret_cast<uint4*>(blob + off_img) = pack8(acc);
       }
       if (XC && NC > 1) {
@@ -1121,6 +1225,10 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
                       acc[2 * i + 1] += x.y;
                     }
                   }
+                if (kSmx && n0 + rem / 8 >= D) {   // eps into ksum (see above)
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) acc[i] += eps;
+                }
                 *reinterpret_cast<uint4*>(blob + off) = pack8(acc);
               }
             }
@@ -1164,7 +1272,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&accempty[a]);
-        const float inv = 1.0f / (den + eps);
+        const float inv = 1.0f / (kSmx ? den : den + eps);   // softmax: eps is in den already
 #pragma unroll
         for (int e = 0; e < kHalfCols; ++e) v[e] *= inv;
         uint8_t* ob = a == 0 ? recv : slots + (C::kSlots - 1) * C::kSlotBytes;
@@ -1330,6 +1438,11 @@ cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
   uint8_t* xchg = reinterpret_cast<uint8_t*>(a.ws + p.off_xchg);
   const int P = p.ctas_per_head, S = p.cluster;
   if (p.D == 128) {
+    if (p.fmap == 2) {
+      if (a.e4m3) return cudaErrorNotSupported;
+      return P > S ? launch_fused<CfgT>(a, fused_t_kernel<2, true, false>, P, S, sync, xchg)
+                   : launch_fused<CfgT>(a, fused_t_kernel<2, false, false>, P, S, sync, xchg);
+    }
     if (a.e4m3) {
       if (P > S)
         return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, true>, P, S, sync, xchg)
@@ -1343,7 +1456,7 @@ cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
     return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, false>, P, S, sync, xchg)
                        : launch_fused<CfgT>(a, fused_t_kernel<1, false, false>, P, S, sync, xchg);
   }
-  if (a.e4m3) return cudaErrorNotSupported;
+  if (a.e4m3 || p.fmap == 2) return cudaErrorNotSupported;
   if (p.D == 64)
     return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>, P, S, sync, xchg)
                        : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>, P, S, sync, xchg);

@@ -22,8 +22,11 @@ constexpr int kFB = 32;     // features per state block
 constexpr int kMaxD = 128;
 constexpr int kMaxFe = 256;
 
-// phi of token row `t` (already in shared memory) for feature f.
-__device__ __forceinline__ float feature(const float* xs, int D, const float* W, int F, int f, int fmap) {
+// phi of token row `t` (already in shared memory) for feature f.  The softmax
+// map (fmap 2, no projection) takes the row's maximum and the reciprocal of
+// its exponential sum from `st` (softmax_stats).
+__device__ __forceinline__ float feature(const float* xs, int D, const float* W, int F, int f, int fmap,
+                                         const float* st) {
   float x;
   if (F) {
     x = 0.f;
@@ -31,7 +34,30 @@ __device__ __forceinline__ float feature(const float* xs, int D, const float* W,
   } else {
     x = xs[f];
   }
+  if (fmap == 2) return expf(x - st[0]) * st[1];
   return phi_accurate(x, fmap);
+}
+
+// Softmax over each row of xs [kT][kMaxD]: st[2 t] = max_d x_td and
+// st[2 t + 1] = 1 / sum_d exp(x_td - max), one warp per row, lanes over d,
+// butterfly reductions (a fixed order: deterministic).  Zero-filled rows
+// give finite values that nothing reads.
+__device__ void softmax_stats(const float* xs, int D, float* st) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int t = warp; t < kT; t += blockDim.x / 32) {
+    float m = -INFINITY;
+    for (int d = lane; d < D; d += 32) m = fmaxf(m, xs[t * kMaxD + d]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = 0.f;
+    for (int d = lane; d < D; d += 32) z += expf(xs[t * kMaxD + d] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      st[2 * t] = m;
+      st[2 * t + 1] = 1.f / z;
+    }
+  }
 }
 
 __device__ __forceinline__ void load_rows(float* dst, const float* src, int rows_valid, int D) {
@@ -55,6 +81,7 @@ __global__ void __launch_bounds__(256) f32_state_partial(const float* __restrict
   __shared__ __align__(16) float Ks[kT * kMaxD];
   __shared__ __align__(16) float Vs[kT * kMaxD];
   __shared__ float Ps[kT * kFB];
+  __shared__ float Kst[2 * kT];
   const int s = blockIdx.x;
   const long long bh = blockIdx.y;
   const int fb = blockIdx.z * kFB;
@@ -72,9 +99,13 @@ __global__ void __launch_bounds__(256) f32_state_partial(const float* __restrict
     load_rows(Ks, kh + static_cast<size_t>(tc) * D, rows, D);
     load_rows(Vs, vh + static_cast<size_t>(tc) * D, rows, D);
     __syncthreads();
+    if (fmap == 2) {
+      softmax_stats(Ks, D, Kst);
+      __syncthreads();
+    }
     for (int e = threadIdx.x; e < kT * kFB; e += blockDim.x) {
       const int t = e / kFB, f = fb + e % kFB;
-      Ps[e] = (t < rows && f < Fe) ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+      Ps[e] = (t < rows && f < Fe) ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap, Kst + 2 * t) : 0.f;
     }
     __syncthreads();
     for (int t = 0; t < kT; ++t) {
@@ -150,6 +181,7 @@ __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, co
   __shared__ __align__(16) float Qs[kT * kMaxD];
   __shared__ float Ps[kT * kMaxFe];
   __shared__ float den[kT];
+  __shared__ float Qst[2 * kT];
   const long long bh = blockIdx.y;
   const int t0 = blockIdx.x * kT;
   const int rows = min(kT, N - t0);
@@ -158,9 +190,13 @@ __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, co
   const float* ksum = fin_ksum + static_cast<size_t>(bh) * Fe;
   load_rows(Qs, q + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
   __syncthreads();
+  if (fmap == 2) {
+    softmax_stats(Qs, D, Qst);
+    __syncthreads();
+  }
   for (int e = threadIdx.x; e < kT * Fe; e += blockDim.x) {
     const int t = e / Fe, f = e % Fe;
-    Ps[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+    Ps[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap, Qst + 2 * t) : 0.f;
   }
   __syncthreads();
   // den[t] = phi(q_t) . ksum + eps : one warp per two rows, lanes split f.
@@ -193,6 +229,7 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
                                                         float* __restrict__ out, int H, int N, int D, int F,
                                                         int Fe, int fmap, float eps, int seg, int S) {
   extern __shared__ __align__(16) float dyn[];
+  __shared__ float Qst[2 * kT], Kst[2 * kT];
   float* Qs = dyn;                 // kT * kMaxD
   float* Ks = Qs + kT * kMaxD;
   float* Vs = Ks + kT * kMaxD;
@@ -215,10 +252,15 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
     load_rows(Ks, k + head + static_cast<size_t>(tc) * D, rows, D);
     load_rows(Vs, v + head + static_cast<size_t>(tc) * D, rows, D);
     __syncthreads();
+    if (fmap == 2) {
+      softmax_stats(Qs, D, Qst);
+      softmax_stats(Ks, D, Kst);
+      __syncthreads();
+    }
     for (int e = threadIdx.x; e < kT * Fe; e += blockDim.x) {
       const int t = e / Fe, f = e % Fe;
-      Pq[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
-      Pk[t * kMaxFe + f] = t < rows ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap) : 0.f;
+      Pq[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap, Qst + 2 * t) : 0.f;
+      Pk[t * kMaxFe + f] = t < rows ? feature(Ks + t * kMaxD, D, Wh, F, f, fmap, Kst + 2 * t) : 0.f;
     }
     __syncthreads();
     for (int t = 0; t < rows; ++t) {

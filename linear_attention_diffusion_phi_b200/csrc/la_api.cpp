@@ -67,7 +67,7 @@ bool device_info(DeviceInfo* out) {
 la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap, float eps,
                         int causal) {
   if (B < 0 || H < 0 || N < 0 || D <= 0 || F < 0) return LA_ERR_INVALID_ARG;
-  if (fmap != LA_PHI_ELU1 && fmap != LA_PHI_RELU) return LA_ERR_INVALID_ARG;
+  if (fmap != LA_PHI_ELU1 && fmap != LA_PHI_RELU && fmap != LA_PHI_SOFTMAX) return LA_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || eps != eps) return LA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return LA_ERR_INVALID_ARG;
   if (F % 256 != 0) return LA_ERR_INVALID_ARG;   // feature_dim: a multiple of 256
@@ -80,6 +80,9 @@ la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F,
     if (F != 0 && (F != 256 || D != 128)) return LA_ERR_UNSUPPORTED;
     if (causal && (F != 0 || D != 64)) return LA_ERR_UNSUPPORTED;
   }
+  // softmax over each row's features: fp32 without a projection, and the
+  // bf16 non-causal D = 128 kernel
+  if (fmap == LA_PHI_SOFTMAX && (F != 0 || (h->dtype == LA_BF16 && (causal || D != 128)))) return LA_ERR_UNSUPPORTED;
   return LA_OK;
 }
 
@@ -478,7 +481,7 @@ la_status_t la_forward_e4m3(la_handle_t h, const void* q, const void* k, const v
   const float sc[3] = {scale_q, scale_k, scale_v};
   for (float x : sc)
     if (!(x > 0.f) || !std::isfinite(x)) return LA_ERR_INVALID_ARG;
-  if (h->dtype != LA_BF16 || D != 128) return LA_ERR_UNSUPPORTED;
+  if (h->dtype != LA_BF16 || D != 128 || fmap == LA_PHI_SOFTMAX) return LA_ERR_UNSUPPORTED;
   return forward_impl(h, q, k, v, out, B, H, N, D, 0, fmap, eps, 0, stream, nullptr, 0, sc);
 }
 

@@ -60,9 +60,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" la_status_t la_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H,
                                           int N, int D, int feature_map, float eps, void* stream) {
   if (B < 0 || H < 0 || N < 0 || D <= 0) return LA_ERR_INVALID_ARG;
-  if (feature_map != LA_PHI_ELU1 && feature_map != LA_PHI_RELU) return LA_ERR_INVALID_ARG;
+  if (feature_map != LA_PHI_ELU1 && feature_map != LA_PHI_RELU && feature_map != LA_PHI_SOFTMAX)
+    return LA_ERR_INVALID_ARG;
   if (!(eps >= 0.f)) return LA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+  if (feature_map == LA_PHI_SOFTMAX && D != 128) return LA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return LA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return LA_OK;
   if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;

@@ -79,7 +79,7 @@ def test_forward_argument_validation(handles):
     # bad values
     assert fwd(f32, B=-1) == 1
     assert fwd(f32, D=0) == 1
-    assert fwd(f32, fmap=2) == 1
+    assert fwd(f32, fmap=3) == 1
     assert fwd(f32, eps=-1.0) == 1
     assert fwd(f32, eps=float("nan")) == 1
     assert fwd(f32, causal=2) == 1
@@ -269,3 +269,24 @@ def test_e4m3_argument_checks_on_the_host(handles):
     assert f(handles["bf16"], 128, 1.0, 1.0, 1.0, fmap=7) == la.LA_ERR_INVALID_ARG
     assert la.la_forward_e4m3(handles["bf16"], 0, 0, 0, 1.0, 1.0, 1.0, 0, 0, 2, 256, 128, la.LA_PHI_ELU1,
                               1e-6, None) == la.LA_OK                        # empty problem
+
+
+
+def test_softmax_support_is_checked_on_the_host(handles):
+    """The softmax feature map runs on fp32 without a projection and on the
+    bf16 non-causal D = 128 kernel; every other combination is refused before
+    anything is enqueued."""
+    SMX = la.LA_PHI_SOFTMAX
+    f = lambda h, D, F, causal: la.la_forward(h, 0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, D, F, SMX, 1e-6,
+                                              causal, None)
+    assert f(handles["f32"], 64, 256, 0) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 64, 0, 0) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 128, 0, 1) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 128, 256, 0) == la.LA_ERR_UNSUPPORTED
+    assert la.la_forward_e4m3(handles["bf16"], 0x1000, 0x1000, 0x1000, 1.0, 1.0, 1.0, 0x2000, 1, 2, 256, 128,
+                              SMX, 1e-6, None) == la.LA_ERR_UNSUPPORTED
+    assert la.la_forward_noalloc(0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, 64, SMX, 1e-6,
+                                 None) == la.LA_ERR_UNSUPPORTED
+    assert la.la_forward(handles["bf16"], 0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, 128, 0, 3, 1e-6, 0,
+                         None) == la.LA_ERR_INVALID_ARG
+

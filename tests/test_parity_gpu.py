@@ -97,6 +97,7 @@ F32_CASES = [
     dict(N=1, D=64), dict(N=37, D=4), dict(N=300, D=36, fmap="relu"), dict(N=1000, D=128),
     dict(N=129, D=64, causal=True), dict(N=700, D=128, causal=True, fmap="relu"),
     dict(N=200, D=128, F=256), dict(N=333, D=64, F=256, causal=True),
+    dict(N=257, D=64, fmap="softmax"), dict(N=300, D=128, causal=True, fmap="softmax"),
 ]
 
 
@@ -127,6 +128,8 @@ def test_f32_shared_projection_and_empty_rows():
 BF16_CASES = [
     dict(N=1, D=128), dict(N=127, D=128), dict(N=129, D=128, fmap="relu"), dict(N=300, D=64),
     dict(N=1000, D=64, fmap="relu"), dict(N=4607, D=128), dict(N=2048, D=128, B=3, H=5),
+    dict(N=1, D=128, fmap="softmax"), dict(N=1000, D=128, fmap="softmax"),
+    dict(N=4607, D=128, B=2, H=3, fmap="softmax"),
 ]
 
 
@@ -171,7 +174,7 @@ def test_bf16_deterministic_and_guard_bands():
 
 HEADER_BYTES = 256 + 4096    # workspace header: status word, synchronisation words
 XCHG_CASES = [dict(B=1, H=2, N=4607), dict(B=1, H=1, N=8192, fmap="relu"), dict(B=3, H=3, N=2100),
-              dict(B=1, H=4, N=65536)]
+              dict(B=1, H=4, N=65536), dict(B=1, H=2, N=8000, fmap="softmax")]
 
 
 @pytest.mark.parametrize("case", XCHG_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
@@ -657,3 +660,22 @@ def test_e4m3_equals_bf16_path_on_dequantised_values():
             assert np.array_equal(as_float64(d), s * ora.e4m3_decode(c.numpy()))
         ref = run_gpu(w.with_(dtype="bf16"), *deq)
         assert torch.equal(got[0].view(torch.int16), ref.view(torch.int16)), (fmap, N)
+
+
+# ------------------------------------------------------ softmax feature map --
+
+def test_flux1024_softmax_full():
+    """The flux1024 shape with the softmax feature map, every output element."""
+    check_workload(WORKLOADS["flux1024"].with_(fmap="softmax"), label="flux1024_softmax (all elements)")
+
+
+def test_bf16_softmax_large_inputs():
+    """Rows whose exponentials overflow fp32 without the row maximum taken out
+    (|x| up to about 200), on both feature sides; against the oracle."""
+    w = Workload("smx_large", B=1, H=3, N=700, D=128, fmap="softmax", seed=91)
+    q, k, v, _ = make_inputs(w)
+    q, k = q * 40, k * 40
+    got = run_gpu(w, q, k, v)
+    ref = ora.forward(as_float64(q), as_float64(k), as_float64(v), "softmax", w.eps, False)
+    assert_parity(got, ref, "bf16")
+

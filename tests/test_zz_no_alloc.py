@@ -26,6 +26,7 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
     dev = torch.device("cuda:0")
     s = torch.cuda.current_stream().cuda_stream
     cases = [WORKLOADS["flux1024"], Workload("noalloc_relu64", B=2, H=3, N=1001, D=64, fmap="relu", seed=21),
+             Workload("noalloc_softmax", B=1, H=4, N=3000, D=128, fmap="softmax", seed=22),
              Workload("noalloc_heads", B=3, H=21845, N=3, D=64, seed=22)]   # B*H = 65535
     for w in cases:
         q, k, v, _ = make_inputs(w)
