@@ -80,13 +80,14 @@ def algorithmic_flops(w):
 # device headers it includes) still hashes to what was captured; else null.
 DEVICE_HEADERS = ("bf16_common.cuh", "sm100.cuh")
 NCU_TRAFFIC = {
-    "flux1024": (89_199_616, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
-    "flux2048_cfg": (780_559_872, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
+    "flux1024": (86_117_824, ("bf16_noncausal.cu",), "68a7daf884705de9"),
+    "flux2048_cfg": (780_954_112, ("bf16_noncausal.cu",), "68a7daf884705de9"),
     "causal32k": (716_144_384, ("bf16_causal.cu",), "3e37cbf7e846ccac"),
     "proj256": (99_814_016, ("bf16_proj.cu", "bf16_image.cu"), "4d91d4572082bf07"),
-    "flux1024_ttr": (144_733_952, ("bf16_noncausal.cu", "bf16_landmark.cu"), "10a1909d84b22ba5"),
-    "flux1024_e4m3": (42_692_992, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
-    "flux2048_cfg_e4m3": (460_586_112, ("bf16_noncausal.cu",), "bb70461a15cb9860"),
+    "flux1024_ttr": (144_304_576, ("bf16_noncausal.cu", "bf16_landmark.cu"), "e67d04ea65498457"),
+    "flux1024_e4m3": (42_677_440, ("bf16_noncausal.cu",), "68a7daf884705de9"),
+    "flux2048_cfg_e4m3": (460_428_544, ("bf16_noncausal.cu",), "68a7daf884705de9"),
+    "flux1024_softmax": (85_902_144, ("bf16_noncausal.cu",), "68a7daf884705de9"),
 }
 
 
