@@ -341,3 +341,41 @@ def forward_e4m3(q8, k8, v8, scales, fmap="elu", eps=1e-6):
     sq, sk, sv = (float(x) for x in scales)
     return forward(sq * e4m3_decode(q8), sk * e4m3_decode(k8), sv * e4m3_decode(v8), fmap, eps, causal=False)
 
+
+# --------------------------------------------------------------------------
+# The attention prologue of Flux's block (page "FLUXNATION", section "What it
+# does": QKV split and RoPE fused into the block's kernel).  Readings: the
+# split q and k of a head pass through Flux's QK norm, an RMS norm over the
+# head dimension times a learned per-feature scale, and then the rotary
+# position embedding, which rotates each feature pair (2i, 2i + 1) of the
+# token at position n by the angle whose (cos, sin) is rope[n, i]; v is left
+# as it is.  The layer then runs on the transformed q and k.
+# --------------------------------------------------------------------------
+
+def rms_norm(x, scale, norm_eps):
+    """x / sqrt(mean_d x_d^2 + norm_eps) * scale over the last axis."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + norm_eps) * np.asarray(scale, dtype=np.float64)
+
+
+def rope(x, table):
+    """Rotate pairs (x_2i, x_2i+1) of token n by rope[n, i] = (cos, sin):
+    (c x_2i - s x_2i+1, s x_2i + c x_2i+1).  x [..., N, D], table [N, D/2, 2]."""
+    x = np.asarray(x, dtype=np.float64)
+    t = np.asarray(table, dtype=np.float64)
+    n = x.shape[-2]
+    c, s = t[:n, :, 0], t[:n, :, 1]
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = c * x0 - s * x1
+    out[..., 1::2] = s * x0 + c * x1
+    return out
+
+
+def forward_prologue(q, k, v, q_scale, k_scale, table, norm_eps=1e-6, fmap="elu", eps=1e-6, causal=False):
+    """The layer on rope(rms_norm(q)), rope(rms_norm(k)), v.  Returns float64."""
+    qn = rope(rms_norm(q, q_scale, norm_eps), table)
+    kn = rope(rms_norm(k, k_scale, norm_eps), table)
+    return forward(qn, kn, v, fmap, eps, causal)
+

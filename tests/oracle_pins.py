@@ -509,6 +509,62 @@ def pin_e4m3_forward(ora):
     _close(twice, 2.0 * ora.forward_e4m3(*codes, scales, "elu", 1e-6), rtol=1e-12)
 
 
+
+# ------------------------------------------------ Flux attention prologue --
+
+def _torch_prologue(x, scale, table, norm_eps):
+    """RMS norm by torch's rms_norm and the rotation by complex multiplication
+    (x_2i + i x_2i+1) (cos + i sin): library routines, independent of the oracle."""
+    import torch
+    xt = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    y = torch.nn.functional.rms_norm(xt, (xt.shape[-1],), torch.from_numpy(np.asarray(scale, np.float64)),
+                                     norm_eps).numpy()
+    n = y.shape[-2]
+    z = (y[..., 0::2] + 1j * y[..., 1::2]) * (table[:n, :, 0] + 1j * table[:n, :, 1])
+    out = np.empty_like(y)
+    out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def _rope_table(n, d, rng):
+    ang = rng.uniform(-np.pi, np.pi, size=(n, d // 2))
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+
+
+def pin_prologue_vs_library(ora):
+    """rms_norm is torch's rms_norm, rope is complex multiplication, and the
+    prologue layer is the layer on inputs transformed that way (norm first)."""
+    rng = _rng(61)
+    B, H, N, D = 1, 2, 11, 8
+    q, k, v = (rng.standard_normal((B, H, N, D)) * 2.0 for _ in range(3))
+    qs, ks = 1.0 + 0.3 * rng.standard_normal(D), 1.0 + 0.3 * rng.standard_normal(D)
+    table = _rope_table(N + 3, D, rng)
+    for norm_eps in (1e-6, 0.5):
+        _close(ora.rms_norm(q, qs, norm_eps), _torch_prologue(q, qs, np.stack([np.ones((N, D // 2)),
+                                                                                np.zeros((N, D // 2))], -1),
+                                                             norm_eps), rtol=1e-12)
+        want = ora.forward(_torch_prologue(q, qs, table, norm_eps), _torch_prologue(k, ks, table, norm_eps), v,
+                           "elu", 1e-6)
+        _close(ora.forward_prologue(q, k, v, qs, ks, table, norm_eps, "elu", 1e-6), want, rtol=1e-12)
+    _close(ora.rope(q, table), _torch_prologue(q / np.sqrt(np.mean(q * q, -1, keepdims=True)), np.ones(D),
+                                               table, 0.0) * np.sqrt(np.mean(q * q, -1, keepdims=True)),
+           rtol=1e-10)
+
+
+def pin_rope_invariants(ora):
+    """A zero angle changes nothing, every pair keeps its length, and rotating
+    by the angle then by its negative gives the input back."""
+    rng = _rng(62)
+    x = rng.standard_normal((2, 9, 6))
+    ident = np.stack([np.ones((9, 3)), np.zeros((9, 3))], -1)
+    _close(ora.rope(x, ident), x, rtol=1e-15)
+    t = _rope_table(9, 6, rng)
+    y = ora.rope(x, t)
+    _close(y[..., 0::2] ** 2 + y[..., 1::2] ** 2, x[..., 0::2] ** 2 + x[..., 1::2] ** 2, rtol=1e-12)
+    back = t.copy()
+    back[..., 1] = -back[..., 1]
+    _close(ora.rope(y, back), x, rtol=1e-12, atol=1e-14)
+
 ALL_PINS = [
     pin_feature_maps,
     pin_feature_map_vs_torch,
@@ -534,4 +590,6 @@ ALL_PINS = [
     pin_softmax_vs_scipy,
     pin_softmax_closed_forms,
     pin_softmax_equal_keys,
+    pin_prologue_vs_library,
+    pin_rope_invariants,
 ]

@@ -60,6 +60,13 @@ MUTANTS = [
     ("softmax_not_normalised", "return e / e.sum(axis=-1, keepdims=True)", "return e"),
     ("softmax_wrong_sign", "e = np.exp(x - x.max(axis=-1, keepdims=True))", "e = np.exp(x.max(axis=-1, keepdims=True) - x)"),
     ("softmax_is_elu", "    if fmap == \"softmax\":\n        return phi_softmax(x)", "    if fmap == \"softmax\":\n        return phi_elu1(x)"),
+    ("rms_no_eps", "x / np.sqrt(ms + norm_eps)", "x / np.sqrt(ms)"),
+    ("rms_sum_not_mean", "ms = np.mean(x * x, axis=-1, keepdims=True)", "ms = np.sum(x * x, axis=-1, keepdims=True)"),
+    ("rope_wrong_sign", "out[..., 0::2] = c * x0 - s * x1", "out[..., 0::2] = c * x0 + s * x1"),
+    ("rope_half_split_pairs", "x0, x1 = x[..., 0::2], x[..., 1::2]",
+     "x0, x1 = x[..., : x.shape[-1] // 2], x[..., x.shape[-1] // 2:]"),
+    ("prologue_scales_swapped", "qn = rope(rms_norm(q, q_scale, norm_eps), table)", "qn = rope(rms_norm(q, k_scale, norm_eps), table)"),
+    ("prologue_rope_before_norm", "qn = rope(rms_norm(q, q_scale, norm_eps), table)", "qn = rms_norm(rope(q, table), q_scale, norm_eps)"),
     ("e4m3_bias_eight", "np.exp2(e - 7.0)", "np.exp2(e - 8.0)"),
     ("e4m3_no_subnormals", "np.where(e == 0, (m / 8.0) * 2.0 ** -6,", "np.where(e < 0, (m / 8.0) * 2.0 ** -6,"),
     ("e4m3_subnormal_scale", "(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7"),
