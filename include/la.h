@@ -96,6 +96,29 @@ la_status_t la_destroy(la_handle_t handle);
  * matrix per head, 0 for one matrix shared by all heads.  F must be a positive
  * multiple of 256 (page "Flux2TTRTrainer", "Inputs worth setting").
  * W = NULL unbinds. */
+/* Bind Flux's attention prologue (page "FLUXNATION", "What it does": the
+ * block's QKV split and RoPE fused into its kernel), applied to q and k as
+ * they are loaded by every later la_forward: the QK norm of Flux's block, an
+ * RMS norm over the head dimension times a per-feature scale,
+ *     x_d / sqrt(mean_d' x_d'^2 + norm_eps) * scale_d,
+ * then the rotary embedding, which turns each feature pair (2i, 2i + 1) of the
+ * token at position n by rope[n][i] = (cos, sin):
+ *     (cos x_2i - sin x_2i+1,  sin x_2i + cos x_2i+1).
+ * v is not transformed.  The page names RoPE; the norm is read from the block
+ * it fuses (Flux's attention normalises q and k before the rotation).
+ * q_scale, k_scale: device fp32 [D]; rope: device fp32 [n_positions][D / 2][2]
+ * (cos, sin), positions 0 .. N - 1 used, shared by all batches and heads; all
+ * 16-byte aligned, not copied (they must stay valid while calls that use them
+ * are pending).  D even and > 0, n_positions > 0, norm_eps >= 0 and finite,
+ * else LA_ERR_INVALID_ARG.  q_scale = NULL unbinds.
+ * la_forward then requires the bound D and N <= n_positions
+ * (LA_ERR_INVALID_ARG) and supports: LA_F32 with F = 0, causal or not;
+ * LA_BF16 with D = 128, F = 0, non-causal, feature map elu+1 or relu.  Other
+ * forwards with a prologue bound (other shapes, la_forward_ttr,
+ * la_forward_e4m3) return LA_ERR_UNSUPPORTED. */
+la_status_t la_set_prologue(la_handle_t handle, const float* q_scale, const float* k_scale, const float* rope,
+                            int D, int n_positions, float norm_eps);
+
 la_status_t la_set_projection(la_handle_t handle, const void* W, int H, int D, int F,
                               long long head_stride);
 

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 
 EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
             "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version",
-            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count", "la_forward_e4m3")
+            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count", "la_forward_e4m3", "la_set_prologue")
 
 
 class LAError(RuntimeError):
@@ -62,13 +62,15 @@ def lib():
     L.la_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
     L.la_forward_ttr.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]
     L.la_forward_e4m3.argtypes = [vp, vp, vp, vp, f32, f32, f32, vp, i32, i32, i32, i32, i32, f32, vp]
+    L.la_set_prologue.argtypes = [vp, vp, vp, vp, i32, i32, f32]
     L.la_landmark_count.argtypes = [i32, f32, i32, i32]
     L.la_landmark_count.restype = i32
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_version.argtypes = []
     for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
-                 "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr", "la_forward_e4m3"):
+                 "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr", "la_forward_e4m3",
+                 "la_set_prologue"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -125,6 +127,11 @@ def la_forward_e4m3(handle, q, k, v, scale_q, scale_k, scale_v, out, B, H, N, D,
     """Non-causal forward on E4M3-stored q, k, v with one scale per tensor; out bf16."""
     return lib().la_forward_e4m3(handle, q, k, v, scale_q, scale_k, scale_v, out, B, H, N, D, feature_map, eps,
                                  stream)
+
+
+def la_set_prologue(handle, q_scale, k_scale, rope, D, n_positions, norm_eps):
+    """Bind Flux's attention prologue (QK RMS norm, then the rotary embedding)."""
+    return lib().la_set_prologue(handle, q_scale, k_scale, rope, D, n_positions, norm_eps)
 
 
 def la_landmark_count(N, fraction, min_count, max_count):
@@ -290,6 +297,26 @@ class LinearAttention:
                                   sq, sk, sv, out.data_ptr(), B, H, N, D, self.fmap, self.eps, s),
                   "la_forward_e4m3")
         return out
+
+    def set_prologue(self, q_scale, k_scale, rope, norm_eps=1e-6):
+        """Bind Flux's attention prologue for the following forwards: RMS norm
+        of q and k over the head dimension times ``q_scale`` / ``k_scale``
+        (float32 CUDA tensors [D]), then the rotation of feature pairs by
+        ``rope`` (float32 CUDA tensor [positions, D/2, 2] of cos, sin).
+        ``q_scale=None`` unbinds."""
+        if q_scale is None:
+            check(la_set_prologue(self.handle, None, None, None, 0, 0, 0.0), "la_set_prologue")
+            self._prologue = None
+            return
+        D = q_scale.numel()
+        for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("rope", rope)):
+            if t.dtype != self.torch.float32 or not t.is_contiguous() or t.device.type != "cuda":
+                raise ValueError(f"{name}: expected a contiguous float32 CUDA tensor")
+        if k_scale.numel() != D or rope.dim() != 3 or rope.shape[1:] != (D // 2, 2):
+            raise ValueError("expected q_scale, k_scale [D] and rope [positions, D/2, 2]")
+        check(la_set_prologue(self.handle, q_scale.data_ptr(), k_scale.data_ptr(), rope.data_ptr(), D,
+                              rope.shape[0], float(norm_eps)), "la_set_prologue")
+        self._prologue = (q_scale, k_scale, rope)   # kept alive while bound
 
     def sync_status(self, stream=None):
         dev = self._ws.device if self._ws is not None else self.torch.cuda.current_device()

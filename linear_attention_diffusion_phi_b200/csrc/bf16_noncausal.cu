@@ -613,19 +613,23 @@ __device__ __forceinline__ uint32_t softmax_pair(uint32_t w, float m0, float rz0
 
 // E8: q, k and v are E4M3 codes (tensor maps of bytes, 128 x 128 boxes) with
 // one scale each; out is bf16 as for bf16 inputs.
-template <int FMAP, bool XC, bool E8>
+// PRO: Flux's attention prologue on q and k (RMS norm times the scales pq /
+// pk, then the rotation table rope [positions][64][2]).
+template <int FMAP, bool XC, bool E8, bool PRO>
 __global__ void __launch_bounds__(CfgT::kThreads, 1)
     fused_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                    int* status, uint32_t* sync, uint8_t* xchg, int N, int tiles, float eps, float sq, float sk,
-                   float sv) {
+                   float sv, const float* pq, const float* pk, const float* rope, float neps) {
   using C = CfgT;
   constexpr int D = C::D;
   // Warps that apply phi to the K tiles: with elu+1 (an exponential per
   // element) the combine warps, idle in phase 1, join the eight phi warps;
   // relu is cheap enough for eight.  With E4M3 inputs the combine warps
   // widen the K and V tiles to bf16 in phase 1 instead.
-  constexpr int kKWarps = FMAP == 0 && !E8 ? 16 : 8;
+  // (with the prologue the combine warps normalise and rotate the K tiles
+  // in phase 1, so eight warps apply phi)
+  constexpr int kKWarps = FMAP == 0 && !E8 && !PRO ? 16 : 8;
   // Softmax (FMAP 2): the combine warps compute each K row's maximum and
   // reciprocal exponential sum in phase 1 (kst, a ring over K tiles; kstat
   // when a tile's rows are in), and read the K slot too.
@@ -645,6 +649,8 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
   __shared__ __align__(8) uint64_t landed[C::kRing1], wready[C::kRing1];
   __shared__ __align__(8) uint64_t kstat[kStatRing];
   __shared__ __align__(16) float2 kst[kSmx ? kStatRing * kTileTokens : 1];
+  // PRO: the norm scales of q (0..127) and k (128..255)
+  __shared__ __align__(16) float pscale[PRO ? 2 * D : 4];
   // A buffers in tensor memory, used in turn by the T key tiles and then the
   // T query tiles: written by the phi warps (aready), read by the MMAs (aempty).
   __shared__ __align__(8) uint64_t aready[C::kABufs], aempty[C::kABufs];
@@ -722,6 +728,9 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     comb_flag = 0;
     ep_flag = 0;
   }
+  if constexpr (PRO) {
+    for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) pscale[i] = i < D ? pq[i] : pk[i - D];
+  }
   // B operand of the ksum MMA: a block of bf16 ones (any layout reads 1.0)
   for (int i = threadIdx.x; i < static_cast<int>(C::kOnesBytes / 16); i += blockDim.x)
     *reinterpret_cast<uint4*>(ones + 16 * i) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
@@ -788,7 +797,7 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
     const int lm = lane >> 3, lr = lane & 7;
     for (int t = 0; t < T; ++t) {
       const int s = (2 * t) % C::kRing1, b = t % C::kABufs;
-      if (!warp_wait(E8 ? &wready[s] : &full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
+      if (!warp_wait(E8 || PRO ? &wready[s] : &full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
       const uint32_t base = smem_u32(slot_ptr(s));
       uint32_t x[2][kBlocks][4];
 #pragma unroll
@@ -843,6 +852,36 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       if (lane == 0) mbar_arrive(&aready[b]);
     }
     return true;
+  };
+
+  // PRO: one 16-byte chunk (features 8 c .. 8 c + 7) of the row at token
+  // position pos, times the row's 1 / rms and the feature scales sc, then its
+  // four feature pairs turned by the rotation table; rounded to bf16.
+  auto prologue_chunk = [&](uint4 x, float rinv, const float* sc, int c, int pos) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const float4* rp = reinterpret_cast<const float4*>(rope + (static_cast<size_t>(pos) * (D / 2) + 4 * c) * 2);
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      const float x0 = v2.x * rinv * sc[8 * c + 2 * e], x1 = v2.y * rinv * sc[8 * c + 2 * e + 1];
+      const float4 cs = __ldg(rp + (e >> 1));   // (cos, sin) of pairs 2 (e >> 1) and 2 (e >> 1) + 1
+      const float cn = (e & 1) ? cs.z : cs.x, sn = (e & 1) ? cs.w : cs.y;
+      const __nv_bfloat162 r = __floats2bfloat162_rn(cn * x0 - sn * x1, sn * x0 + cn * x1);
+      o[e] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  // sum of squares of the 8 bf16 values of a chunk
+  auto chunk_ss = [](uint4 x) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      ss = fmaf(v2.x, v2.x, fmaf(v2.y, v2.y, ss));
+    }
+    return ss;
   };
 
   if (warp == 0) {
@@ -930,6 +969,23 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
         if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
 #pragma unroll
         for (int m = 0; m < 4; ++m) e4m3x16_to_bf16(raw[m], sq, x[2 * m], x[2 * m + 1]);
+      } else if constexpr (PRO) {
+        // the row's sum of squares over all 128 features (the other half's
+        // chunks are read for it, before the slot is released)
+        float ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
+          ss += chunk_ss(x[m]) + chunk_ss(*reinterpret_cast<const uint4*>(src + swz_off(i, 8 * (1 - hf) + m)));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfree[s]);   // the Q tile is in registers
+        const int pos = (tile0 + u) * kTileTokens + i;
+        if (pos < N) {   // rows past the sequence end are never stored
+          const float rinv = 1.f / sqrtf(ss * (1.f / D) + neps);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) x[m] = prologue_chunk(x[m], rinv, pscale, 8 * hf + m, pos);
+        }
       } else {
 #pragma unroll
         for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4*>(src + swz_off(i, 8 * hf + m));
@@ -1062,7 +1118,41 @@ __global__ void __launch_bounds__(CfgT::kThreads, 1)
       }
       return true;
     };
-    bool got = E8 ? widen() : (kSmx ? kstats() : (kKWarps == 16 ? k_phase() : true));
+    // PRO: every K tile normalised and rotated in place before the phi warps
+    // read it: warp w takes rows 16 w .. 16 w + 15, eight lanes per row (two
+    // chunks each, features 16 c .. 16 c + 15), the row's sum of squares over
+    // the eight lanes by shuffles; each warp arrives on wready.
+    auto kprologue = [&]() {
+      const int w8 = warp - C::kCombWarp0, c = lane & 7;
+      for (int t = 0; t < T; ++t) {
+        const int s = (2 * t) % C::kRing1;
+        if (!warp_wait(&full[s], ((2 * t) / C::kRing1) & 1, status)) return false;
+        uint8_t* slot = slot_ptr(s);
+#pragma unroll 1
+        for (int r = 0; r < 4; ++r) {
+          const int row = 16 * w8 + 4 * r + (lane >> 3);
+          uint4 a = *reinterpret_cast<const uint4*>(slot + swz_off(row, 2 * c));
+          uint4 b = *reinterpret_cast<const uint4*>(slot + swz_off(row, 2 * c + 1));
+          float ss = chunk_ss(a) + chunk_ss(b);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+          const int pos = (tile0 + t) * kTileTokens + row;
+          if (pos < N) {   // rows past the sequence end are masked to zero later
+            const float rinv = 1.f / sqrtf(ss * (1.f / D) + neps);
+            a = prologue_chunk(a, rinv, pscale + D, 2 * c, pos);
+            b = prologue_chunk(b, rinv, pscale + D, 2 * c + 1, pos);
+            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c)) = a;
+            *reinterpret_cast<uint4*>(slot + swz_off(row, 2 * c + 1)) = b;
+          }
+        }
+        fence_proxy_async_smem();   // TMA refills the slot later
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wready[s]);
+      }
+      return true;
+    };
+    bool got = E8 ? widen() : (kSmx ? kstats() : (PRO ? kprologue() : (kKWarps == 16 ? k_phase() : true)));
     auto sync_ok = [&](bool mine) {
       if (leader && !mine) comb_flag = 1;
       named_bar_sync(3, 256);
@@ -1369,7 +1459,7 @@ int pick_cluster(const void* kern, uint32_t smem, int threads, long long BH, int
 // it only pays where one cluster per head would use few SMs (few heads).
 // Heads that outnumber the SMs run one CTA each, in waves.
 void geometry_t(long long BH, int tiles, int num_sms, int* P_out, int* S_out) {
-  const void* kern = reinterpret_cast<const void*>(fused_t_kernel<0, false, false>);
+  const void* kern = reinterpret_cast<const void*>(fused_t_kernel<0, false, false, false>);
   const int s1 = pick_cluster(kern, CfgT::kSmemBytes, CfgT::kThreads, BH, tiles);
   *P_out = s1;
   *S_out = s1;
@@ -1410,7 +1500,7 @@ cudaError_t launch_fused(const LaunchArgs& a, Kern kern, int P, int S, uint32_t*
   int* status = reinterpret_cast<int*>(a.ws + p.off_status);
   if constexpr (std::is_same<C, CfgT>::value)
     return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, sync, xchg, p.N, p.tiles,
-                              p.eps, a.scale_q, a.scale_k, a.scale_v);
+                              p.eps, a.scale_q, a.scale_k, a.scale_v, a.pro_q, a.pro_k, a.pro_rope, a.pro_eps);
   else
     return cudaLaunchKernelEx(&cfg, kern, *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, status, p.N, p.tiles, p.eps);
 }
@@ -1438,25 +1528,33 @@ cudaError_t launch_bf16_noncausal(const LaunchArgs& a) {
   uint8_t* xchg = reinterpret_cast<uint8_t*>(a.ws + p.off_xchg);
   const int P = p.ctas_per_head, S = p.cluster;
   if (p.D == 128) {
+    if (a.prologue) {
+      if (a.e4m3 || p.fmap == 2) return cudaErrorNotSupported;
+      if (P > S)
+        return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, false, true>, P, S, sync, xchg)
+                           : launch_fused<CfgT>(a, fused_t_kernel<1, true, false, true>, P, S, sync, xchg);
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, false, true>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, false, false, true>, P, S, sync, xchg);
+    }
     if (p.fmap == 2) {
       if (a.e4m3) return cudaErrorNotSupported;
-      return P > S ? launch_fused<CfgT>(a, fused_t_kernel<2, true, false>, P, S, sync, xchg)
-                   : launch_fused<CfgT>(a, fused_t_kernel<2, false, false>, P, S, sync, xchg);
+      return P > S ? launch_fused<CfgT>(a, fused_t_kernel<2, true, false, false>, P, S, sync, xchg)
+                   : launch_fused<CfgT>(a, fused_t_kernel<2, false, false, false>, P, S, sync, xchg);
     }
     if (a.e4m3) {
       if (P > S)
-        return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, true>, P, S, sync, xchg)
-                           : launch_fused<CfgT>(a, fused_t_kernel<1, true, true>, P, S, sync, xchg);
-      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, true>, P, S, sync, xchg)
-                         : launch_fused<CfgT>(a, fused_t_kernel<1, false, true>, P, S, sync, xchg);
+        return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, true, false>, P, S, sync, xchg)
+                           : launch_fused<CfgT>(a, fused_t_kernel<1, true, true, false>, P, S, sync, xchg);
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, true, false>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, false, true, false>, P, S, sync, xchg);
     }
     if (P > S)
-      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, false>, P, S, sync, xchg)
-                         : launch_fused<CfgT>(a, fused_t_kernel<1, true, false>, P, S, sync, xchg);
-    return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, false>, P, S, sync, xchg)
-                       : launch_fused<CfgT>(a, fused_t_kernel<1, false, false>, P, S, sync, xchg);
+      return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, true, false, false>, P, S, sync, xchg)
+                         : launch_fused<CfgT>(a, fused_t_kernel<1, true, false, false>, P, S, sync, xchg);
+    return p.fmap == 0 ? launch_fused<CfgT>(a, fused_t_kernel<0, false, false, false>, P, S, sync, xchg)
+                       : launch_fused<CfgT>(a, fused_t_kernel<1, false, false, false>, P, S, sync, xchg);
   }
-  if (a.e4m3 || p.fmap == 2) return cudaErrorNotSupported;
+  if (a.e4m3 || p.fmap == 2 || a.prologue) return cudaErrorNotSupported;
   if (p.D == 64)
     return p.fmap == 0 ? launch_fused<Cfg<64>>(a, fused_kernel<64, 0>, P, S, sync, xchg)
                        : launch_fused<Cfg<64>>(a, fused_kernel<64, 1>, P, S, sync, xchg);

@@ -60,6 +60,33 @@ __device__ void softmax_stats(const float* xs, int D, float* st) {
   }
 }
 
+// Flux's attention prologue on the first `rows` rows of xs [kT][kMaxD] (token
+// positions t0 + t): x_d / sqrt(mean x^2 + neps) * scale_d, then each pair
+// (2i, 2i + 1) turned by rope[t0 + t][i] = (cos, sin).  One warp per row.
+struct Prologue {
+  const float* scale;   // [D]; nullptr: no prologue
+  const float* rope;    // [positions][D / 2][2]
+  float eps;
+};
+__device__ void prologue_rows(float* xs, int rows, int D, int t0, Prologue pr) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int t = warp; t < rows; t += blockDim.x / 32) {
+    float* x = xs + t * kMaxD;
+    float ss = 0.f;
+    for (int d = lane; d < D; d += 32) ss = fmaf(x[d], x[d], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = 1.f / sqrtf(ss / static_cast<float>(D) + pr.eps);
+    const float* rp = pr.rope + static_cast<size_t>(t0 + t) * D;
+    for (int i = lane; i < D / 2; i += 32) {
+      const float x0 = x[2 * i] * r * __ldg(pr.scale + 2 * i), x1 = x[2 * i + 1] * r * __ldg(pr.scale + 2 * i + 1);
+      const float c = __ldg(rp + 2 * i), sn = __ldg(rp + 2 * i + 1);
+      x[2 * i] = c * x0 - sn * x1;
+      x[2 * i + 1] = sn * x0 + c * x1;
+    }
+  }
+}
+
 __device__ __forceinline__ void load_rows(float* dst, const float* src, int rows_valid, int D) {
   // dst[kT][kMaxD]; rows >= rows_valid are zero-filled.  D % 4 == 0.
   const int d4 = D / 4;
@@ -77,7 +104,7 @@ __global__ void __launch_bounds__(256) f32_state_partial(const float* __restrict
                                                          const float* __restrict__ W, long long wstride,
                                                          float* __restrict__ part, float* __restrict__ part_ksum,
                                                          int H, int N, int D, int F, int Fe, int fmap, int seg,
-                                                         int S) {
+                                                         int S, Prologue pk) {
   __shared__ __align__(16) float Ks[kT * kMaxD];
   __shared__ __align__(16) float Vs[kT * kMaxD];
   __shared__ float Ps[kT * kFB];
@@ -99,6 +126,10 @@ __global__ void __launch_bounds__(256) f32_state_partial(const float* __restrict
     load_rows(Ks, kh + static_cast<size_t>(tc) * D, rows, D);
     load_rows(Vs, vh + static_cast<size_t>(tc) * D, rows, D);
     __syncthreads();
+    if (pk.scale) {
+      prologue_rows(Ks, rows, D, tc, pk);
+      __syncthreads();
+    }
     if (fmap == 2) {
       softmax_stats(Ks, D, Kst);
       __syncthreads();
@@ -177,7 +208,8 @@ __global__ void f32_state_scan(float* __restrict__ part, float* __restrict__ par
 __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, const float* __restrict__ W,
                                                  long long wstride, const float* __restrict__ fin,
                                                  const float* __restrict__ fin_ksum, float* __restrict__ out,
-                                                 int H, int N, int D, int F, int Fe, int fmap, float eps) {
+                                                 int H, int N, int D, int F, int Fe, int fmap, float eps,
+                                                 Prologue pq) {
   __shared__ __align__(16) float Qs[kT * kMaxD];
   __shared__ float Ps[kT * kMaxFe];
   __shared__ float den[kT];
@@ -190,6 +222,10 @@ __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, co
   const float* ksum = fin_ksum + static_cast<size_t>(bh) * Fe;
   load_rows(Qs, q + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
   __syncthreads();
+  if (pq.scale) {
+    prologue_rows(Qs, rows, D, t0, pq);
+    __syncthreads();
+  }
   if (fmap == 2) {
     softmax_stats(Qs, D, Qst);
     __syncthreads();
@@ -227,7 +263,8 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
                                                         long long wstride, const float* __restrict__ pre,
                                                         const float* __restrict__ pre_ksum,
                                                         float* __restrict__ out, int H, int N, int D, int F,
-                                                        int Fe, int fmap, float eps, int seg, int S) {
+                                                        int Fe, int fmap, float eps, int seg, int S, Prologue pq,
+                                                        Prologue pk) {
   extern __shared__ __align__(16) float dyn[];
   __shared__ float Qst[2 * kT], Kst[2 * kT];
   float* Qs = dyn;                 // kT * kMaxD
@@ -252,6 +289,11 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
     load_rows(Ks, k + head + static_cast<size_t>(tc) * D, rows, D);
     load_rows(Vs, v + head + static_cast<size_t>(tc) * D, rows, D);
     __syncthreads();
+    if (pq.scale) {
+      prologue_rows(Qs, rows, D, tc, pq);
+      prologue_rows(Ks, rows, D, tc, pk);
+      __syncthreads();
+    }
     if (fmap == 2) {
       softmax_stats(Qs, D, Qst);
       softmax_stats(Ks, D, Kst);
@@ -299,8 +341,10 @@ cudaError_t launch_f32(const LaunchArgs& a) {
   const int n_state = p.Fe * p.D + p.Fe;
 
   dim3 g1(S, static_cast<unsigned>(p.BH), (p.Fe + kFB - 1) / kFB);
+  const Prologue pq = {a.prologue ? a.pro_q : nullptr, a.pro_rope, a.pro_eps};
+  const Prologue pk = {a.prologue ? a.pro_k : nullptr, a.pro_rope, a.pro_eps};
   f32_state_partial<<<g1, 256, 0, a.stream>>>(k, v, W, a.w_head_stride, part, part_ksum, p.H, p.N, p.D, p.F, p.Fe,
-                                              p.fmap, p.seg_len, S);
+                                              p.fmap, p.seg_len, S, pk);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   dim3 g2(static_cast<unsigned>(p.BH), (n_state + 255) / 256);
@@ -311,7 +355,7 @@ cudaError_t launch_f32(const LaunchArgs& a) {
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     dim3 g3((p.N + kT - 1) / kT, static_cast<unsigned>(p.BH));
     f32_apply<<<g3, 256, 0, a.stream>>>(q, W, a.w_head_stride, fin, fin_ksum, out, p.H, p.N, p.D, p.F, p.Fe, p.fmap,
-                                        p.eps);
+                                        p.eps, pq);
     return cudaGetLastError();
   }
   f32_state_scan<<<g2, 256, 0, a.stream>>>(part, part_ksum, p.Fe, p.D, S);
@@ -322,7 +366,7 @@ cudaError_t launch_f32(const LaunchArgs& a) {
   if (err != cudaSuccess) return err;
   dim3 g3(S, static_cast<unsigned>(p.BH));
   f32_causal_apply<<<g3, 256, dyn, a.stream>>>(q, k, v, W, a.w_head_stride, part, part_ksum, out, p.H, p.N, p.D, p.F,
-                                               p.Fe, p.fmap, p.eps, p.seg_len, S);
+                                               p.Fe, p.fmap, p.eps, p.seg_len, S, pq, pk);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,12 @@ struct la_handle_s {
   const void* W;
   int wH, wD, wF;
   long long w_head_stride;
+  // attention prologue (la_set_prologue); pro_q == nullptr: none
+  const float* pro_q;
+  const float* pro_k;
+  const float* pro_rope;
+  int pro_D, pro_npos;
+  float pro_eps;
   void* ws;
   size_t ws_bytes;
   // The status word of a newly bound workspace is cleared by the next call
@@ -320,6 +326,26 @@ la_status_t la_destroy(la_handle_t handle) {
   return LA_OK;
 }
 
+la_status_t la_set_prologue(la_handle_t h, const float* q_scale, const float* k_scale, const float* rope, int D,
+                            int n_positions, float norm_eps) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  if (!q_scale) {
+    h->pro_q = h->pro_k = h->pro_rope = nullptr;
+    h->pro_D = h->pro_npos = 0;
+    return LA_OK;
+  }
+  if (!k_scale || !rope || D <= 0 || D % 2 != 0 || n_positions <= 0) return LA_ERR_INVALID_ARG;
+  if (!(norm_eps >= 0.f) || !std::isfinite(norm_eps)) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q_scale) || !aligned16(k_scale) || !aligned16(rope)) return LA_ERR_MISALIGNED;
+  h->pro_q = q_scale;
+  h->pro_k = k_scale;
+  h->pro_rope = rope;
+  h->pro_D = D;
+  h->pro_npos = n_positions;
+  h->pro_eps = norm_eps;
+  return LA_OK;
+}
+
 la_status_t la_set_projection(la_handle_t h, const void* W, int H, int D, int F, long long head_stride) {
   if (!h) return LA_ERR_INVALID_ARG;
   if (!W) {
@@ -385,6 +411,13 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
     if (!h->W) return LA_ERR_INVALID_ARG;
     if (h->wD != D || h->wF != F || (h->w_head_stride != 0 && h->wH < H)) return LA_ERR_INVALID_ARG;
   }
+  const bool pro = h->pro_q != nullptr;
+  if (pro) {
+    if (h->pro_D != D || N > h->pro_npos) return LA_ERR_INVALID_ARG;
+    const bool fits = F == 0 && !gate && !scales &&
+                      (h->dtype == LA_F32 || (D == 128 && !causal && fmap != LA_PHI_SOFTMAX));
+    if (!fits) return LA_ERR_UNSUPPORTED;
+  }
   // The kernels write out and the workspace while q, k, v and W are still
   // being read, so neither may share a byte with them or with each other; q,
   // k and v are only read and may coincide.
@@ -401,6 +434,12 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
       if (h->ws && la::overlap(h->ws, h->ws_bytes, x, nin)) return LA_ERR_INVALID_ARG;
     }
     if (F > 0 && la::overlap(out, nb, h->W, wb)) return LA_ERR_INVALID_ARG;
+    if (pro) {   // out is written while the prologue's scales and table are read
+      const size_t sb = static_cast<size_t>(D) * 4, rb = static_cast<size_t>(h->pro_npos) * D * 4;
+      if (la::overlap(out, nb, h->pro_q, sb) || la::overlap(out, nb, h->pro_k, sb) ||
+          la::overlap(out, nb, h->pro_rope, rb))
+        return LA_ERR_INVALID_ARG;
+    }
     if (h->ws && (la::overlap(h->ws, h->ws_bytes, out, nb) || (F > 0 && la::overlap(h->ws, h->ws_bytes, h->W, wb))))
       return LA_ERR_INVALID_ARG;
   }
@@ -412,6 +451,9 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   if (!h->ws || h->ws_bytes < p.bytes) return LA_ERR_WORKSPACE;
   if (!la::on_current_device(q) || !la::on_current_device(k) || !la::on_current_device(v) ||
       !la::on_current_device(out) || !la::on_current_device(h->ws) || (F > 0 && !la::on_current_device(h->W)))
+    return LA_ERR_INVALID_ARG;
+  if (pro && (!la::on_current_device(h->pro_q) || !la::on_current_device(h->pro_k) ||
+              !la::on_current_device(h->pro_rope)))
     return LA_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (h->ws_clear_pending) {
@@ -429,6 +471,11 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   a.w_head_stride = h->w_head_stride;
   a.ws = static_cast<char*>(h->ws);
   a.stream = cs;
+  a.prologue = pro;
+  a.pro_q = h->pro_q;
+  a.pro_k = h->pro_k;
+  a.pro_rope = h->pro_rope;
+  a.pro_eps = h->pro_eps;
 
   cudaError_t err;
   if (h->dtype == LA_F32) {

@@ -64,6 +64,14 @@ struct LaunchArgs {
   // bytes), dequantised as scale x code value; out stays bf16
   bool e4m3;
   float scale_q, scale_k, scale_v;
+  // Flux's attention prologue on q and k (la_set_prologue): RMS norm with the
+  // scales pro_q / pro_k (fp32 [D]), then the rotation table pro_rope (fp32
+  // [positions][D / 2][2], cos and sin)
+  bool prologue;
+  const float* pro_q;
+  const float* pro_k;
+  const float* pro_rope;
+  float pro_eps;
 };
 
 // Host helpers defined in la_api.cpp for other host translation units.

@@ -117,3 +117,20 @@ def make_e4m3_inputs(w: Workload, seed=None):
         scales.append(s)
     return codes[0], codes[1], codes[2], tuple(scales)
 
+
+def make_prologue_params(w: Workload, seed=None, base=10000.0):
+    """Parameters of Flux's attention prologue for workload w, as float32 CPU
+    torch tensors: (q_scale [D], k_scale [D], rope [N, D/2, 2]).
+
+    The norm scales are 1 + 0.1 N(0, 1) draws; the rotation table holds
+    (cos, sin) of the angles n base^(-2 i / D) of the usual rotary frequencies,
+    evaluated in float64 and stored as float32.
+    """
+    import torch
+    rng = np.random.default_rng((w.seed if seed is None else seed) + 40009)
+    qs = (1.0 + 0.1 * rng.standard_normal(w.D)).astype(np.float32)
+    ks = (1.0 + 0.1 * rng.standard_normal(w.D)).astype(np.float32)
+    ang = np.arange(w.N, dtype=np.float64)[:, None] * base ** (-2.0 * np.arange(w.D // 2) / w.D)[None, :]
+    rope = np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+    return torch.from_numpy(qs), torch.from_numpy(ks), torch.from_numpy(np.ascontiguousarray(rope))
+

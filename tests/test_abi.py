@@ -290,3 +290,30 @@ def test_softmax_support_is_checked_on_the_host(handles):
     assert la.la_forward(handles["bf16"], 0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, 128, 0, 3, 1e-6, 0,
                          None) == la.LA_ERR_INVALID_ARG
 
+
+def test_prologue_binding_and_support_checks(handles):
+    """la_set_prologue checks its arguments; la_forward with a prologue bound
+    refuses other shapes and paths before anything is enqueued."""
+    f = lambda h, D=128, npos=256, eps=1e-6, qs=0x1000, ks=0x2000, rope=0x3000: la.la_set_prologue(
+        h, qs, ks, rope, D, npos, eps)
+    bf = handles["bf16"]
+    assert f(bf, D=127) == la.LA_ERR_INVALID_ARG
+    assert f(bf, npos=0) == la.LA_ERR_INVALID_ARG
+    assert f(bf, eps=-1.0) == la.LA_ERR_INVALID_ARG
+    assert f(bf, ks=None) == la.LA_ERR_INVALID_ARG
+    assert f(bf, rope=0x3004) == la.LA_ERR_MISALIGNED
+    assert f(bf) == la.LA_OK
+    fwd = lambda h, D=128, N=256, causal=0, fmap=la.LA_PHI_ELU1: la.la_forward(
+        h, 0x10000, 0x10000, 0x10000, 0x20000, 1, 2, N, D, 0, fmap, 1e-6, causal, None)
+    assert fwd(bf, N=257) == la.LA_ERR_INVALID_ARG                 # more positions than the table
+    assert fwd(bf, causal=1, D=128) == la.LA_ERR_UNSUPPORTED
+    assert fwd(bf, fmap=la.LA_PHI_SOFTMAX) == la.LA_ERR_UNSUPPORTED
+    assert la.la_forward_e4m3(bf, 0x10000, 0x10000, 0x10000, 1.0, 1.0, 1.0, 0x20000, 1, 2, 256, 128,
+                              la.LA_PHI_ELU1, 1e-6, None) == la.LA_ERR_UNSUPPORTED
+    assert la.la_forward_ttr(bf, 0x10000, 0x10000, 0x10000, 0x20000, 1, 2, 256, 128, 0, la.LA_PHI_ELU1, 1e-6, 8,
+                             0x80000, None) == la.LA_ERR_UNSUPPORTED
+    assert f(bf, D=64) == la.LA_OK
+    assert fwd(bf, D=128) == la.LA_ERR_INVALID_ARG                 # the bound D differs
+    assert fwd(bf, D=64) == la.LA_ERR_UNSUPPORTED                  # bf16 prologue needs D = 128
+    assert la.la_set_prologue(bf, None, None, None, 0, 0, 0.0) == la.LA_OK
+

@@ -10,7 +10,8 @@ import pytest
 
 import linear_attention_diffusion_phi_b200 as la
 from linear_attention_diffusion_phi_b200 import build as la_build
-from linear_attention_diffusion_phi_b200.inputs import WORKLOADS, Workload, as_float64, make_e4m3_inputs, make_inputs
+from linear_attention_diffusion_phi_b200.inputs import (WORKLOADS, Workload, as_float64, make_e4m3_inputs, make_inputs,
+                                                        make_prologue_params)
 from oracle import la_oracle as ora
 
 pytestmark = pytest.mark.gpu
@@ -678,4 +679,45 @@ def test_bf16_softmax_large_inputs():
     got = run_gpu(w, q, k, v)
     ref = ora.forward(as_float64(q), as_float64(k), as_float64(v), "softmax", w.eps, False)
     assert_parity(got, ref, "bf16")
+
+
+# ------------------------------------------------- Flux attention prologue --
+
+PRO_CASES = [
+    dict(B=1, H=2, N=300, D=64, dtype="f32"),
+    dict(B=1, H=2, N=257, D=128, dtype="f32", causal=True, fmap="relu"),
+    dict(B=1, H=2, N=1, D=128),
+    dict(B=1, H=3, N=1000, D=128, fmap="relu"),
+    dict(B=2, H=3, N=4607, D=128),
+    dict(B=1, H=2, N=8000, D=128),      # heads over several clusters
+]
+
+
+def run_prologue(w, norm_eps=1e-6):
+    import torch
+    q, k, v, _ = make_inputs(w)
+    qs, ks, rope = make_prologue_params(w)
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch_dtype(w), w.fmap, w.eps, w.causal)
+    op.set_prologue(qs.to(dev), ks.to(dev), rope.to(dev), norm_eps)
+    got = op(q.to(dev), k.to(dev), v.to(dev)).cpu()
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    op.close()
+    ref = ora.forward_prologue(as_float64(q), as_float64(k), as_float64(v), qs.numpy(), ks.numpy(), rope.numpy(),
+                               norm_eps, w.fmap, w.eps, w.causal)
+    return got, ref
+
+
+@pytest.mark.parametrize("case", PRO_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_prologue_shapes(case):
+    w = Workload("prologue_case", seed=2300 + case["N"], **case)
+    got, ref = run_prologue(w)
+    assert_parity(got, ref, w.dtype)
+
+
+def test_flux1024_prologue_full():
+    w = WORKLOADS["flux1024"]
+    got, ref = run_prologue(w)
+    assert_parity(got, ref, "bf16", "flux1024_prologue (all elements)")
 
