@@ -348,7 +348,7 @@ def parity_samples(w):
     return [(b, h, sl) for b, h in heads[:2]]
 
 
-def parity_block(w, q, k, v, W, got, ttr=None, e4m3=False):
+def parity_block(w, q, k, v, W, got, ttr=None, e4m3=False, prologue=None):
     """Error figures of the GPU output `got` against the float64 oracle on
     the sampled heads / rows (CPU torch tensors of the stored values); with
     `ttr` = (landmark count, logits), against the oracle's TTR layer; with
@@ -367,6 +367,10 @@ def parity_block(w, q, k, v, W, got, ttr=None, e4m3=False):
         if ttr is not None:
             ref = ora.ttr_forward(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1],
                                   [ttr[1][h]], ttr[0], w.fmap, w.eps, Wh)[0, 0]
+        elif prologue is not None:
+            qs, ks, rope = (t.numpy() for t in prologue)
+            ref = ora.forward_prologue(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1], qs, ks, rope,
+                                       1e-6, w.fmap, w.eps, w.causal)[0, 0]
         elif rows is None:
             ref = ora.forward(qf[b:b + 1, h:h + 1], kf[b:b + 1, h:h + 1], vf[b:b + 1, h:h + 1], w.fmap, w.eps,
                               w.causal, Wh)[0, 0]
@@ -402,7 +406,7 @@ class Timed:
     shifted along the sequence, so every step reads memory the previous steps
     did not touch), the operator, and CUDA graphs of its steps."""
 
-    def __init__(self, w, dev, rank, graphs=True, ttr=None, e4m3=False):
+    def __init__(self, w, dev, rank, graphs=True, ttr=None, e4m3=False, prologue=False):
         import torch
         import linear_attention_diffusion_phi_b200 as la
         from linear_attention_diffusion_phi_b200.inputs import make_e4m3_inputs, make_inputs
@@ -431,6 +435,12 @@ class Timed:
             sh = (97 * i) % max(w.N, 1)
             self.sets.append(tuple(torch.roll(x, shifts=sh, dims=2) for x in base) + (new_out(),))
         self.op = la.LinearAttention(dt, w.fmap, w.eps, w.causal, None if W is None else W.to(dev))
+        # prologue: Flux's QK norm and rotary embedding ahead of the layer
+        self.pro_host = None
+        if prologue:
+            from linear_attention_diffusion_phi_b200.inputs import make_prologue_params
+            self.pro_host = make_prologue_params(w)
+            self.op.set_prologue(*(t.to(dev) for t in self.pro_host))
         self.graphs = graphs
         self.g_all = None
         self.g_all_steps = 0
@@ -562,7 +572,7 @@ def roofline_e4m3(w, per_step_s, hbm, src, name):
 
 
 EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr", "flux1024_e4m3", "flux2048_cfg_e4m3",
-                   "flux1024_softmax")
+                   "flux1024_softmax", "flux1024_prologue")
 # The TTR layer on the flux1024 shape: 128 landmarks (the page's knobs at
 # fraction 1/32, min 16, max 128) and one logit per head, spread over [-2, 2].
 TTR_LANDMARKS = (1 / 32, 16, 128)
@@ -583,11 +593,14 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
     ttr = name.endswith("_ttr")
     e8 = name.endswith("_e4m3")
     smx = name.endswith("_softmax")   # the same shapes with the softmax feature map
-    x = WORKLOADS[name[:-4] if ttr else (name[:-5] if e8 else (name[:-8] if smx else name))]
+    pro = name.endswith("_prologue")  # the same shapes behind Flux's attention prologue
+    base = name[:-4] if ttr else (name[:-5] if e8 else (name[:-8] if smx else (name[:-9] if pro else name)))
+    x = WORKLOADS[base]
     if smx:
         x = x.with_(fmap="softmax")
     try:
-        tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8)
+        tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8,
+                   prologue=pro)
         xsteps = max(args.steps, 100)
         tx.steps_hint = xsteps
         smp = ClockSampler(local)
@@ -607,8 +620,10 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
             xroof["landmarks"], xroof["gates"] = tx.ttr[0], "linspace(-2, 2, H)"
         if e8:
             xroof = roofline_e4m3(x, xms / 1e3 / xsteps, hbm, src, name)
-        if smx:
+        if smx or pro:
             xroof["traffic"] = captured_traffic(x, name)
+        if pro:
+            xroof["kernel"] = "fused_t_kernel with the prologue (one cluster launch per step)"
         ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
                "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
                "ms_per_step": xms / xsteps,
@@ -616,7 +631,7 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
                "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
                "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
         if not args.no_parity:
-            ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8)
+            ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8, prologue=tx.pro_host)
         tx.close()
         del tx
     except Exception as e:   # an extra figure never costs the headline line
