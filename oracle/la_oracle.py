@@ -379,3 +379,59 @@ def forward_prologue(q, k, v, q_scale, k_scale, table, norm_eps=1e-6, fmap="elu"
     kn = rope(rms_norm(k, k_scale, norm_eps), table)
     return forward(qn, kn, v, fmap, eps, causal)
 
+
+# --------------------------------------------------------------------------
+# Backward pass of the non-causal layer (page "Flux2TTRTrainer", "How the
+# distillation works": the student layer is trained by distillation, which
+# needs the gradients of the loss with respect to q, k and v).  For a loss L
+# with dL/dout = dout, per head with F = D features:
+#   den_i = phi(q_i).z + eps, out_i = phi(q_i) kv / den_i,
+#   g_i = dout_i / den_i,  h_i = -(dout_i . out_i) / den_i,
+#   dphi(q_i) = kv g_i + h_i z,   dkv = sum_i phi(q_i) g_i^T,   dz = sum_i h_i phi(q_i),
+#   dphi(k_j) = dkv v_j + dz,     dv_j = dkv^T phi(k_j),
+# and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k) elementwise.
+# --------------------------------------------------------------------------
+
+def feature_map_grad(x, fmap):
+    """phi'(x) elementwise: elu(x)+1 -> 1 for x > 0, exp(x) otherwise; relu ->
+    1 for x > 0, 0 otherwise (0 at x = 0)."""
+    x = np.asarray(x, dtype=np.float64)
+    if fmap == "elu":
+        return np.where(x > 0.0, 1.0, np.exp(np.minimum(x, 0.0)))
+    if fmap == "relu":
+        return np.where(x > 0.0, 1.0, 0.0)
+    raise ValueError(f"no gradient for feature map {fmap!r}")
+
+
+def backward_head(q, k, v, dout, fmap, eps):
+    """(dq, dk, dv) of one non-causal head without projection, float64."""
+    q, k, v, dout = (np.asarray(a, dtype=np.float64) for a in (q, k, v, dout))
+    pq, pk = feature_map(q, fmap), feature_map(k, fmap)
+    kv = pk.T @ v
+    z = pk.sum(axis=0)
+    den = pq @ z + eps
+    out = (pq @ kv) / den[:, None]
+    g = dout / den[:, None]
+    h = -(dout * out).sum(axis=1) / den
+    dpq = g @ kv.T + h[:, None] * z[None, :]
+    dkv = pq.T @ g
+    dz = pq.T @ h
+    dpk = v @ dkv.T + dz[None, :]
+    dv = pk @ dkv
+    return dpq * feature_map_grad(q, fmap), dpk * feature_map_grad(k, fmap), dv
+
+
+def backward(q, k, v, dout, fmap="elu", eps=1e-6):
+    """Gradients (dq, dk, dv) of sum(out * dout) over all heads, non-causal,
+    no projection; float64 [B, H, N, D] each."""
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    _check(q, k, v, fmap, eps)
+    if fmap not in ("elu", "relu"):
+        raise ValueError("backward: elu or relu feature maps")
+    dout = np.asarray(dout, dtype=np.float64)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            dq[b, h], dk[b, h], dv[b, h] = backward_head(q[b, h], k[b, h], v[b, h], dout[b, h], fmap, eps)
+    return dq, dk, dv
+

@@ -565,6 +565,53 @@ def pin_rope_invariants(ora):
     back[..., 1] = -back[..., 1]
     _close(ora.rope(y, back), x, rtol=1e-12, atol=1e-14)
 
+
+# ------------------------------------------------------------ backward pass --
+
+def pin_backward_finite_differences(ora):
+    """Each gradient entry equals the central difference of sum(out * dout)
+    computed with the definition (brute force), for elu and relu, at points
+    away from relu's kink."""
+    rng = _rng(71)
+    B, H, N, D = 1, 2, 5, 3
+    q, k, v, dout = (rng.standard_normal((B, H, N, D)) for _ in range(4))
+    for fmap in ("elu", "relu"):
+        if fmap == "relu":   # keep every entry away from 0
+            q = np.where(np.abs(q) < 0.2, q + np.sign(q + 1e-9) * 0.3, q)
+            k = np.where(np.abs(k) < 0.2, k + np.sign(k + 1e-9) * 0.3, k)
+        eps = 0.3
+        grads = ora.backward(q, k, v, dout, fmap, eps)
+        loss = lambda qq, kk, vv: float((ora.brute_force(qq, kk, vv, fmap, eps) * dout).sum())
+        step = 1e-6
+        for which, g in enumerate(grads):
+            for idx in [(0, 0, 0, 0), (0, 1, 3, 2), (0, 0, 4, 1), (0, 1, 2, 0)]:
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += step
+                up = loss(*args)
+                args[which][idx] -= 2 * step
+                dn = loss(*args)
+                fd = (up - dn) / (2 * step)
+                assert abs(g[idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (fmap, which, idx, g[idx], fd)
+
+
+def pin_backward_linear_in_dout(ora):
+    """The gradients are linear in dout, and dv of a ones-weighted loss with
+    eps = 0 has the closed form sum_i w_ij / den_i (phi(q_i).phi(k_j) = w_ij)."""
+    rng = _rng(72)
+    q, k, v = (rng.standard_normal((1, 1, 6, 4)) for _ in range(3))
+    d1, d2 = rng.standard_normal((2, 1, 1, 6, 4))
+    a = ora.backward(q, k, v, d1, "elu", 1e-3)
+    b = ora.backward(q, k, v, d2, "elu", 1e-3)
+    c = ora.backward(q, k, v, 2.0 * d1 - d2, "elu", 1e-3)
+    for x, y, w in zip(a, b, c):
+        _close(w, 2.0 * x - y, rtol=1e-10, atol=1e-12)
+    ones = np.ones((1, 1, 6, 4))
+    dv = ora.backward(q, k, v, ones, "elu", 0.0)[2][0, 0]
+    pq, pk = ora.phi_elu1(q[0, 0]), ora.phi_elu1(k[0, 0])
+    w = pq @ pk.T
+    want = (w / w.sum(axis=1, keepdims=True)).sum(axis=0)
+    _close(dv, np.repeat(want[:, None], 4, axis=1), rtol=1e-12)
+
 ALL_PINS = [
     pin_feature_maps,
     pin_feature_map_vs_torch,
@@ -592,4 +639,6 @@ ALL_PINS = [
     pin_softmax_equal_keys,
     pin_prologue_vs_library,
     pin_rope_invariants,
+    pin_backward_finite_differences,
+    pin_backward_linear_in_dout,
 ]

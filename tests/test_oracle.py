@@ -67,6 +67,12 @@ MUTANTS = [
      "x0, x1 = x[..., : x.shape[-1] // 2], x[..., x.shape[-1] // 2:]"),
     ("prologue_scales_swapped", "qn = rope(rms_norm(q, q_scale, norm_eps), table)", "qn = rope(rms_norm(q, k_scale, norm_eps), table)"),
     ("prologue_rope_before_norm", "qn = rope(rms_norm(q, q_scale, norm_eps), table)", "qn = rms_norm(rope(q, table), q_scale, norm_eps)"),
+    ("backward_drops_h", "dpq = g @ kv.T + h[:, None] * z[None, :]", "dpq = g @ kv.T"),
+    ("backward_h_sign", "h = -(dout * out).sum(axis=1) / den", "h = (dout * out).sum(axis=1) / den"),
+    ("backward_dkv_uses_keys", "dkv = pq.T @ g", "dkv = pk.T @ g"),
+    ("backward_dz_missing", "dpk = v @ dkv.T + dz[None, :]", "dpk = v @ dkv.T"),
+    ("backward_dv_transposed", "dv = pk @ dkv", "dv = pq @ dkv"),
+    ("backward_elu_grad_one", "return np.where(x > 0.0, 1.0, np.exp(np.minimum(x, 0.0)))", "return np.ones_like(x)"),
     ("e4m3_bias_eight", "np.exp2(e - 7.0)", "np.exp2(e - 8.0)"),
     ("e4m3_no_subnormals", "np.where(e == 0, (m / 8.0) * 2.0 ** -6,", "np.where(e < 0, (m / 8.0) * 2.0 ** -6,"),
     ("e4m3_subnormal_scale", "(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7"),
