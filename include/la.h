@@ -217,6 +217,30 @@ la_status_t la_forward_e4m3(la_handle_t handle, const void* q, const void* k, co
                             float scale_k, float scale_v, void* out, int B, int H, int N, int D,
                             int feature_map, float eps, void* stream);
 
+/* Backward pass (page "Flux2TTRTrainer", "How the distillation works": the
+ * student layer is trained): given dout = dL/dout of a forward with the same
+ * arguments, writes dq, dk, dv = dL/dq, dL/dk, dL/dv.  With
+ * den_i = phi(q_i).z + eps, out_i = phi(q_i) kv / den_i, g_i = dout_i / den_i
+ * and h_i = -(dout_i . out_i) / den_i:
+ *     dq_i = (kv g_i + h_i z) * phi'(q_i),
+ *     dk_j = (dkv v_j + dz) * phi'(k_j),   dv_j = dkv^T phi(k_j),
+ * where dkv = sum_i phi(q_i) g_i^T and dz = sum_i h_i phi(q_i); phi' of elu+1
+ * is 1 for x > 0 and exp(x) otherwise, of relu 1 for x > 0 and 0 otherwise.
+ * Supported: LA_F32 handles, non-causal, no projection, elu+1 or relu, no
+ * prologue bound, D <= 128 with D % 4 == 0 (else LA_ERR_UNSUPPORTED).
+ * q, k, v, dout: device fp32 [B, H, N, D], read only (may coincide); dq, dk,
+ * dv: device fp32 [B, H, N, D], pairwise disjoint and sharing no byte with
+ * the inputs or the workspace (else LA_ERR_INVALID_ARG); all 16-byte aligned.
+ * Workspace: la_backward_workspace_bytes of the same shape.  Five launches on
+ * `stream`; deterministic. */
+la_status_t la_backward(la_handle_t handle, const void* q, const void* k, const void* v, const void* dout,
+                        void* dq, void* dk, void* dv, int B, int H, int N, int D, int feature_map, float eps,
+                        void* stream);
+
+/* Workspace bytes la_backward needs for this shape (0 for an unsupported or
+ * invalid one). */
+size_t la_backward_workspace_bytes(la_handle_t handle, int B, int H, int N, int D);
+
 /* Landmark count of the page's knobs (landmark fraction, min, max; page
  * "Flux2TTRTrainer", "Inputs worth setting"): round(fraction * N) (half up)
  * clamped to [min_count, max_count], then to [1, N].  0 for invalid arguments

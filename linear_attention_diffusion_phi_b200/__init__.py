@@ -28,7 +28,8 @@ STATUS_NAMES = {
 
 EXPORTED = ("la_create", "la_destroy", "la_set_projection", "la_workspace_bytes", "la_set_workspace",
             "la_forward", "la_forward_host", "la_sync_status", "la_status_string", "la_version",
-            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count", "la_forward_e4m3", "la_set_prologue")
+            "la_forward_noalloc", "la_forward_ttr", "la_landmark_count", "la_forward_e4m3", "la_set_prologue",
+            "la_backward", "la_backward_workspace_bytes")
 
 
 class LAError(RuntimeError):
@@ -63,6 +64,9 @@ def lib():
     L.la_forward_ttr.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]
     L.la_forward_e4m3.argtypes = [vp, vp, vp, vp, f32, f32, f32, vp, i32, i32, i32, i32, i32, f32, vp]
     L.la_set_prologue.argtypes = [vp, vp, vp, vp, i32, i32, f32]
+    L.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
+    L.la_backward_workspace_bytes.argtypes = [vp, i32, i32, i32, i32]
+    L.la_backward_workspace_bytes.restype = sz
     L.la_landmark_count.argtypes = [i32, f32, i32, i32]
     L.la_landmark_count.restype = i32
     L.la_status_string.argtypes = [i32]
@@ -70,7 +74,7 @@ def lib():
     L.la_version.argtypes = []
     for name in ("la_create", "la_destroy", "la_set_projection", "la_set_workspace", "la_forward",
                  "la_forward_host", "la_sync_status", "la_forward_noalloc", "la_forward_ttr", "la_forward_e4m3",
-                 "la_set_prologue"):
+                 "la_set_prologue", "la_backward"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -132,6 +136,15 @@ def la_forward_e4m3(handle, q, k, v, scale_q, scale_k, scale_v, out, B, H, N, D,
 def la_set_prologue(handle, q_scale, k_scale, rope, D, n_positions, norm_eps):
     """Bind Flux's attention prologue (QK RMS norm, then the rotary embedding)."""
     return lib().la_set_prologue(handle, q_scale, k_scale, rope, D, n_positions, norm_eps)
+
+
+def la_backward(handle, q, k, v, dout, dq, dk, dv, B, H, N, D, feature_map, eps, stream):
+    """Gradients dq, dk, dv of sum(out * dout) (fp32, non-causal, no projection)."""
+    return lib().la_backward(handle, q, k, v, dout, dq, dk, dv, B, H, N, D, feature_map, eps, stream)
+
+
+def la_backward_workspace_bytes(handle, B, H, N, D):
+    return lib().la_backward_workspace_bytes(handle, B, H, N, D)
 
 
 def la_landmark_count(N, fraction, min_count, max_count):
@@ -317,6 +330,24 @@ class LinearAttention:
         check(la_set_prologue(self.handle, q_scale.data_ptr(), k_scale.data_ptr(), rope.data_ptr(), D,
                               rope.shape[0], float(norm_eps)), "la_set_prologue")
         self._prologue = (q_scale, k_scale, rope)   # kept alive while bound
+
+    def backward(self, q, k, v, dout, stream=None):
+        """dq, dk, dv of sum(out * dout) for this operator's forward (la_backward:
+        fp32, non-causal, no projection, elu+1 or relu)."""
+        self._check_tensors(q, k, v, dout)
+        B, H, N, D = q.shape
+        dq, dk, dv = (self.torch.empty_like(q) for _ in range(3))
+        with self.torch.cuda.device(q.device):
+            need = la_backward_workspace_bytes(self.handle, B, H, N, D)
+            if need == 0:
+                raise LAError(2, "la_backward_workspace_bytes")
+            if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
+                self._ws = self.torch.empty(need, dtype=self.torch.uint8, device=q.device)
+                check(la_set_workspace(self.handle, self._ws.data_ptr(), self._ws.numel()), "la_set_workspace")
+            s = stream if stream is not None else self.torch.cuda.current_stream(q.device).cuda_stream
+            check(la_backward(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                              dk.data_ptr(), dv.data_ptr(), B, H, N, D, self.fmap, self.eps, s), "la_backward")
+        return dq, dk, dv
 
     def sync_status(self, stream=None):
         dev = self._ws.device if self._ws is not None else self.torch.cuda.current_device()

@@ -326,6 +326,144 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
   }
 }
 
+// ------------------------------------------------------------ backward
+// Gradients of sum(out * dout), non-causal, no projection (features = D), for
+// a loss whose gradient with respect to out is dout (page "Flux2TTRTrainer",
+// "How the distillation works": the student layer is trained).  With
+// den_i = phi(q_i).z + eps, out_i = phi(q_i) kv / den_i, g_i = dout_i / den_i
+// and h_i = -(dout_i . out_i) / den_i:
+//   dq_i = (kv g_i + h_i z) * phi'(q_i),
+//   dkv = sum_i phi(q_i) g_i^T,  dz = sum_i h_i phi(q_i),
+//   dk_j = (dkv v_j + dz) * phi'(k_j),  dv_j = dkv^T phi(k_j).
+
+__device__ __forceinline__ float phi_grad(float x, int fmap) {
+  if (fmap == 0) return x > 0.f ? 1.f : expf(x);
+  return x > 0.f ? 1.f : 0.f;
+}
+
+// Query rows of split s of head bh: dq, and the split's partials of dkv
+// ([bh][s][D][D], row f = feature) and dz ([bh][s][D]).
+__global__ void __launch_bounds__(256) f32_bwd_query(const float* __restrict__ q, const float* __restrict__ dout,
+                                                     const float* __restrict__ fin, const float* __restrict__ fin_ksum,
+                                                     float* __restrict__ dq, float* __restrict__ part_dkv,
+                                                     float* __restrict__ part_dz, int N, int D, int fmap, float eps,
+                                                     int seg, int S) {
+  __shared__ __align__(16) float Qs[kT * kMaxD];
+  __shared__ __align__(16) float Ps[kT * kMaxD];
+  __shared__ __align__(16) float Gs[kT * kMaxD];
+  __shared__ float dens[kT], hs[kT];
+  const int s = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const float* kv = fin + static_cast<size_t>(bh) * D * D;
+  const float* z = fin_ksum + static_cast<size_t>(bh) * D;
+  const float* qh = q + static_cast<size_t>(bh) * N * D;
+  const float* oh = dout + static_cast<size_t>(bh) * N * D;
+  const int t0 = s * seg, t1 = min(N, t0 + seg);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int kAcc = kMaxD * kMaxD / 256;
+  float acc[kAcc];
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) acc[j] = 0.f;
+  float dzacc = 0.f;
+  for (int tc = t0; tc < t1; tc += kT) {
+    const int rows = min(kT, t1 - tc);
+    load_rows(Qs, qh + static_cast<size_t>(tc) * D, rows, D);
+    load_rows(Gs, oh + static_cast<size_t>(tc) * D, rows, D);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * D; e += blockDim.x) {
+      const int t = e / D, f = e % D;
+      Ps[t * kMaxD + f] = t < rows ? phi_accurate(Qs[t * kMaxD + f], fmap) : 0.f;
+    }
+    __syncthreads();
+    // den_t and h_t = -(dout_t . num_t) / den_t^2: one warp per two rows
+    for (int t = warp; t < kT; t += blockDim.x / 32) {
+      float den = 0.f, dot = 0.f;
+      for (int f = lane; f < D; f += 32) den = fmaf(Ps[t * kMaxD + f], z[f], den);
+      for (int d = lane; d < D; d += 32) {
+        float num = 0.f;
+        for (int f = 0; f < D; ++f) num = fmaf(Ps[t * kMaxD + f], kv[static_cast<size_t>(f) * D + d], num);
+        dot = fmaf(Gs[t * kMaxD + d], num, dot);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+        dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      }
+      den += eps;
+      if (lane == 0) {
+        dens[t] = den;
+        hs[t] = -dot / (den * den);
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * D; e += blockDim.x) {   // g = dout / den
+      const int t = e / D, d = e % D;
+      Gs[t * kMaxD + d] /= dens[t];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
+      const int t = e / D, f = e % D;
+      float g = hs[t] * z[f];
+      for (int d = 0; d < D; ++d) g = fmaf(kv[static_cast<size_t>(f) * D + d], Gs[t * kMaxD + d], g);
+      dq[(static_cast<size_t>(bh) * N + tc + t) * D + f] = g * phi_grad(Qs[t * kMaxD + f], fmap);
+    }
+#pragma unroll
+    for (int j = 0; j < kAcc; ++j) {
+      const int e = threadIdx.x + 256 * j;
+      if (e < D * D) {
+        const int f = e / D, d = e % D;
+        float a = acc[j];
+        for (int t = 0; t < kT; ++t) a = fmaf(Ps[t * kMaxD + f], Gs[t * kMaxD + d], a);
+        acc[j] = a;
+      }
+    }
+    if (threadIdx.x < D)
+      for (int t = 0; t < kT; ++t) dzacc = fmaf(hs[t], Ps[t * kMaxD + threadIdx.x], dzacc);
+    __syncthreads();
+  }
+  float* dst = part_dkv + (static_cast<size_t>(bh) * S + s) * D * D;
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) {
+    const int e = threadIdx.x + 256 * j;
+    if (e < D * D) dst[e] = acc[j];
+  }
+  if (threadIdx.x < D) part_dz[(static_cast<size_t>(bh) * S + s) * D + threadIdx.x] = dzacc;
+}
+
+// Key rows [blockIdx.x * kT, +kT) of head bh: dk and dv from dkv, dz.
+__global__ void __launch_bounds__(256) f32_bwd_key(const float* __restrict__ k, const float* __restrict__ v,
+                                                   const float* __restrict__ fin_dkv,
+                                                   const float* __restrict__ fin_dz, float* __restrict__ dk,
+                                                   float* __restrict__ dv, int N, int D, int fmap) {
+  __shared__ __align__(16) float Ks[kT * kMaxD];
+  __shared__ __align__(16) float Vs[kT * kMaxD];
+  __shared__ __align__(16) float Ps[kT * kMaxD];
+  const long long bh = blockIdx.y;
+  const int t0 = blockIdx.x * kT;
+  const int rows = min(kT, N - t0);
+  const float* dkv = fin_dkv + static_cast<size_t>(bh) * D * D;
+  const float* dz = fin_dz + static_cast<size_t>(bh) * D;
+  load_rows(Ks, k + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
+  load_rows(Vs, v + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
+  __syncthreads();
+  for (int e = threadIdx.x; e < kT * D; e += blockDim.x) {
+    const int t = e / D, f = e % D;
+    Ps[t * kMaxD + f] = t < rows ? phi_accurate(Ks[t * kMaxD + f], fmap) : 0.f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
+    const int t = e / D, c = e % D;
+    float gk = dz[c], gv = 0.f;
+    for (int x = 0; x < D; ++x) {
+      gk = fmaf(dkv[static_cast<size_t>(c) * D + x], Vs[t * kMaxD + x], gk);   // (dkv v_t)_c
+      gv = fmaf(Ps[t * kMaxD + x], dkv[static_cast<size_t>(x) * D + c], gv);   // (dkv^T phi(k_t))_c
+    }
+    const size_t o = (static_cast<size_t>(bh) * N + t0 + t) * D + c;
+    dk[o] = gk * phi_grad(Ks[t * kMaxD + c], fmap);
+    dv[o] = gv;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_f32(const LaunchArgs& a) {
@@ -367,6 +505,44 @@ cudaError_t launch_f32(const LaunchArgs& a) {
   dim3 g3(S, static_cast<unsigned>(p.BH));
   f32_causal_apply<<<g3, 256, dyn, a.stream>>>(q, k, v, W, a.w_head_stride, part, part_ksum, out, p.H, p.N, p.D, p.F,
                                                p.Fe, p.fmap, p.eps, p.seg_len, S, pq, pk);
+  return cudaGetLastError();
+}
+
+// Backward of the fp32 non-causal layer without projection: the forward
+// state (kv, z) into the plan's final region, then per-split partials of
+// (dkv, dz) into the plan's partial region (no longer needed), summed in
+// ascending split order into bfin / bfin_z, then dk and dv.
+cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq, void* dk, void* dv, float* bfin,
+                                float* bfin_z) {
+  const Plan& p = *a.p;
+  if (p.F != 0 || p.causal || p.fmap > 1 || a.prologue) return cudaErrorNotSupported;
+  const float* q = static_cast<const float*>(a.q);
+  const float* k = static_cast<const float*>(a.k);
+  const float* v = static_cast<const float*>(a.v);
+  float* part = reinterpret_cast<float*>(a.ws + p.off_partial);
+  float* part_ksum = reinterpret_cast<float*>(a.ws + p.off_ksum_partial);
+  float* fin = reinterpret_cast<float*>(a.ws + p.off_final);
+  float* fin_ksum = reinterpret_cast<float*>(a.ws + p.off_final_ksum);
+  const int S = p.splits;
+  const int n_state = p.D * p.D + p.D;
+  const Prologue none = {nullptr, nullptr, 0.f};
+  dim3 g1(S, static_cast<unsigned>(p.BH), (p.D + kFB - 1) / kFB);
+  f32_state_partial<<<g1, 256, 0, a.stream>>>(k, v, nullptr, 0, part, part_ksum, p.H, p.N, p.D, 0, p.D, p.fmap,
+                                              p.seg_len, S, none);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dim3 g2(static_cast<unsigned>(p.BH), (n_state + 255) / 256);
+  f32_state_combine<<<g2, 256, 0, a.stream>>>(part, part_ksum, fin, fin_ksum, p.D, p.D, S);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  f32_bwd_query<<<dim3(S, static_cast<unsigned>(p.BH)), 256, 0, a.stream>>>(
+      q, static_cast<const float*>(dout), fin, fin_ksum, static_cast<float*>(dq), part, part_ksum, p.N, p.D, p.fmap,
+      p.eps, p.seg_len, S);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  f32_state_combine<<<g2, 256, 0, a.stream>>>(part, part_ksum, bfin, bfin_z, p.D, p.D, S);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  dim3 g3((p.N + kT - 1) / kT, static_cast<unsigned>(p.BH));
+  f32_bwd_key<<<g3, 256, 0, a.stream>>>(k, v, bfin, bfin_z, static_cast<float*>(dk), static_cast<float*>(dv), p.N,
+                                        p.D, p.fmap);
   return cudaGetLastError();
 }
 

@@ -532,6 +532,101 @@ la_status_t la_forward_e4m3(la_handle_t h, const void* q, const void* k, const v
   return forward_impl(h, q, k, v, out, B, H, N, D, 0, fmap, eps, 0, stream, nullptr, 0, sc);
 }
 
+namespace {
+
+// The backward's workspace: the forward plan of the same shape, then the
+// [BH][D][D] dkv and [BH][D] dz sums.
+size_t backward_plan(la_handle_t h, int B, int H, int N, int D, int fmap, float eps, int sms, Plan* p,
+                     size_t* off_bfin, size_t* off_bfin_z) {
+  make_plan(h, B, H, N, D, 0, fmap, eps, 0, sms, p);
+  const size_t BH = static_cast<size_t>(std::max<long long>(p->BH, 1));
+  *off_bfin = align256(p->bytes);
+  *off_bfin_z = align256(*off_bfin + BH * D * D * 4);
+  return align256(*off_bfin_z + BH * D * 4);
+}
+
+la_status_t check_backward(la_handle_t h, int B, int H, int N, int D, int fmap, float eps) {
+  if (!h) return LA_ERR_INVALID_ARG;
+  la_status_t st = check_shape(h, B, H, N, D, 0, fmap, eps, 0);
+  if (st != LA_OK) return st;
+  if (h->dtype != LA_F32 || fmap == LA_PHI_SOFTMAX || h->pro_q) return LA_ERR_UNSUPPORTED;
+  return LA_OK;
+}
+
+}  // namespace
+
+size_t la_backward_workspace_bytes(la_handle_t h, int B, int H, int N, int D) {
+  if (check_backward(h, B, H, N, D, LA_PHI_ELU1, 0.f) != LA_OK) return 0;
+  DeviceInfo di;
+  const int sms = device_info(&di) ? di.sms : 148;
+  Plan p;
+  size_t a, b;
+  return backward_plan(h, B, H, N, D, LA_PHI_ELU1, 0.f, sms, &p, &a, &b);
+}
+
+la_status_t la_backward(la_handle_t h, const void* q, const void* k, const void* v, const void* dout, void* dq,
+                        void* dk, void* dv, int B, int H, int N, int D, int fmap, float eps, void* stream) {
+  la_status_t st = check_backward(h, B, H, N, D, fmap, eps);
+  if (st != LA_OK) return st;
+  if (static_cast<long long>(B) * H * N == 0) return LA_OK;
+  const void* ins[4] = {q, k, v, dout};
+  void* outs[3] = {dq, dk, dv};
+  for (const void* x : ins)
+    if (!x) return LA_ERR_INVALID_ARG;
+  for (void* x : outs)
+    if (!x) return LA_ERR_INVALID_ARG;
+  for (const void* x : ins)
+    if (!aligned16(x)) return LA_ERR_MISALIGNED;
+  for (void* x : outs)
+    if (!aligned16(x)) return LA_ERR_MISALIGNED;
+  const size_t nb = static_cast<size_t>(B) * H * N * D * 4;
+  // the outputs are written while the inputs are read: no output shares a
+  // byte with an input, another output or the workspace
+  for (int i = 0; i < 3; ++i) {
+    for (const void* x : ins)
+      if (la::overlap(outs[i], nb, x, nb)) return LA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (la::overlap(outs[i], nb, outs[j], nb)) return LA_ERR_INVALID_ARG;
+    if (h->ws && la::overlap(h->ws, h->ws_bytes, outs[i], nb)) return LA_ERR_INVALID_ARG;
+  }
+  for (const void* x : ins)
+    if (h->ws && la::overlap(h->ws, h->ws_bytes, x, nb)) return LA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if (!device_info(&di)) return LA_ERR_NO_DEVICE;
+  if (di.major != 10 || di.minor != 0) return LA_ERR_NO_DEVICE;
+  Plan p;
+  size_t off_bfin, off_bfin_z;
+  const size_t need = backward_plan(h, B, H, N, D, fmap, eps, di.sms, &p, &off_bfin, &off_bfin_z);
+  if (!h->ws || h->ws_bytes < need) return LA_ERR_WORKSPACE;
+  for (const void* x : ins)
+    if (!la::on_current_device(x)) return LA_ERR_INVALID_ARG;
+  for (void* x : outs)
+    if (!la::on_current_device(x)) return LA_ERR_INVALID_ARG;
+  if (!la::on_current_device(h->ws)) return LA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (h->ws_clear_pending) {
+    if (cudaMemsetAsync(h->ws, 0, la::kHeaderBytes, cs) != cudaSuccess) {
+      cudaGetLastError();
+      return LA_ERR_CUDA;
+    }
+    h->ws_clear_pending = false;
+  }
+  la::LaunchArgs a = {};
+  a.p = &p;
+  a.q = q; a.k = k; a.v = v;
+  a.ws = static_cast<char*>(h->ws);
+  a.stream = cs;
+  char* ws = static_cast<char*>(h->ws);
+  const cudaError_t err = la::launch_f32_backward(a, dout, dq, dk, dv, reinterpret_cast<float*>(ws + off_bfin),
+                                                  reinterpret_cast<float*>(ws + off_bfin_z));
+  if (err == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
+  if (err != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
 int la_landmark_count(int N, float fraction, int min_count, int max_count) {
   if (N < 1 || !(fraction >= 0.f) || min_count < 0 || max_count < 1) return 0;
   const double want = std::floor(static_cast<double>(fraction) * N + 0.5);

@@ -317,3 +317,22 @@ def test_prologue_binding_and_support_checks(handles):
     assert fwd(bf, D=64) == la.LA_ERR_UNSUPPORTED                  # bf16 prologue needs D = 128
     assert la.la_set_prologue(bf, None, None, None, 0, 0, 0.0) == la.LA_OK
 
+
+def test_backward_checks_on_the_host(handles):
+    """la_backward runs on fp32 handles without projection or prologue, elu+1
+    or relu; it refuses overlapping outputs before anything is enqueued."""
+    f32, bf = handles["f32"], handles["bf16"]
+    assert la.la_backward_workspace_bytes(f32, 1, 2, 256, 64) > 0
+    assert la.la_backward_workspace_bytes(bf, 1, 2, 256, 128) == 0
+    nb = 1 * 2 * 256 * 64 * 4
+    base = 0x100000
+    ins = [base, base, base, base + nb]
+    outs = [base + 4 * nb, base + 6 * nb, base + 8 * nb]
+    b = lambda h, o=outs, fmap=la.LA_PHI_ELU1, D=64: la.la_backward(h, *ins, *o, 1, 2, 256, D, fmap, 1e-6, None)
+    assert b(bf, D=128) == la.LA_ERR_UNSUPPORTED
+    assert b(f32, fmap=la.LA_PHI_SOFTMAX) == la.LA_ERR_UNSUPPORTED
+    assert b(f32, o=[outs[0], outs[0], outs[2]]) == la.LA_ERR_INVALID_ARG     # dq and dk coincide
+    assert b(f32, o=[base + nb // 2, outs[1], outs[2]]) == la.LA_ERR_INVALID_ARG   # dq over the inputs
+    assert b(f32, o=[outs[0] + 4, outs[1], outs[2]]) == la.LA_ERR_MISALIGNED
+    assert la.la_backward(f32, 0, 0, 0, 0, 0, 0, 0, 1, 0, 256, 64, la.LA_PHI_ELU1, 1e-6, None) == la.LA_OK
+

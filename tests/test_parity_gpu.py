@@ -721,3 +721,61 @@ def test_flux1024_prologue_full():
     got, ref = run_prologue(w)
     assert_parity(got, ref, "bf16", "flux1024_prologue (all elements)")
 
+
+# ------------------------------------------------------------ backward pass --
+
+BWD_CASES = [
+    dict(B=1, H=2, N=300, D=64, fmap="elu"), dict(B=2, H=1, N=1000, D=128, fmap="relu"),
+    dict(B=1, H=1, N=1, D=32, fmap="elu"), dict(B=1, H=3, N=37, D=4, fmap="elu"),
+    dict(B=1, H=2, N=4608, D=128, fmap="elu"),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_f32_backward(case):
+    """dq, dk, dv of sum(out * dout) against the oracle's backward, each at the
+    fp32 bar (relative to its own largest magnitude), and bitwise repeatable."""
+    import torch
+    w = Workload("bwd", dtype="f32", seed=2500 + case["N"], **case)
+    q, k, v, _ = make_inputs(w)
+    dout = make_inputs(w, seed=w.seed + 1)[0]
+    dev = torch.device("cuda:0")
+    op = la.LinearAttention(torch.float32, w.fmap, w.eps)
+    args = [t.to(dev) for t in (q, k, v, dout)]
+    got = op.backward(*args)
+    again = op.backward(*args)
+    torch.cuda.synchronize()
+    assert op.sync_status() == la.LA_OK
+    for a, b in zip(got, again):
+        assert torch.equal(a, b)
+    op.close()
+    qf, kf, vf, of = (as_float64(t) for t in (q, k, v, dout))
+    ref = ora.backward(qf, kf, vf, of, w.fmap, w.eps)
+    scales = backward_term_scales(qf, kf, vf, of, w.fmap, w.eps)
+    for name, g, r, sc in zip(("dq", "dk", "dv"), got, ref, scales):
+        err = np.abs(as_float64(g.cpu()) - r)
+        # fp32 bar against the size of the terms each gradient sums: a
+        # gradient that is itself a cancellation (dq of a one-token head is
+        # eps-small) is held to the precision of its summands
+        assert np.all(np.isfinite(err)) and err.max() <= F32_REL * sc, (name, err.max(), sc, np.abs(r).max())
+
+
+def backward_term_scales(q, k, v, dout, fmap, eps):
+    """Largest magnitude of the summed terms of dq, dk and dv (absolute values
+    through every product of the backward's formulas)."""
+    out = []
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            pq, pk = ora.feature_map(q[b, h], fmap), ora.feature_map(k[b, h], fmap)
+            kv, z = pk.T @ v[b, h], pk.sum(axis=0)
+            den = pq @ z + eps
+            o = (pq @ kv) / den[:, None]
+            ag = np.abs(dout[b, h]) / den[:, None]
+            ah = (np.abs(dout[b, h]) * np.abs(o)).sum(axis=1) / den
+            adkv, adz = pq.T @ ag, pq.T @ ah
+            sq = (ag @ np.abs(kv).T + ah[:, None] * z[None, :]) * np.abs(ora.feature_map_grad(q[b, h], fmap))
+            sk = (np.abs(v[b, h]) @ adkv.T + adz[None, :]) * np.abs(ora.feature_map_grad(k[b, h], fmap))
+            sv = pk @ adkv
+            out.append((sq.max(), sk.max(), sv.max()))
+    return tuple(max(x[i] for x in out) for i in range(3))
+
