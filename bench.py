@@ -406,7 +406,7 @@ class Timed:
     shifted along the sequence, so every step reads memory the previous steps
     did not touch), the operator, and CUDA graphs of its steps."""
 
-    def __init__(self, w, dev, rank, graphs=True, ttr=None, e4m3=False, prologue=False):
+    def __init__(self, w, dev, rank, graphs=True, ttr=None, e4m3=False, prologue=False, backward=False):
         import torch
         import linear_attention_diffusion_phi_b200 as la
         from linear_attention_diffusion_phi_b200.inputs import make_e4m3_inputs, make_inputs
@@ -429,6 +429,13 @@ class Timed:
             q, k, v, W = self.host
             out_like = None
         base = (q.to(dev), k.to(dev), v.to(dev))
+        # backward: each step computes dq, dk, dv of sum(out * dout) (la_backward)
+        self.bwd = None
+        if backward:
+            dout = make_inputs(w, seed=input_seed(w, 0, rank) + 1)[0]
+            self.bwd = (dout.to(dev), [torch.empty_like(base[0]) for _ in range(3)])
+            self.host = (q, k, v, dout)
+            self.set_bytes += 3 * w.B * w.H * w.N * w.D * 4
         new_out = out_like or (lambda: torch.empty_like(base[0]))
         self.sets = [base + (new_out(),)]
         for i in range(1, self.nsets):
@@ -452,7 +459,9 @@ class Timed:
 
     def step(self, i):
         q, k, v, o = self.sets[i % self.nsets]
-        if self.e4m3:
+        if self.bwd is not None:
+            self.op.backward(q, k, v, self.bwd[0], outs=self.bwd[1])
+        elif self.e4m3:
             self.op.e4m3(q, k, v, self.scales, out=o)
         elif self.ttr is None:
             self.op(q, k, v, out=o)
@@ -560,6 +569,25 @@ def roofline(w, per_step_s, hbm, tflops, src, sms):
     return roof, launches
 
 
+def backward_parity(w, tx):
+    """Largest error of dq, dk, dv on two sampled heads against the oracle's
+    backward, relative to each gradient's largest magnitude."""
+    import torch
+    from linear_attention_diffusion_phi_b200.inputs import as_float64
+    from oracle import la_oracle as ora
+    tx.step(0)
+    torch.cuda.synchronize()
+    q, k, v, dout = tx.host
+    got = [g.cpu() for g in tx.bwd[1]]
+    worst = 0.0
+    for b, h in ((0, 0), (w.B - 1, w.H - 1)):
+        ref = ora.backward_head(*(as_float64(t[b, h]) for t in (q, k, v, dout)), w.fmap, w.eps)
+        for g, r in zip(got, ref):
+            worst = max(worst, float(np.abs(as_float64(g[b, h]) - r).max() / max(np.abs(r).max(), 1e-300)))
+    return {"rel_inf": worst, "bar": {"rel_inf": F32_REL_INF}, "pass": bool(worst <= F32_REL_INF),
+            "heads_checked": 2}
+
+
 def roofline_e4m3(w, per_step_s, hbm, src, name):
     """HBM roofline of the E4M3-input forward (one launch per step): q, k, v
     read once at one byte per element, out written once in bf16."""
@@ -572,7 +600,7 @@ def roofline_e4m3(w, per_step_s, hbm, src, name):
 
 
 EXTRA_WORKLOADS = ("flux2048_cfg", "proj256", "causal32k", "flux1024_ttr", "flux1024_e4m3", "flux2048_cfg_e4m3",
-                   "flux1024_softmax", "flux1024_prologue")
+                   "flux1024_softmax", "flux1024_prologue", "flux1024_f32_backward")
 # The TTR layer on the flux1024 shape: 128 landmarks (the page's knobs at
 # fraction 1/32, min 16, max 128) and one logit per head, spread over [-2, 2].
 TTR_LANDMARKS = (1 / 32, 16, 128)
@@ -594,13 +622,18 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
     e8 = name.endswith("_e4m3")
     smx = name.endswith("_softmax")   # the same shapes with the softmax feature map
     pro = name.endswith("_prologue")  # the same shapes behind Flux's attention prologue
+    bwd = name.endswith("_backward")  # the fp32 backward pass on the same shapes
     base = name[:-4] if ttr else (name[:-5] if e8 else (name[:-8] if smx else (name[:-9] if pro else name)))
+    if bwd:
+        base = name[:-len("_f32_backward")]
     x = WORKLOADS[base]
+    if bwd:
+        x = x.with_(dtype="f32")
     if smx:
         x = x.with_(fmap="softmax")
     try:
         tx = Timed(x, dev, rank, graphs=not args.no_graph, ttr=ttr_params(x) if ttr else None, e4m3=e8,
-                   prologue=pro)
+                   prologue=pro, backward=bwd)
         xsteps = max(args.steps, 100)
         tx.steps_hint = xsteps
         smp = ClockSampler(local)
@@ -624,14 +657,27 @@ def run_extra(name, args, dev, rank, local, stream, ws, hbm, tflops, src, sms):
             xroof["traffic"] = captured_traffic(x, name)
         if pro:
             xroof["kernel"] = "fused_t_kernel with the prologue (one cluster launch per step)"
+        if bwd:
+            # q, k, v, dout read and dq, dk, dv written once, fp32
+            abytes = 7 * x.B * x.H * x.N * x.D * 4
+            xroof = {"bound": "hbm", "achieved": abytes / (xms / 1e3 / xsteps) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": abytes / (xms / 1e3 / xsteps) / 1e9 / hbm, "traffic": None,
+                     "peak_source": f"{src} hbm_gbs", "frac_of": src, "algorithmic_bytes_per_step": abytes,
+                     "kernel": "f32_state_partial, f32_state_combine, f32_bwd_query, f32_state_combine, f32_bwd_key "
+                               "(five launches per step)"}
+            xl = 5
         ent = {"workload": name, "B": x.B, "H": x.H, "N": x.N, "D": x.D, "F": x.F, "feature_map": x.fmap,
                "causal": x.causal, "dtype": "e4m3 in, bf16 out" if e8 else x.dtype, "steps": xsteps,
                "ms_per_step": xms / xsteps,
                "value": x.tokens / (xms / 1e3 / xsteps), "unit": UNIT, "roofline": xroof,
                "gpu_launches": None if xl is None else xl * xsteps, "clocks": xclk,
                "l2": f"{tx.nsets} rotating input sets, {tx.nsets * tx.set_bytes / 2**20:.0f} MiB > 3x L2"}
-        if not args.no_parity:
+        if bwd:
+            ent["dtype"] = "f32"
+        if not args.no_parity and not bwd:
             ent["parity"] = parity_block(x, *tx.host, tx.output0(), ttr=tx.ttr, e4m3=e8, prologue=tx.pro_host)
+        if not args.no_parity and bwd:
+            ent["parity"] = backward_parity(x, tx)
         tx.close()
         del tx
     except Exception as e:   # an extra figure never costs the headline line

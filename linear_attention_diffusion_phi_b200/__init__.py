@@ -331,12 +331,16 @@ class LinearAttention:
                               rope.shape[0], float(norm_eps)), "la_set_prologue")
         self._prologue = (q_scale, k_scale, rope)   # kept alive while bound
 
-    def backward(self, q, k, v, dout, stream=None):
+    def backward(self, q, k, v, dout, outs=None, stream=None):
         """dq, dk, dv of sum(out * dout) for this operator's forward (la_backward:
-        fp32, non-causal, no projection, elu+1 or relu)."""
+        fp32, non-causal, no projection, elu+1 or relu); ``outs`` = (dq, dk, dv)
+        to write into."""
         self._check_tensors(q, k, v, dout)
         B, H, N, D = q.shape
-        dq, dk, dv = (self.torch.empty_like(q) for _ in range(3))
+        dq, dk, dv = outs if outs is not None else (self.torch.empty_like(q) for _ in range(3))
+        for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+            if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
+                raise ValueError(f"{name}: expected a contiguous tensor like q")
         with self.torch.cuda.device(q.device):
             need = la_backward_workspace_bytes(self.handle, B, H, N, D)
             if need == 0:

@@ -352,9 +352,13 @@ __global__ void __launch_bounds__(256) f32_bwd_query(const float* __restrict__ q
   __shared__ __align__(16) float Ps[kT * kMaxD];
   __shared__ __align__(16) float Gs[kT * kMaxD];
   __shared__ float dens[kT], hs[kT];
+  // the head's kv, rows padded to D + 1 floats: conflict-free whether the
+  // lanes run along a row or down a column
+  extern __shared__ float kvs[];
   const int s = blockIdx.x;
   const long long bh = blockIdx.y;
-  const float* kv = fin + static_cast<size_t>(bh) * D * D;
+  const float* kvg = fin + static_cast<size_t>(bh) * D * D;
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) kvs[(e / D) * (D + 1) + e % D] = kvg[e];
   const float* z = fin_ksum + static_cast<size_t>(bh) * D;
   const float* qh = q + static_cast<size_t>(bh) * N * D;
   const float* oh = dout + static_cast<size_t>(bh) * N * D;
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(256) f32_bwd_query(const float* __restrict__ q
       for (int f = lane; f < D; f += 32) den = fmaf(Ps[t * kMaxD + f], z[f], den);
       for (int d = lane; d < D; d += 32) {
         float num = 0.f;
-        for (int f = 0; f < D; ++f) num = fmaf(Ps[t * kMaxD + f], kv[static_cast<size_t>(f) * D + d], num);
+        for (int f = 0; f < D; ++f) num = fmaf(Ps[t * kMaxD + f], kvs[f * (D + 1) + d], num);
         dot = fmaf(Gs[t * kMaxD + d], num, dot);
       }
 #pragma unroll
@@ -404,7 +408,7 @@ __global__ void __launch_bounds__(256) f32_bwd_query(const float* __restrict__ q
     for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
       const int t = e / D, f = e % D;
       float g = hs[t] * z[f];
-      for (int d = 0; d < D; ++d) g = fmaf(kv[static_cast<size_t>(f) * D + d], Gs[t * kMaxD + d], g);
+      for (int d = 0; d < D; ++d) g = fmaf(kvs[f * (D + 1) + d], Gs[t * kMaxD + d], g);
       dq[(static_cast<size_t>(bh) * N + tc + t) * D + f] = g * phi_grad(Qs[t * kMaxD + f], fmap);
     }
 #pragma unroll
@@ -430,7 +434,9 @@ __global__ void __launch_bounds__(256) f32_bwd_query(const float* __restrict__ q
   if (threadIdx.x < D) part_dz[(static_cast<size_t>(bh) * S + s) * D + threadIdx.x] = dzacc;
 }
 
-// Key rows [blockIdx.x * kT, +kT) of head bh: dk and dv from dkv, dz.
+// Key rows [blockIdx.x * kBwdRows, +kBwdRows) of head bh, in chunks of kT:
+// dk and dv from dkv and dz.
+constexpr int kBwdRows = 64;
 __global__ void __launch_bounds__(256) f32_bwd_key(const float* __restrict__ k, const float* __restrict__ v,
                                                    const float* __restrict__ fin_dkv,
                                                    const float* __restrict__ fin_dz, float* __restrict__ dk,
@@ -438,11 +444,14 @@ __global__ void __launch_bounds__(256) f32_bwd_key(const float* __restrict__ k, 
   __shared__ __align__(16) float Ks[kT * kMaxD];
   __shared__ __align__(16) float Vs[kT * kMaxD];
   __shared__ __align__(16) float Ps[kT * kMaxD];
+  extern __shared__ float dkvs[];   // dkv, rows padded to D + 1 floats
   const long long bh = blockIdx.y;
-  const int t0 = blockIdx.x * kT;
-  const int rows = min(kT, N - t0);
-  const float* dkv = fin_dkv + static_cast<size_t>(bh) * D * D;
+  const float* dkvg = fin_dkv + static_cast<size_t>(bh) * D * D;
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) dkvs[(e / D) * (D + 1) + e % D] = dkvg[e];
   const float* dz = fin_dz + static_cast<size_t>(bh) * D;
+  for (int t0 = blockIdx.x * kBwdRows; t0 < min(N, (blockIdx.x + 1) * kBwdRows); t0 += kT) {
+  const int rows = min(kT, N - t0);
+  __syncthreads();
   load_rows(Ks, k + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
   load_rows(Vs, v + (static_cast<size_t>(bh) * N + t0) * D, rows, D);
   __syncthreads();
@@ -455,12 +464,13 @@ __global__ void __launch_bounds__(256) f32_bwd_key(const float* __restrict__ k, 
     const int t = e / D, c = e % D;
     float gk = dz[c], gv = 0.f;
     for (int x = 0; x < D; ++x) {
-      gk = fmaf(dkv[static_cast<size_t>(c) * D + x], Vs[t * kMaxD + x], gk);   // (dkv v_t)_c
-      gv = fmaf(Ps[t * kMaxD + x], dkv[static_cast<size_t>(x) * D + c], gv);   // (dkv^T phi(k_t))_c
+      gk = fmaf(dkvs[c * (D + 1) + x], Vs[t * kMaxD + x], gk);   // (dkv v_t)_c
+      gv = fmaf(Ps[t * kMaxD + x], dkvs[x * (D + 1) + c], gv);   // (dkv^T phi(k_t))_c
     }
     const size_t o = (static_cast<size_t>(bh) * N + t0 + t) * D + c;
     dk[o] = gk * phi_grad(Ks[t * kMaxD + c], fmap);
     dv[o] = gv;
+  }
   }
 }
 
@@ -510,10 +520,10 @@ cudaError_t launch_f32(const LaunchArgs& a) {
 
 // Backward of the fp32 non-causal layer without projection: the forward
 // state (kv, z) into the plan's final region, then per-split partials of
-// (dkv, dz) into the plan's partial region (no longer needed), summed in
-// ascending split order into bfin / bfin_z, then dk and dv.
-cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq, void* dk, void* dv, float* bfin,
-                                float* bfin_z) {
+// (dkv, dz) with dq, summed in ascending split order into bfin / bfin_z, then
+// dk and dv.
+cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq, void* dk, void* dv, int splits,
+                                int seg, float* bpart, float* bpart_z, float* bfin, float* bfin_z) {
   const Plan& p = *a.p;
   if (p.F != 0 || p.causal || p.fmap > 1 || a.prologue) return cudaErrorNotSupported;
   const float* q = static_cast<const float*>(a.q);
@@ -534,14 +544,20 @@ cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq,
   dim3 g2(static_cast<unsigned>(p.BH), (n_state + 255) / 256);
   f32_state_combine<<<g2, 256, 0, a.stream>>>(part, part_ksum, fin, fin_ksum, p.D, p.D, S);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  f32_bwd_query<<<dim3(S, static_cast<unsigned>(p.BH)), 256, 0, a.stream>>>(
-      q, static_cast<const float*>(dout), fin, fin_ksum, static_cast<float*>(dq), part, part_ksum, p.N, p.D, p.fmap,
-      p.eps, p.seg_len, S);
+  const size_t mat = static_cast<size_t>(p.D) * (p.D + 1) * sizeof(float);
+  if ((err = cudaFuncSetAttribute(f32_bwd_query, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mat))) !=
+          cudaSuccess ||
+      (err = cudaFuncSetAttribute(f32_bwd_key, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mat))) !=
+          cudaSuccess)
+    return err;
+  f32_bwd_query<<<dim3(splits, static_cast<unsigned>(p.BH)), 256, mat, a.stream>>>(
+      q, static_cast<const float*>(dout), fin, fin_ksum, static_cast<float*>(dq), bpart, bpart_z, p.N, p.D, p.fmap,
+      p.eps, seg, splits);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  f32_state_combine<<<g2, 256, 0, a.stream>>>(part, part_ksum, bfin, bfin_z, p.D, p.D, S);
+  f32_state_combine<<<g2, 256, 0, a.stream>>>(bpart, bpart_z, bfin, bfin_z, p.D, p.D, splits);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  dim3 g3((p.N + kT - 1) / kT, static_cast<unsigned>(p.BH));
-  f32_bwd_key<<<g3, 256, 0, a.stream>>>(k, v, bfin, bfin_z, static_cast<float*>(dk), static_cast<float*>(dv), p.N,
+  dim3 g3((p.N + kBwdRows - 1) / kBwdRows, static_cast<unsigned>(p.BH));
+  f32_bwd_key<<<g3, 256, mat, a.stream>>>(k, v, bfin, bfin_z, static_cast<float*>(dk), static_cast<float*>(dv), p.N,
                                         p.D, p.fmap);
   return cudaGetLastError();
 }

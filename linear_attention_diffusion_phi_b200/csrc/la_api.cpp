@@ -535,14 +535,25 @@ la_status_t la_forward_e4m3(la_handle_t h, const void* q, const void* k, const v
 namespace {
 
 // The backward's workspace: the forward plan of the same shape, then the
-// [BH][D][D] dkv and [BH][D] dz sums.
+// query pass's per-split [D][D] dkv and [D] dz partials (splits of whole
+// 16-token chunks, about two blocks per SM in all), then their sums.
+struct BwdLayout {
+  int splits, seg;
+  size_t off_part, off_part_z, off_fin, off_fin_z, bytes;
+};
 size_t backward_plan(la_handle_t h, int B, int H, int N, int D, int fmap, float eps, int sms, Plan* p,
-                     size_t* off_bfin, size_t* off_bfin_z) {
+                     BwdLayout* b) {
   make_plan(h, B, H, N, D, 0, fmap, eps, 0, sms, p);
-  const size_t BH = static_cast<size_t>(std::max<long long>(p->BH, 1));
-  *off_bfin = align256(p->bytes);
-  *off_bfin_z = align256(*off_bfin + BH * D * D * 4);
-  return align256(*off_bfin_z + BH * D * 4);
+  const long long BH = std::max<long long>(p->BH, 1);
+  const long long want = std::max<long long>(1, cdiv(2LL * sms, BH));
+  b->seg = static_cast<int>(std::max<long long>(16, cdiv(cdiv(std::max(N, 1), want), 16) * 16));
+  b->splits = static_cast<int>(std::max<long long>(1, cdiv(std::max(N, 1), b->seg)));
+  b->off_part = align256(p->bytes);
+  b->off_part_z = align256(b->off_part + static_cast<size_t>(BH) * b->splits * D * D * 4);
+  b->off_fin = align256(b->off_part_z + static_cast<size_t>(BH) * b->splits * D * 4);
+  b->off_fin_z = align256(b->off_fin + static_cast<size_t>(BH) * D * D * 4);
+  b->bytes = align256(b->off_fin_z + static_cast<size_t>(BH) * D * 4);
+  return b->bytes;
 }
 
 la_status_t check_backward(la_handle_t h, int B, int H, int N, int D, int fmap, float eps) {
@@ -560,8 +571,8 @@ size_t la_backward_workspace_bytes(la_handle_t h, int B, int H, int N, int D) {
   DeviceInfo di;
   const int sms = device_info(&di) ? di.sms : 148;
   Plan p;
-  size_t a, b;
-  return backward_plan(h, B, H, N, D, LA_PHI_ELU1, 0.f, sms, &p, &a, &b);
+  BwdLayout b;
+  return backward_plan(h, B, H, N, D, LA_PHI_ELU1, 0.f, sms, &p, &b);
 }
 
 la_status_t la_backward(la_handle_t h, const void* q, const void* k, const void* v, const void* dout, void* dq,
@@ -595,8 +606,8 @@ la_status_t la_backward(la_handle_t h, const void* q, const void* k, const void*
   if (!device_info(&di)) return LA_ERR_NO_DEVICE;
   if (di.major != 10 || di.minor != 0) return LA_ERR_NO_DEVICE;
   Plan p;
-  size_t off_bfin, off_bfin_z;
-  const size_t need = backward_plan(h, B, H, N, D, fmap, eps, di.sms, &p, &off_bfin, &off_bfin_z);
+  BwdLayout bl;
+  const size_t need = backward_plan(h, B, H, N, D, fmap, eps, di.sms, &p, &bl);
   if (!h->ws || h->ws_bytes < need) return LA_ERR_WORKSPACE;
   for (const void* x : ins)
     if (!la::on_current_device(x)) return LA_ERR_INVALID_ARG;
@@ -617,8 +628,10 @@ la_status_t la_backward(la_handle_t h, const void* q, const void* k, const void*
   a.ws = static_cast<char*>(h->ws);
   a.stream = cs;
   char* ws = static_cast<char*>(h->ws);
-  const cudaError_t err = la::launch_f32_backward(a, dout, dq, dk, dv, reinterpret_cast<float*>(ws + off_bfin),
-                                                  reinterpret_cast<float*>(ws + off_bfin_z));
+  const cudaError_t err = la::launch_f32_backward(
+      a, dout, dq, dk, dv, bl.splits, bl.seg, reinterpret_cast<float*>(ws + bl.off_part),
+      reinterpret_cast<float*>(ws + bl.off_part_z), reinterpret_cast<float*>(ws + bl.off_fin),
+      reinterpret_cast<float*>(ws + bl.off_fin_z));
   if (err == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
   if (err != cudaSuccess) {
     cudaGetLastError();

@@ -93,10 +93,12 @@ cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes);
 // f32 CUDA-core path (all modes).
 cudaError_t launch_f32(const LaunchArgs& a);
 // Backward of the fp32 non-causal layer (F = 0, elu+1 or relu): dq, dk, dv of
-// sum(out * dout); bfin / bfin_z: the workspace's [BH][D][D] and [BH][D]
-// regions past the forward plan.
-cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq, void* dk, void* dv, float* bfin,
-                                float* bfin_z);
+// sum(out * dout).  The query pass runs `splits` splits of `seg` tokens per
+// head; bpart / bpart_z: their [BH][splits][D][D] and [BH][splits][D]
+// partials, bfin / bfin_z: the [BH][D][D] and [BH][D] sums (workspace regions
+// past the forward plan).
+cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq, void* dk, void* dv, int splits,
+                                int seg, float* bpart, float* bpart_z, float* bfin, float* bfin_z);
 // bf16 tensor-core paths.
 // CTAs per head and cluster size of the bf16 non-causal kernel for p's shape
 // on the current device (from its cluster occupancy), and the bytes of the
