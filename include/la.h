@@ -70,7 +70,7 @@ typedef enum {
   LA_OK = 0,
   LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, eps < 0, bad enum,
                                an output overlapping an input                  */
-  LA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape/dtype this build runs   */
+  LA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape/dtype this library runs */
   LA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
   LA_ERR_WORKSPACE = 4,     /* no workspace bound, or it is too small         */
   LA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed    */
