@@ -113,7 +113,8 @@ la_status_t la_destroy(la_handle_t handle);
  * else LA_ERR_INVALID_ARG.  q_scale = NULL unbinds.
  * la_forward then requires the bound D and N <= n_positions
  * (LA_ERR_INVALID_ARG) and supports: LA_F32 with F = 0, causal or not;
- * LA_BF16 with D = 128, F = 0, non-causal, feature map elu+1 or relu.  Other
+ * LA_BF16 with F = 0 either at D = 128, non-causal, feature map elu+1 or relu
+ * (the tensor-core kernel) or on a shape that runs widened (see la_forward).  Other
  * forwards with a prologue bound (other shapes, la_forward_ttr,
  * la_forward_e4m3) return LA_ERR_UNSUPPORTED. */
 la_status_t la_set_prologue(la_handle_t handle, const float* q_scale, const float* k_scale, const float* rope,
@@ -134,7 +135,9 @@ la_status_t la_set_projection(la_handle_t handle, const void* W, int H, int D, i
  * (B*H) as SMs need the header only.  Otherwise the workspace holds fp32
  * partial states and grows with B*H and the number of splits per head: on
  * 148 SMs about 2 MB for causal [4, 8, 32768, 64], 11 MB for
- * [1, 24, 4608, 128] with F = 256, and 13.5 GB for B*H = 65535 with F = 256. */
+ * [1, 24, 4608, 128] with F = 256, and 13.5 GB for B*H = 65535 with F = 256.
+ * A bf16 shape that runs widened (see la_forward) needs the fp32 plan plus
+ * fp32 copies of q, k, v and out (16 * B*H*N*D bytes) and of W. */
 size_t la_workspace_bytes(la_handle_t handle, int B, int H, int N, int D, int F, int causal);
 
 /* Bind a caller-owned device workspace (256-byte aligned).  The library writes
@@ -147,12 +150,17 @@ la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
  * B, H, N >= 0 (any of them 0: nothing is enqueued, LA_OK); D > 0; F = 0 or a
  * positive multiple of 256 with a projection bound; feature_map is a
  * la_feature_map_t; eps >= 0; causal is 0 or 1.
- * Supported: LA_F32: D <= 128, D % 4 == 0, F in {0, 256}.
- *            LA_BF16: D in {64, 128}; F in {0, 256} with D = 128 when F > 0;
- *            causal with F = 0 and D = 64.
- *            LA_PHI_SOFTMAX: F = 0; on LA_BF16 non-causal with D = 128 only
- *            (also through la_forward_ttr and la_forward_noalloc; not
- *            la_forward_e4m3).  Other combinations: LA_ERR_UNSUPPORTED.
+ * Supported: D <= 128, D % 4 == 0, F in {0, 256}; LA_PHI_SOFTMAX with F = 0
+ *            only.  Other combinations: LA_ERR_UNSUPPORTED.
+ *            LA_BF16 runs on the tensor-core kernels for non-causal D = 64
+ *            or 128 (F = 256 with D = 128 only) and causal D = 64 with
+ *            F = 0 (also the shapes of la_forward_ttr and
+ *            la_forward_noalloc); of these, LA_PHI_SOFTMAX runs at
+ *            non-causal D = 128 only.  Any other LA_BF16 shape runs
+ *            widened: q, k, v (and W) are converted to fp32 copies
+ *            in the workspace on `stream`, the fp32 kernels run on them and
+ *            out is their result rounded to bf16 (four more launches, five
+ *            with W).
  * The result is deterministic: the same arguments give bitwise the same out. */
 la_status_t la_forward(la_handle_t handle, const void* q, const void* k, const void* v,
                        void* out, int B, int H, int N, int D, int F, int feature_map,

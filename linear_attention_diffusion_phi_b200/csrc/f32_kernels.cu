@@ -9,7 +9,10 @@
 // the state over the sequence: each segment's state is reduced, an exclusive
 // scan over segments gives every segment its starting state, and each segment
 // then walks its tokens in order (update with token i, then read row i).
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "la_internal.h"
 #include "sm100.cuh"
@@ -326,6 +329,18 @@ __global__ void __launch_bounds__(256) f32_causal_apply(const float* __restrict_
   }
 }
 
+// ------------------------------------------------- storage conversions
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ in, float* __restrict__ out, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    out[i] = __bfloat162float(in[i]);
+}
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    out[i] = __float2bfloat16_rn(in[i]);
+}
+
 // ------------------------------------------------------------ backward
 // Gradients of sum(out * dout), non-causal, no projection (features = D), for
 // a loss whose gradient with respect to out is dout (page "Flux2TTRTrainer",
@@ -559,6 +574,20 @@ cudaError_t launch_f32_backward(const LaunchArgs& a, const void* dout, void* dq,
   dim3 g3((p.N + kBwdRows - 1) / kBwdRows, static_cast<unsigned>(p.BH));
   f32_bwd_key<<<g3, 256, mat, a.stream>>>(k, v, bfin, bfin_z, static_cast<float*>(dk), static_cast<float*>(dv), p.N,
                                         p.D, p.fmap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_to_f32(const void* in, float* out, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096));
+  bf16_to_f32_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(in), out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096));
+  f32_to_bf16_kernel<<<blocks, 256, 0, stream>>>(in, static_cast<__nv_bfloat16*>(out), n);
   return cudaGetLastError();
 }
 

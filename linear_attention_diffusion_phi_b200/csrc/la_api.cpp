@@ -69,6 +69,17 @@ bool device_info(DeviceInfo* out) {
   return true;
 }
 
+// Whether the bf16 tensor-core kernels cover a shape: non-causal D = 64 or
+// 128 (projected only at D = 128, F = 256) and causal D = 64 without
+// projection.  Other valid bf16 shapes run widened on the fp32 kernels, so
+// the plan, and the workspace, depend on the shape alone.
+bool bf16_native(int D, int F, int causal) {
+  if (D != 64 && D != 128) return false;
+  if (F != 0 && (F != 256 || D != 128)) return false;
+  if (causal && (F != 0 || D != 64)) return false;
+  return true;
+}
+
 // Shape/dtype validation shared by la_workspace_bytes and la_forward.
 la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap, float eps,
                         int causal) {
@@ -78,17 +89,16 @@ la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F,
   if (causal != 0 && causal != 1) return LA_ERR_INVALID_ARG;
   if (F % 256 != 0) return LA_ERR_INVALID_ARG;   // feature_dim: a multiple of 256
   if (static_cast<long long>(B) * H > 65535) return LA_ERR_UNSUPPORTED;
-  if (h->dtype == LA_F32) {
+  // the fp32 kernels' range (bf16 shapes outside the bf16 kernels' run there,
+  // widened)
+  const bool native = h->dtype == LA_BF16 && bf16_native(D, F, causal);
+  if (!native) {
     if (D > 128 || D % 4 != 0) return LA_ERR_UNSUPPORTED;
     if (F != 0 && F != 256) return LA_ERR_UNSUPPORTED;
-  } else {
-    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
-    if (F != 0 && (F != 256 || D != 128)) return LA_ERR_UNSUPPORTED;
-    if (causal && (F != 0 || D != 64)) return LA_ERR_UNSUPPORTED;
   }
-  // softmax over each row's features: fp32 without a projection, and the
-  // bf16 non-causal D = 128 kernel
-  if (fmap == LA_PHI_SOFTMAX && (F != 0 || (h->dtype == LA_BF16 && (causal || D != 128)))) return LA_ERR_UNSUPPORTED;
+  // softmax over each row's features: no projection; among the bf16 kernels
+  // only the non-causal D = 128 one
+  if (fmap == LA_PHI_SOFTMAX && (F != 0 || (native && (causal || D != 128)))) return LA_ERR_UNSUPPORTED;
   return LA_OK;
 }
 
@@ -104,7 +114,8 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
   p->num_sms = num_sms > 0 ? num_sms : 148;
   const long long BH = std::max<long long>(p->BH, 1);
   size_t partial_floats = 0, ksum_floats = 0, final_bytes = 0, final_ksum_bytes = 0, blob_total = 0, xchg_bytes = 0;
-  if (h->dtype == LA_F32) {
+  p->widened = h->dtype == LA_BF16 && !bf16_native(D, F, causal);
+  if (h->dtype == LA_F32 || p->widened) {
     // Enough (head, split, feature-block) blocks for ~2 waves; splits of whole
     // 16-token chunks (non-causal) or >= 64 tokens (causal).
     const long long fblocks = cdiv(p->Fe, 32);
@@ -162,6 +173,18 @@ void make_plan(const la_handle_s* h, int B, int H, int N, int D, int F, int fmap
   p->off_final_ksum = off;    off = align256(off + final_ksum_bytes);
   p->off_blob = off;          off = align256(off + blob_total);
   p->off_xchg = off;          off = align256(off + xchg_bytes);
+  if (p->widened) {
+    // fp32 copies of q, k, v, out and W (W with its head stride)
+    const size_t n = static_cast<size_t>(BH) * std::max(N, 1) * D;
+    p->w_elems = F == 0 ? 0
+                        : (h->w_head_stride ? static_cast<size_t>(std::max(H, 1) - 1) * h->w_head_stride : 0) +
+                              static_cast<size_t>(D) * F;
+    p->off_wq = off;            off = align256(off + n * 4);
+    p->off_wk = off;            off = align256(off + n * 4);
+    p->off_wv = off;            off = align256(off + n * 4);
+    p->off_wo = off;            off = align256(off + n * 4);
+    p->off_wW = off;            off = align256(off + p->w_elems * 4);
+  }
   p->bytes = off;
 }
 
@@ -415,7 +438,8 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   if (pro) {
     if (h->pro_D != D || N > h->pro_npos) return LA_ERR_INVALID_ARG;
     const bool fits = F == 0 && !gate && !scales &&
-                      (h->dtype == LA_F32 || (D == 128 && !causal && fmap != LA_PHI_SOFTMAX));
+                      (h->dtype == LA_F32 || !bf16_native(D, F, causal) ||
+                       (D == 128 && !causal && fmap != LA_PHI_SOFTMAX));
     if (!fits) return LA_ERR_UNSUPPORTED;
   }
   // The kernels write out and the workspace while q, k, v and W are still
@@ -448,6 +472,7 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   if (di.major != 10 || di.minor != 0) return LA_ERR_NO_DEVICE;   // kernels are built for sm_100a
   Plan p;
   make_plan(h, B, H, N, D, F, fmap, eps, causal, di.sms, &p);
+  if (p.widened && (gate || scales)) return LA_ERR_UNSUPPORTED;
   if (!h->ws || h->ws_bytes < p.bytes) return LA_ERR_WORKSPACE;
   if (!la::on_current_device(q) || !la::on_current_device(k) || !la::on_current_device(v) ||
       !la::on_current_device(out) || !la::on_current_device(h->ws) || (F > 0 && !la::on_current_device(h->W)))
@@ -480,6 +505,25 @@ la_status_t forward_impl(la_handle_t h, const void* q, const void* k, const void
   cudaError_t err;
   if (h->dtype == LA_F32) {
     err = la::launch_f32(a);
+  } else if (p.widened) {
+    // widen q, k, v (and W) into the workspace, run the fp32 kernels there
+    // and round their output back to bf16
+    const size_t n = static_cast<size_t>(B) * H * N * D;
+    float* wq = reinterpret_cast<float*>(a.ws + p.off_wq);
+    float* wk = reinterpret_cast<float*>(a.ws + p.off_wk);
+    float* wv = reinterpret_cast<float*>(a.ws + p.off_wv);
+    float* wo = reinterpret_cast<float*>(a.ws + p.off_wo);
+    float* wW = reinterpret_cast<float*>(a.ws + p.off_wW);
+    err = la::launch_bf16_to_f32(q, wq, n, cs);
+    if (err == cudaSuccess) err = la::launch_bf16_to_f32(k, wk, n, cs);
+    if (err == cudaSuccess) err = la::launch_bf16_to_f32(v, wv, n, cs);
+    if (err == cudaSuccess && F > 0) err = la::launch_bf16_to_f32(h->W, wW, p.w_elems, cs);
+    if (err == cudaSuccess) {
+      a.q = wq; a.k = wk; a.v = wv; a.out = wo;
+      a.W = F ? wW : nullptr;
+      err = la::launch_f32(a);
+    }
+    if (err == cudaSuccess) err = la::launch_f32_to_bf16(wo, out, n, cs);
   } else {
     CUtensorMap tq, tk, tv, to, tw;
     const long long BH = p.BH;

@@ -42,6 +42,11 @@ struct Plan {
   // workspace layout (byte offsets from the workspace base, 256-aligned)
   size_t off_status, off_sync, off_partial, off_ksum_partial, off_final, off_final_ksum, off_blob, off_xchg, bytes;
   size_t blob_bytes;   // bf16 [kv | ksum | 0]^T image per head (projected path)
+  // bf16 storage of a shape the bf16 kernels do not cover: q, k, v (and W) are
+  // widened to fp32 copies in the workspace, the fp32 kernels run on them, and
+  // their output is rounded back to bf16 (the plan is the fp32 one)
+  bool widened;
+  size_t off_wq, off_wk, off_wv, off_wo, off_wW, w_elems;
 };
 
 struct LaunchArgs {
@@ -92,6 +97,10 @@ cudaError_t ensure_smem_attr(const void* kernel, uint32_t bytes);
 
 // f32 CUDA-core path (all modes).
 cudaError_t launch_f32(const LaunchArgs& a);
+// Elementwise bf16 -> fp32 (exact) and fp32 -> bf16 (round to nearest even) of
+// n elements, on `stream`.
+cudaError_t launch_bf16_to_f32(const void* in, float* out, size_t n, cudaStream_t stream);
+cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t stream);
 // Backward of the fp32 non-causal layer (F = 0, elu+1 or relu): dq, dk, dv of
 // sum(out * dout).  The query pass runs `splits` splits of `seg` tokens per
 // head; bpart / bpart_z: their [BH][splits][D][D] and [BH][splits][D]

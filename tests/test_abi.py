@@ -74,6 +74,11 @@ def fwd(h, B=1, H=2, N=256, D=64, F=0, fmap=0, eps=1e-6, causal=0, ptr=0x1000, o
     return la.la_forward(h, ptr, ptr, ptr, out, B, H, N, D, F, fmap, eps, causal, None)
 
 
+# A call that passed every host check stops at the device: no sm_100 device
+# here, or no workspace bound on a B200.
+PAST_CHECKS = (7, 4)
+
+
 def test_forward_argument_validation(handles):
     f32, b16 = handles["f32"], handles["bf16"]
     # bad values
@@ -88,11 +93,15 @@ def test_forward_argument_validation(handles):
     # valid but not run by this build
     assert fwd(f32, D=130) == 2
     assert fwd(f32, D=6) == 2
-    assert fwd(b16, D=96) == 2
-    assert fwd(b16, D=64, F=256) == 2
+    assert fwd(b16, D=130) == 2
+    assert fwd(b16, D=6) == 2
     assert fwd(b16, D=128, F=512) == 2
-    assert fwd(b16, D=128, F=256, causal=1) == 2
-    assert fwd(b16, D=128, causal=1) == 2   # bf16 causal: D = 64 only
+    assert fwd(b16, D=64, F=256) == 1       # no projection bound
+    assert fwd(b16, D=128, F=256, causal=1) == 1
+    # bf16 shapes outside the tensor-core kernels run widened on the fp32 ones
+    assert fwd(b16, D=96) in PAST_CHECKS
+    assert fwd(b16, D=32, causal=1) in PAST_CHECKS
+    assert fwd(b16, D=128, causal=1) in PAST_CHECKS
     assert fwd(f32, B=300, H=300) == 2      # B*H beyond the grid limit
     # empty problems are a no-op
     assert fwd(f32, N=0, ptr=0, out=0) == 0
@@ -139,7 +148,7 @@ def test_projection_validation(handles):
     assert la.la_set_projection(h, 0x1000, 24, 128, 256, 100) == 1   # stride < D*F
     assert la.la_set_projection(h, 0x1008, 24, 128, 256, 0) == 3
     assert la.la_set_projection(h, 0x1000, 24, 128, 256, 128 * 256) == 0
-    assert fwd(h, D=64, F=256) == 2
+    assert fwd(h, D=64, F=256) == 1       # the bound W is 128 x 256
     # out may not overlap the part of W the call reads: heads 0..H-1 at the
     # bound stride, bf16 (two heads here: 2 * 128 * 256 * 2 bytes from 0x1000)
     wend = 0x1000 + 2 * 128 * 256 * 2
@@ -273,15 +282,18 @@ def test_e4m3_argument_checks_on_the_host(handles):
 
 
 def test_softmax_support_is_checked_on_the_host(handles):
-    """The softmax feature map runs on fp32 without a projection and on the
-    bf16 non-causal D = 128 kernel; every other combination is refused before
-    anything is enqueued."""
+    """The softmax feature map runs without a projection: on the bf16
+    non-causal D = 128 kernel and on the fp32 kernels (bf16 shapes outside
+    the tensor-core kernels widened); the other bf16 kernel shapes, a
+    projection and E4M3 inputs are refused before anything is enqueued."""
     SMX = la.LA_PHI_SOFTMAX
-    f = lambda h, D, F, causal: la.la_forward(h, 0x1000, 0x1000, 0x1000, 0x2000, 1, 2, 256, D, F, SMX, 1e-6,
+    f = lambda h, D, F, causal: la.la_forward(h, 0x1000, 0x1000, 0x1000, 0x4000_0000, 1, 2, 256, D, F, SMX, 1e-6,
                                               causal, None)
     assert f(handles["f32"], 64, 256, 0) == la.LA_ERR_UNSUPPORTED
-    assert f(handles["bf16"], 64, 0, 0) == la.LA_ERR_UNSUPPORTED
-    assert f(handles["bf16"], 128, 0, 1) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 64, 0, 0) == la.LA_ERR_UNSUPPORTED     # the bf16 D = 64 kernels
+    assert f(handles["bf16"], 64, 0, 1) == la.LA_ERR_UNSUPPORTED
+    assert f(handles["bf16"], 128, 0, 1) in PAST_CHECKS               # widened
+    assert f(handles["bf16"], 96, 0, 0) in PAST_CHECKS
     assert f(handles["bf16"], 128, 256, 0) == la.LA_ERR_UNSUPPORTED
     assert la.la_forward_e4m3(handles["bf16"], 0x1000, 0x1000, 0x1000, 1.0, 1.0, 1.0, 0x2000, 1, 2, 256, 128,
                               SMX, 1e-6, None) == la.LA_ERR_UNSUPPORTED
@@ -304,9 +316,9 @@ def test_prologue_binding_and_support_checks(handles):
     assert f(bf, rope=0x3004) == la.LA_ERR_MISALIGNED
     assert f(bf) == la.LA_OK
     fwd = lambda h, D=128, N=256, causal=0, fmap=la.LA_PHI_ELU1: la.la_forward(
-        h, 0x10000, 0x10000, 0x10000, 0x20000, 1, 2, N, D, 0, fmap, 1e-6, causal, None)
+        h, 0x10000, 0x10000, 0x10000, 0x4000_0000, 1, 2, N, D, 0, fmap, 1e-6, causal, None)
     assert fwd(bf, N=257) == la.LA_ERR_INVALID_ARG                 # more positions than the table
-    assert fwd(bf, causal=1, D=128) == la.LA_ERR_UNSUPPORTED
+    assert fwd(bf, causal=1, D=128) in PAST_CHECKS                # widened onto the fp32 kernels
     assert fwd(bf, fmap=la.LA_PHI_SOFTMAX) == la.LA_ERR_UNSUPPORTED
     assert la.la_forward_e4m3(bf, 0x10000, 0x10000, 0x10000, 1.0, 1.0, 1.0, 0x20000, 1, 2, 256, 128,
                               la.LA_PHI_ELU1, 1e-6, None) == la.LA_ERR_UNSUPPORTED

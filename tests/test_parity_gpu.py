@@ -681,6 +681,35 @@ def test_bf16_softmax_large_inputs():
     assert_parity(got, ref, "bf16")
 
 
+# ------------------------------------- bf16 shapes run widened on fp32 kernels
+
+WIDE_CASES = [
+    dict(D=128, causal=True, N=1000), dict(D=128, causal=True, N=129, fmap="relu", B=2, H=3),
+    dict(D=32, causal=True, N=300, fmap="relu"), dict(D=96, N=4607), dict(D=4, N=37, H=3),
+    dict(D=64, F=256, N=1000), dict(D=128, F=256, causal=True, N=777, fmap="relu"),
+    dict(D=128, causal=True, N=500, fmap="softmax"), dict(D=96, N=1, fmap="softmax"),
+]
+
+
+@pytest.mark.parametrize("case", WIDE_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_bf16_widened_shapes(case):
+    """bf16 shapes outside the tensor-core kernels (causal D != 64, a
+    projection at D != 128 or causal, D other than 64 and 128, causal softmax)
+    run on the fp32 kernels over on-device fp32 copies: every element against
+    the oracle, and bitwise the fp32 path's output on the widened inputs,
+    rounded to bf16 (same plan, same kernels)."""
+    import torch
+    case = dict(case)
+    B, H = case.pop("B", 1), case.pop("H", 2)
+    w = Workload("bf16wide", B=B, H=H, seed=2700 + case["N"], **case)
+    q, k, v, W = make_inputs(w)
+    got = run_gpu(w, q, k, v, W)
+    assert_parity(got, oracle_full(w, q, k, v, W), "bf16")
+    w32 = w.with_(dtype="f32")
+    ref32 = run_gpu(w32, q.float(), k.float(), v.float(), None if W is None else W.float())
+    assert torch.equal(got, ref32.to(torch.bfloat16))
+
+
 # ------------------------------------------------- Flux attention prologue --
 
 PRO_CASES = [
@@ -690,6 +719,7 @@ PRO_CASES = [
     dict(B=1, H=3, N=1000, D=128, fmap="relu"),
     dict(B=2, H=3, N=4607, D=128),
     dict(B=1, H=2, N=8000, D=128),      # heads over several clusters
+    dict(B=1, H=2, N=300, D=128, causal=True),   # bf16 widened onto the fp32 kernels
 ]
 
 
