@@ -150,10 +150,11 @@ la_status_t la_set_workspace(la_handle_t handle, void* dev_ptr, size_t bytes);
  * B, H, N >= 0 (any of them 0: nothing is enqueued, LA_OK); D > 0; F = 0 or a
  * positive multiple of 256 with a projection bound; feature_map is a
  * la_feature_map_t; eps >= 0; causal is 0 or 1.
- * Supported: D <= 128, D % 4 == 0, F in {0, 256}; LA_PHI_SOFTMAX with F = 0
- *            only.  Other combinations: LA_ERR_UNSUPPORTED.
+ * Supported: D <= 128, D % 4 == 0; F <= 4096 non-causal, F <= 256 causal;
+ *            LA_PHI_SOFTMAX with F = 0 only.  Other combinations:
+ *            LA_ERR_UNSUPPORTED.
  *            LA_BF16 runs on the tensor-core kernels for non-causal D = 64
- *            or 128 (F = 256 with D = 128 only) and causal D = 64 with
+ *            or 128 (F > 0: F = 256 with D = 128 only) and causal D = 64 with
  *            F = 0 (also the shapes of la_forward_ttr and
  *            la_forward_noalloc); of these, LA_PHI_SOFTMAX runs at
  *            non-causal D = 128 only.  Any other LA_BF16 shape runs

@@ -207,7 +207,8 @@ __global__ void f32_state_scan(float* __restrict__ part, float* __restrict__ par
   }
 }
 
-// out rows [blockIdx.x*16, +16) of head bh from the final state.
+// out rows [blockIdx.x*16, +16) of head bh from the final state, the
+// features taken in groups of kMaxFe (ascending; one group when Fe <= 256).
 __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, const float* __restrict__ W,
                                                  long long wstride, const float* __restrict__ fin,
                                                  const float* __restrict__ fin_ksum, float* __restrict__ out,
@@ -233,28 +234,51 @@ __global__ void __launch_bounds__(256) f32_apply(const float* __restrict__ q, co
     softmax_stats(Qs, D, Qst);
     __syncthreads();
   }
-  for (int e = threadIdx.x; e < kT * Fe; e += blockDim.x) {
-    const int t = e / Fe, f = e % Fe;
-    Ps[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f, fmap, Qst + 2 * t) : 0.f;
-  }
-  __syncthreads();
-  // den[t] = phi(q_t) . ksum + eps : one warp per two rows, lanes split f.
-  {
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int t = warp; t < kT; t += blockDim.x / 32) {
-      float acc = 0.f;
-      for (int f = lane; f < Fe; f += 32) acc = fmaf(Ps[t * kMaxFe + f], ksum[f], acc);
+  // Thread j of the block owns output elements e = j + 256 i (i < 8) of the
+  // kT x D tile; their numerators run over all feature groups in registers.
+  constexpr int kPer = kT * kMaxD / 256;
+  float num[kPer];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) den[t] = acc + eps;
+  for (int i = 0; i < kPer; ++i) num[i] = 0.f;
+  if (threadIdx.x < kT) den[threadIdx.x] = 0.f;
+  for (int f0 = 0; f0 < Fe; f0 += kMaxFe) {
+    const int fe = min(kMaxFe, Fe - f0);
+    for (int e = threadIdx.x; e < kT * fe; e += blockDim.x) {
+      const int t = e / fe, f = e % fe;
+      Ps[t * kMaxFe + f] = t < rows ? feature(Qs + t * kMaxD, D, Wh, F, f0 + f, fmap, Qst + 2 * t) : 0.f;
     }
+    __syncthreads();
+    // den[t] += phi(q_t) . ksum over the group: one warp per two rows, lanes split f.
+    {
+      const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+      for (int t = warp; t < kT; t += blockDim.x / 32) {
+        float acc = 0.f;
+        for (int f = lane; f < fe; f += 32) acc = fmaf(Ps[t * kMaxFe + f], ksum[f0 + f], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) den[t] += acc;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = threadIdx.x + 256 * i;
+      if (e < rows * D) {
+        const int t = e / D, d = e % D;
+        const float* kvf = kv + static_cast<size_t>(f0) * D + d;
+        float acc = num[i];
+        for (int f = 0; f < fe; ++f) acc = fmaf(Ps[t * kMaxFe + f], kvf[static_cast<size_t>(f) * D], acc);
+        num[i] = acc;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
-    const int t = e / D, d = e % D;
-    float num = 0.f;
-    for (int f = 0; f < Fe; ++f) num = fmaf(Ps[t * kMaxFe + f], kv[static_cast<size_t>(f) * D + d], num);
-    out[(static_cast<size_t>(bh) * N + t0 + t) * D + d] = num / den[t];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = threadIdx.x + 256 * i;
+    if (e < rows * D) {
+      const int t = e / D, d = e % D;
+      out[(static_cast<size_t>(bh) * N + t0 + t) * D + d] = num[i] / (den[t] + eps);
+    }
   }
 }
 

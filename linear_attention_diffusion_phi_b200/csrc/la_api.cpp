@@ -93,8 +93,10 @@ la_status_t check_shape(const la_handle_s* h, int B, int H, int N, int D, int F,
   // widened)
   const bool native = h->dtype == LA_BF16 && bf16_native(D, F, causal);
   if (!native) {
+    // fp32 kernels: features in groups of 256 (non-causal, up to 4096); the
+    // causal state of 256 features x D fills the shared memory
     if (D > 128 || D % 4 != 0) return LA_ERR_UNSUPPORTED;
-    if (F != 0 && F != 256) return LA_ERR_UNSUPPORTED;
+    if (F > 4096 || (causal && F > 256)) return LA_ERR_UNSUPPORTED;
   }
   // softmax over each row's features: no projection; among the bf16 kernels
   // only the non-causal D = 128 one

@@ -95,7 +95,10 @@ def test_forward_argument_validation(handles):
     assert fwd(f32, D=6) == 2
     assert fwd(b16, D=130) == 2
     assert fwd(b16, D=6) == 2
-    assert fwd(b16, D=128, F=512) == 2
+    assert fwd(b16, D=128, F=512) == 1      # no projection bound (widened when bound)
+    assert fwd(f32, D=64, F=512, causal=1) == 2   # causal: F <= 256
+    assert fwd(b16, D=128, F=512, causal=1) == 2
+    assert fwd(f32, D=64, F=4352) == 2      # non-causal: F <= 4096
     assert fwd(b16, D=64, F=256) == 1       # no projection bound
     assert fwd(b16, D=128, F=256, causal=1) == 1
     # bf16 shapes outside the tensor-core kernels run widened on the fp32 ones

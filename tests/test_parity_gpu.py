@@ -99,6 +99,7 @@ F32_CASES = [
     dict(N=129, D=64, causal=True), dict(N=700, D=128, causal=True, fmap="relu"),
     dict(N=200, D=128, F=256), dict(N=333, D=64, F=256, causal=True),
     dict(N=257, D=64, fmap="softmax"), dict(N=300, D=128, causal=True, fmap="softmax"),
+    dict(N=300, D=64, F=512), dict(N=77, D=128, F=768, fmap="relu"),   # several feature groups
 ]
 
 
@@ -688,6 +689,7 @@ WIDE_CASES = [
     dict(D=32, causal=True, N=300, fmap="relu"), dict(D=96, N=4607), dict(D=4, N=37, H=3),
     dict(D=64, F=256, N=1000), dict(D=128, F=256, causal=True, N=777, fmap="relu"),
     dict(D=128, causal=True, N=500, fmap="softmax"), dict(D=96, N=1, fmap="softmax"),
+    dict(D=128, F=512, N=1000),
 ]
 
 
