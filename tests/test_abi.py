@@ -188,6 +188,29 @@ def test_workspace_bytes_and_binding(handles):
     assert la.la_sync_status(h, None) == 4                    # no workspace bound
 
 
+def test_widened_workspace_holds_the_fp32_plan_and_copies(handles):
+    """A bf16 shape outside the tensor-core kernels runs on the fp32 kernels:
+    its workspace is the fp32 plan of the same shape plus fp32 copies of q, k,
+    v and out and of the part of W the call reads, each 256-byte aligned."""
+    f32, b16 = handles["f32"], handles["bf16"]
+    a256 = lambda x: (x + 255) // 256 * 256
+    shapes = [(1, 2, 1000, 128, 0, 1), (2, 3, 77, 96, 0, 0), (1, 2, 300, 32, 0, 1), (1, 24, 4608, 64, 256, 0),
+              (1, 2, 1000, 128, 512, 0), (1, 3, 5, 4, 256, 1)]
+    for B, H, N, D, F, causal in shapes:
+        n = B * H * N * D
+        got = la.la_workspace_bytes(b16, B, H, N, D, F, causal)
+        assert got == la.la_workspace_bytes(f32, B, H, N, D, F, causal) + 4 * a256(4 * n) + a256(4 * D * F), \
+            (B, H, N, D, F, causal)
+    # W bound with a head stride: heads 0 .. H - 1 are copied
+    assert la.la_set_projection(b16, 0x1000, 24, 64, 256, 64 * 256 + 64) == 0
+    n = 24 * 4608 * 64
+    assert la.la_workspace_bytes(b16, 1, 24, 4608, 64, 256, 0) == (
+        la.la_workspace_bytes(f32, 1, 24, 4608, 64, 256, 0) + 4 * a256(4 * n) + a256(4 * (23 * (64 * 256 + 64) + 64 * 256)))
+    assert la.la_set_projection(b16, None, 0, 0, 0, 0) == 0
+    # shapes the tensor-core kernels run keep their own plans, without copies
+    assert la.la_workspace_bytes(b16, 1, 24, 4608, 128, 256, 0) < 4 * 24 * 4608 * 128
+
+
 def test_no_device_is_reported_not_faked(handles):
     torch = pytest.importorskip("torch")
     if torch.cuda.is_available():
